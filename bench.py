@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Throughput of the batched Dion optimizer step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one dion_step_batched call over every weight matrix of the workload
+(default: 7B-like transformer, 32 layers, hidden 4096, MLP 11008, rank 256 = 1/16,
+bf16-input GEMMs, fp32 state; 224 matrices, 6.476e9 parameters).  Inputs are
+synthetic and already resident in HBM when the timed region starts; they are far
+larger than L2 (126 MB), so no L2 flush is needed between steps.
+
+Prints one JSON line (rank 0).  Under torchrun every rank updates its own full set of
+matrices (weak scaling, no collective on the data path); the step time is the max over
+ranks of the device-timed region.
+
+``--impl reference`` times the fp64 CPU oracle instead, on a bounded sample of the same
+workload (one matrix per shape bucket per step), extrapolated to the whole workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "params updated/s (Dion steps/s) at 7B shapes; % of roofline"
+UNIT = "params/s"
+
+
+# ------------------------------------------------------------ distributed plumbing
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def dist_setup(backend: str):
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and str(device).startswith("cuda"):
+            dist.barrier(device_ids=[int(str(device).split(":")[1])])
+        else:
+            dist.barrier()
+
+
+def whole_job_rate(units_per_rank: float, world: int, seconds_max: float) -> float:
+    """Units processed by all ranks divided by the slowest rank's time."""
+    return units_per_rank * world / seconds_max
+
+
+# ------------------------------------------------------------------ clocks sampler
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clocks not sampled"]}
+        sm = [float(r[1]) for r in rows]
+        smax = max(float(r[2]) for r in rows)
+        loaded = [s for s, r in zip(sm, rows) if float(r[3]) > 200.0] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows)}
+
+
+# ------------------------------------------------------------------ roofline figures
+def algorithmic(wl: W.Workload):
+    """Per step: flops of the four rank-r contractions + Cholesky-QR, and the bytes the
+    method must move (32 B per weight element: three dependent sweeps over B, plus the
+    r-sized factors); and the bytes of the fused update alone (20 B per element)."""
+    flops = sum(b.count * (8 * b.m * b.n * b.r + 3 * b.m * b.r ** 2 + b.r ** 3 / 3)
+                for b in wl.buckets)
+    bytes_ = sum(b.count * (32 * b.m * b.n + 4 * (3 * b.m * b.r + 6 * b.n * b.r))
+                 for b in wl.buckets)
+    update_bytes = sum(b.count * 20 * b.m * b.n for b in wl.buckets)
+    return flops, bytes_, update_bytes
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def update_traffic():
+    """DRAM bytes per element of the fused update from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", "update_traffic.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("dram_bytes_per_element"), d.get("kernel_source_hash")
+    return None, None
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rank_orthonormalized_optimizer_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_sample(wl: W.Workload, steps: int, budget_s: float = 20.0):
+    """Time the fp64 oracle on one matrix per bucket; returns (params/s, seconds, cores, note)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 0) for i in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        cores = os.cpu_count()
+    per_bucket = []
+    spent = 0.0
+    for bi, b in enumerate(wl.buckets):
+        X = W.weights(wl, bi, "cpu", slots=[0])[0].double().numpy()
+        M = W.momentum(wl, bi, "cpu", slots=[0])[0].double().numpy()
+        Q = W.right_factor(wl, bi, "cpu", slots=[0])[0].double().numpy()
+        G = W.gradient(wl, bi, 0, "cpu", slots=[0])[0].double().numpy()
+        times = []
+        for _ in range(max(1, steps)):
+            t0 = time.perf_counter()
+            X, M, Q, _, _ = oracle.dion_step(X, M, G, Q, wl.mu, wl.lr)
+            times.append(time.perf_counter() - t0)
+            spent += times[-1]
+            if spent > budget_s:
+                break
+        per_bucket.append(statistics.median(times))
+    step_s = sum(b.count * t for b, t in zip(wl.buckets, per_bucket))
+    note = (f"fp64 NumPy oracle, one matrix per bucket "
+            f"({', '.join(f'{b.m}x{b.n}' for b in wl.buckets)}), median of up to {steps} steps each, "
+            f"scaled by bucket counts ({', '.join(str(b.count) for b in wl.buckets)}) to the full "
+            f"{wl.params:.4g}-parameter step ({step_s:.1f} s extrapolated)")
+    return wl.params / step_s, step_s, cores, note
+
+
+# ------------------------------------------------------------------ the GPU arm
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    rank, world = dist_setup("nccl")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from rank_orthonormalized_optimizer_b200 import DionB200
+
+    wl = W.WORKLOADS[args.workload]
+    opt = DionB200([(b.count, b.m, b.n, b.r) for b in wl.buckets], mu=wl.mu,
+                   precision=wl.precision, kernel_path=args.kernel_path)
+    nb = len(wl.buckets)
+    X = [W.weights(wl, i, dev) for i in range(nb)]
+    M = [W.momentum(wl, i, dev) for i in range(nb)]
+    Q = [W.right_factor(wl, i, dev) for i in range(nb)]
+    G = [W.gradient(wl, i, 0, dev) for i in range(nb)]
+    ws = opt.alloc_workspace(dev)
+    status = opt.alloc_status(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        opt.step(X, M, G, Q, wl.lr, ws, status, stream)
+    torch.cuda.synchronize(dev)
+
+    # timed region: K steps, barrier + sync on both sides, device events
+    opt.profile_enable(True)
+    launches = 0
+    with Clocks(local) as clk:
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            opt.step(X, M, G, Q, wl.lr, ws, status, stream)
+            launches += opt.last_launch_count
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+    clocks = clk.summary()
+    ms_local = t0.elapsed_time(t1) / args.steps
+    prof = opt.profile_read()
+    opt.profile_enable(False)
+    ms = max_over_ranks(ms_local, dev)
+    st = status.cpu()
+
+    value = whole_job_rate(wl.params, world, ms / 1e3)
+    flops, bytes_alg, upd_bytes = algorithmic(wl)
+    peaks = measured_peaks()
+    upd_ms = prof["update"][0] / args.steps
+    upd_launches = prof["update"][1] / args.steps
+    achieved = upd_bytes / (upd_ms / 1e3) / 1e9
+    traffic_per_elem, traffic_hash = update_traffic()
+    traffic = None
+    if traffic_per_elem is not None and traffic_hash == kernel_source_hash():
+        traffic = traffic_per_elem * sum(b.params for b in wl.buckets) / max(upd_launches, 1)
+    roof_t = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_alg / (peaks["hbm_gbs"] * 1e9))
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "steps_per_s": 1e3 / ms * 1.0,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.precision == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "matrices": sum(b.count for b in wl.buckets),
+                   "params_per_gpu": wl.params,
+                   "buckets": [[b.count, b.m, b.n, b.r] for b in wl.buckets],
+                   "state": "fp32 X, M, G, Q", "gemm_inputs": wl.precision,
+                   "kernel_path": args.kernel_path,
+                   "parallelism": f"matrix-partitioned x{world} (each rank its own matrices)",
+                   "l2": "inputs (78 GB) far larger than L2; no flush"},
+        "roofline": {"bound": "hbm", "kernel": "fused update (M and X)",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "peak_source": peaks["source"],
+                     "per_step_ms": upd_ms, "algorithmic_bytes_per_step": upd_bytes},
+        "step_roofline": {"t_roofline_ms": roof_t * 1e3, "frac": roof_t * 1e3 / ms,
+                          "flops": flops, "bytes": bytes_alg},
+        "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items()},
+        "gpu_launches": launches,
+        "status_bits": int(np.bitwise_or.reduce(st.numpy())) if st.numel() else 0,
+        "clocks": clocks,
+    }
+
+    # end to end through the C ABI with the gradients in pinned host memory
+    if not args.no_e2e:
+        Gh = []
+        for g in G:
+            h = torch.empty(g.shape, dtype=g.dtype, pin_memory=True)
+            h.copy_(g)
+            Gh.append(h)
+        hs = torch.zeros(opt.num_matrices, dtype=torch.int32).pin_memory()
+        opt.step_from_host(X, M, G, Q, Gh, wl.lr, ws, status, hs, stream)
+        barrier(dev)
+        t_start = time.perf_counter()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            opt.step_from_host(X, M, G, Q, Gh, wl.lr, ws, status, hs, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
+        result["e2e"] = {"value": whole_job_rate(wl.params, world, e2e_ms / 1e3), "unit": UNIT,
+                         "h2d_bytes_per_step": sum(g.numel() * 4 for g in Gh),
+                         "d2h_bytes_per_step": hs.numel() * 4, "ms_per_step": e2e_ms,
+                         "steps": args.e2e_steps,
+                         "note": "gradients uploaded from pinned host memory and the per-matrix "
+                                 "status read back every step (dion_step_batched_from_host)"}
+        del Gh
+        _ = time.perf_counter() - t_start
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, step_s, cores, note = oracle_sample(wl, steps=2)
+        result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                  "sample": note}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    opt.close()
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ the oracle arm
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        oracle_sample(wl, steps=1, budget_s=5.0)
+    t0 = time.perf_counter()
+    vals = []
+    cores = note = None
+    for _ in range(args.steps):
+        v, step_s, cores, note = oracle_sample(wl, steps=1, budget_s=10.0)
+        vals.append(step_s)
+    wall = time.perf_counter() - t0
+    step_s = statistics.median(vals)
+    value = wl.params / step_s
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": wl.name, "params": wl.params},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": note},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": wall}), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=W.HEADLINE, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--kernel-path", default="tensor", choices=["tensor", "simt"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

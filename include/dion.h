@@ -1,0 +1,221 @@
+/*
+ * dion.h -- C ABI of the batched Dion optimizer step on NVIDIA B200 (sm_100a).
+ *
+ * One call updates every 2-D weight matrix of a model.  For a weight X
+ * (m x n, row-major fp32), its error-feedback momentum M (m x n), its
+ * gradient G (m x n) and the right factor Q (n x r) kept between steps:
+ *
+ *   B  = M + G
+ *   P  = orth(B Q)             Cholesky-QR, Householder QR when ill-conditioned
+ *   R  = B^T P
+ *   M <- B - (1 - mu) P R^T    error feedback
+ *   Q <- colnorm(R)            unit columns (a zero column stays zero)
+ *   X <- X - lr * s * P Q^T    s = sqrt(m / n) unless given
+ *
+ * Sources: rivista.ai, "Dion e la fine del monopolio di Adam negli optimizer
+ * AI distribuiti" (the article on "Dion: Distributed Orthonormalized
+ * Updates"): paragraph 2 (only the top-r singular directions are
+ * orthonormalised), paragraph 3 (error feedback re-injects what the low-rank
+ * update missed), paragraph 5 (amortised power iteration with QR and Cholesky
+ * decompositions; 2-D parameters only, biases and 1-D weights go elsewhere).
+ * Matrices of one shape are stacked into a [count, m, n] tensor and processed
+ * together, as "DASH: Faster Shampoo via Batched Block Preconditioning and
+ * Efficient Inverse-Root Solvers" (Methodologie, section 1) stacks blocks.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named d_* / in dion_bucket_ptrs are DEVICE pointers on the
+ *    handle's device; all others are host pointers.
+ *  - The caller owns every buffer (weights, state, gradients, workspace,
+ *    status) and the stream.  The library never allocates or frees device
+ *    memory and never synchronises the device, except where stated.
+ *  - Errors in arguments are returned synchronously as a dion_status and
+ *    leave every buffer untouched; dion_last_error() then gives a message.
+ *    Numerical events are reported per matrix in the device status array.
+ *  - No C++ exception crosses this interface.  A handle must not be used
+ *    from two threads or two streams at the same time.
+ */
+#ifndef DION_H
+#define DION_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct dion_ctx* dion_handle;
+
+/* Host-side return codes. */
+typedef enum dion_status {
+  DION_OK = 0,
+  DION_ERR_INVALID_ARG = 1,         /* null pointer, bad count, bad option value  */
+  DION_ERR_UNSUPPORTED_SHAPE = 2,   /* shape outside the supported set (see dion_init) */
+  DION_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace smaller than dion_init reported  */
+  DION_ERR_CUDA = 4,                /* a CUDA runtime call failed (message says which) */
+  DION_ERR_NOT_INITIALIZED = 5,     /* null or freed handle                       */
+  DION_ERR_DEVICE = 6,              /* current device is not sm_100 (B200)       */
+  DION_ERR_MISALIGNED = 7           /* a device pointer is not 16-byte aligned    */
+} dion_status;
+
+/* Per-matrix status bits written to d_status[] by every step (OR-ed). */
+enum {
+  DION_MAT_OK = 0,
+  DION_MAT_FALLBACK = 1,      /* Cholesky-QR rejected; Householder QR produced P        */
+  DION_MAT_CHOLQR2 = 2,       /* a second Cholesky-QR pass was applied                   */
+  DION_MAT_NONFINITE = 4,     /* a Gram matrix held Inf/NaN (inputs were not finite)     */
+  DION_MAT_TIMEOUT = 8,       /* a bounded device wait ran out; this matrix's outputs
+                                 are not valid and X, M, Q may be partly updated         */
+  DION_MAT_ZERO_COLUMN = 16   /* some column of R had zero norm; its Q column is zero    */
+};
+
+/* Arithmetic of the four rank-r contractions (B Q, B^T P, P R^T, P Q^T). */
+typedef enum dion_precision {
+  DION_PREC_FP32 = 0,  /* fp32 operands, fp32 accumulation                           */
+  DION_PREC_BF16 = 1   /* B, Q, P, R rounded to bf16 (round to nearest even), fp32
+                          accumulation; Gram, Cholesky and the triangular apply stay
+                          fp32                                                       */
+} dion_precision;
+
+/* How P = orth(B Q) is formed. */
+typedef enum dion_orth_mode {
+  DION_ORTH_AUTO = 0,        /* Cholesky-QR; a second pass when max|P^T P - I| > orth_tol;
+                                Householder when a pivot fails or the Cholesky diagonal
+                                ratio exceeds fallback_cond                              */
+  DION_ORTH_CHOLQR = 1,      /* one Cholesky-QR pass (+ Householder fallback)            */
+  DION_ORTH_CHOLQR2 = 2,     /* always two passes (+ Householder fallback)               */
+  DION_ORTH_HOUSEHOLDER = 3  /* Householder QR for every matrix                          */
+} dion_orth_mode;
+
+/* Which kernels run the contractions. */
+typedef enum dion_kernel_path {
+  DION_PATH_TENSOR = 0,  /* tcgen05 tensor-core kernels fed by TMA where the precision
+                            and shape allow; the SIMT kernels elsewhere               */
+  DION_PATH_SIMT = 1     /* CUDA-core kernels everywhere (a cross-check)               */
+} dion_kernel_path;
+
+/* One bucket: `count` matrices of identical shape (m, n), updated at rank r. */
+typedef struct dion_bucket_desc {
+  int64_t m, n, r;
+  int32_t count;
+  float scale;     /* s in X -= lr*s*P Q^T; <= 0 selects sqrt(m / n) */
+} dion_bucket_desc;
+
+typedef struct dion_options {
+  float mu;                /* error-feedback decay, 0 <= mu < 1 (default 0.95)            */
+  int32_t precision;       /* dion_precision (default DION_PREC_BF16)                      */
+  int32_t orth_mode;       /* dion_orth_mode (default DION_ORTH_AUTO)                      */
+  float fallback_cond;     /* Householder when max L_kk / min L_kk exceeds it (1e3)        */
+  float orth_tol;          /* AUTO: second pass when max|P^T P - I| > orth_tol (2e-5)      */
+  int32_t kernel_path;     /* dion_kernel_path (default DION_PATH_TENSOR)                  */
+  int64_t max_wait_spins;  /* bound on every device-side wait; when it runs out the
+                              kernel sets DION_MAT_TIMEOUT and returns (default 1<<26)     */
+} dion_options;
+
+/* Device buffers of one bucket, all contiguous, row-major, 16-byte aligned:
+ *   X, M, G : fp32 [count, m, n]     X and M updated in place, G read only
+ *   Q       : fp32 [count, n, r]     read (previous factor) and overwritten
+ * Q must hold unit-norm columns before the first step (any such Q). */
+typedef struct dion_bucket_ptrs {
+  float* X;
+  float* M;
+  const float* G;
+  float* Q;
+} dion_bucket_ptrs;
+
+/* Fill *opt with the defaults listed above. */
+dion_status dion_default_options(dion_options* opt);
+
+/*
+ * Plan a step over `nbuckets` buckets (host only; touches no device).
+ * Supported shapes: count >= 1, 1 <= r <= min(m, n), r % 16 == 0, n % 8 == 0,
+ * m >= 1, and every buffer below 2^40 elements; otherwise
+ * DION_ERR_UNSUPPORTED_SHAPE.  opt may be NULL (defaults).
+ * On success *out receives a handle (host memory owned by the library until
+ * dion_free) and *workspace_bytes the size of the device workspace that
+ * every dion_step_batched call must be given.
+ */
+dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets,
+                      const dion_options* opt, dion_handle* out,
+                      size_t* workspace_bytes);
+
+/*
+ * One Dion step over every bucket, enqueued on `stream` (a cudaStream_t; NULL
+ * is the legacy default stream) of the current device.  Returns as soon as
+ * the work is enqueued.
+ *   ptrs        host array of nbuckets device-pointer sets, in the order the
+ *               buckets were given to dion_init
+ *   lr          learning rate eta of this step
+ *   d_workspace device scratch of at least *workspace_bytes from dion_init,
+ *               16-byte aligned; its contents need not be preserved between
+ *               calls, and it must not be shared by two steps in flight
+ *   d_status    device int32 array, one word per matrix (bucket by bucket,
+ *               slot by slot), overwritten with DION_MAT_* bits; may be NULL
+ * Within a bucket the matrices are independent.  X, M and Q are written only
+ * by the last kernels of the step.
+ */
+dion_status dion_step_batched(dion_handle h, const dion_bucket_ptrs* ptrs,
+                              int32_t nbuckets, float lr, void* d_workspace,
+                              size_t workspace_bytes, int32_t* d_status, void* stream);
+
+/*
+ * The same step with the gradients coming from HOST memory: copies
+ * host_grads[b] (fp32 [count, m, n], pinned for asynchronous copies) into the
+ * device buffer ptrs[b].G (which this call therefore overwrites), runs the
+ * step, copies d_status back to host_status (one int32 per matrix), and
+ * synchronises `stream` before returning, so host_status is valid on return.
+ */
+dion_status dion_step_batched_from_host(dion_handle h, const dion_bucket_ptrs* ptrs,
+                                        const float* const* host_grads, int32_t nbuckets,
+                                        float lr, void* d_workspace, size_t workspace_bytes,
+                                        int32_t* d_status, int32_t* host_status,
+                                        void* stream);
+
+/* Release the handle (host memory only).  NULL is accepted. */
+dion_status dion_free(dion_handle h);
+
+/* Static text for a status code. */
+const char* dion_status_string(dion_status s);
+
+/* Message of the last error raised on this thread ("" if none). */
+const char* dion_last_error(void);
+
+/* Total number of matrices over all buckets (the length of d_status). */
+int64_t dion_num_matrices(dion_handle h);
+
+/* Kernel launches made by the most recent dion_step_batched call (0 before). */
+int32_t dion_last_launch_count(dion_handle h);
+
+/* Intermediates of the most recent step, for inspection after the stream has
+ * been synchronised: which = DION_VIEW_P gives P (fp32 [count, m, r]),
+ * DION_VIEW_R gives R (fp32 [count, n, r]).  *d_ptr points into d_workspace. */
+enum { DION_VIEW_P = 0, DION_VIEW_R = 1 };
+dion_status dion_workspace_view(dion_handle h, int32_t bucket, int32_t which,
+                                void* d_workspace, void** d_ptr, size_t* bytes);
+
+/*
+ * Per-kernel timing with CUDA events recorded on the step's stream.
+ * dion_profile_enable(h, 1) starts recording around every kernel class of
+ * every later step (and clears the totals); dion_profile_read synchronises
+ * the recorded events and returns, per class, the summed milliseconds and
+ * the number of launches.  Classes are numbered as DION_KCLASS_*.
+ */
+enum {
+  DION_KCLASS_FORM_B = 0,   /* B = M + G in GEMM precision                */
+  DION_KCLASS_PREP_Q = 1,   /* previous Q into GEMM layout               */
+  DION_KCLASS_GEMM_BQ = 2,  /* P0 = B Q                                  */
+  DION_KCLASS_ORTH = 3,     /* Gram, Cholesky, inverse, apply, fallback  */
+  DION_KCLASS_GEMM_BTP = 4, /* R = B^T P                                 */
+  DION_KCLASS_COLNORM = 5,  /* Q = colnorm(R) and the update operands     */
+  DION_KCLASS_UPDATE = 6,   /* fused M and X update                      */
+  DION_KCLASS_COUNT = 7
+};
+dion_status dion_profile_enable(dion_handle h, int32_t on);
+dion_status dion_profile_read(dion_handle h, double* ms, int64_t* launches,
+                              int32_t nclasses);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DION_H */

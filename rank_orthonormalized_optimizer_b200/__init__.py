@@ -1,0 +1,243 @@
+"""Batched Dion optimizer step on NVIDIA B200 (sm_100a): Python binding.
+
+The arithmetic runs in the CUDA library ``lib/libdion_b200.so`` behind the C ABI
+of ``include/dion.h``; this module only marshals arguments (torch tensors to
+device pointers and the current CUDA stream).  PyTorch provides device memory
+and streams.  There is no CPU implementation: importing this module fails if
+the library has not been built (``python -m rank_orthonormalized_optimizer_b200.build``).
+
+One step, for every matrix of every bucket (see include/dion.h):
+    B = M + G;  P = orth(B Q);  R = B^T P;  M <- B - (1 - mu) P R^T;
+    Q <- colnorm(R);  X <- X - lr * s * P Q^T,  s = sqrt(m / n)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libdion_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build the CUDA library first with "
+        "`python -m rank_orthonormalized_optimizer_b200.build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+c_int32, c_int64, c_float, c_void_p, c_size_t = (ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                                                 ctypes.c_void_p, ctypes.c_size_t)
+
+# status codes and bits, mirrored from include/dion.h
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_WORKSPACE_TOO_SMALL, ERR_CUDA, \
+    ERR_NOT_INITIALIZED, ERR_DEVICE, ERR_MISALIGNED = range(8)
+MAT_OK, MAT_FALLBACK, MAT_CHOLQR2, MAT_NONFINITE, MAT_TIMEOUT, MAT_ZERO_COLUMN = 0, 1, 2, 4, 8, 16
+PRECISIONS = {"fp32": 0, "bf16": 1}
+ORTH_MODES = {"auto": 0, "cholqr": 1, "cholqr2": 2, "householder": 3}
+KERNEL_PATHS = {"tensor": 0, "simt": 1}
+KERNEL_CLASSES = ["form_b", "prep_q", "gemm_bq", "orth", "gemm_btp", "colnorm", "update"]
+VIEW_P, VIEW_R = 0, 1
+
+
+class BucketDesc(ctypes.Structure):
+    _fields_ = [("m", c_int64), ("n", c_int64), ("r", c_int64), ("count", c_int32),
+                ("scale", c_float)]
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("mu", c_float), ("precision", c_int32), ("orth_mode", c_int32),
+                ("fallback_cond", c_float), ("orth_tol", c_float), ("kernel_path", c_int32),
+                ("max_wait_spins", c_int64)]
+
+
+class BucketPtrs(ctypes.Structure):
+    _fields_ = [("X", c_void_p), ("M", c_void_p), ("G", c_void_p), ("Q", c_void_p)]
+
+
+def _sig(name, restype, *args):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = list(args)
+    return f
+
+
+dion_default_options = _sig("dion_default_options", c_int32, ctypes.POINTER(Options))
+dion_init = _sig("dion_init", c_int32, ctypes.POINTER(BucketDesc), c_int32,
+                 ctypes.POINTER(Options), ctypes.POINTER(c_void_p), ctypes.POINTER(c_size_t))
+dion_step_batched = _sig("dion_step_batched", c_int32, c_void_p, ctypes.POINTER(BucketPtrs),
+                         c_int32, c_float, c_void_p, c_size_t, c_void_p, c_void_p)
+dion_step_batched_from_host = _sig("dion_step_batched_from_host", c_int32, c_void_p,
+                                   ctypes.POINTER(BucketPtrs), ctypes.POINTER(c_void_p), c_int32,
+                                   c_float, c_void_p, c_size_t, c_void_p, c_void_p, c_void_p)
+dion_free = _sig("dion_free", c_int32, c_void_p)
+dion_status_string = _sig("dion_status_string", ctypes.c_char_p, c_int32)
+dion_last_error = _sig("dion_last_error", ctypes.c_char_p)
+dion_num_matrices = _sig("dion_num_matrices", c_int64, c_void_p)
+dion_last_launch_count = _sig("dion_last_launch_count", c_int32, c_void_p)
+dion_workspace_view = _sig("dion_workspace_view", c_int32, c_void_p, c_int32, c_int32, c_void_p,
+                           ctypes.POINTER(c_void_p), ctypes.POINTER(c_size_t))
+dion_profile_enable = _sig("dion_profile_enable", c_int32, c_void_p, c_int32)
+dion_profile_read = _sig("dion_profile_read", c_int32, c_void_p, ctypes.POINTER(ctypes.c_double),
+                         ctypes.POINTER(c_int64), c_int32)
+
+#: every entry point include/dion.h declares
+EXPORTED = ["dion_default_options", "dion_init", "dion_step_batched",
+            "dion_step_batched_from_host", "dion_free", "dion_status_string", "dion_last_error",
+            "dion_num_matrices", "dion_last_launch_count", "dion_workspace_view",
+            "dion_profile_enable", "dion_profile_read"]
+
+
+class DionError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = dion_status_string(code).decode()
+        detail = dion_last_error().decode()
+        super().__init__(f"{where}: {msg} ({code}): {detail}")
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise DionError(code, where)
+
+
+def default_options() -> Options:
+    o = Options()
+    _check(dion_default_options(ctypes.byref(o)), "dion_default_options")
+    return o
+
+
+@dataclass(frozen=True)
+class Shape:
+    count: int
+    m: int
+    n: int
+    r: int
+
+
+class DionB200:
+    """Handle of one planned step over a fixed list of shape buckets.
+
+    ``buckets``: sequence of (count, m, n, r).  Keyword options map onto
+    dion_options (include/dion.h).  All tensors handed to ``step`` are
+    contiguous CUDA tensors: X, M, G fp32 [count, m, n]; Q fp32 [count, n, r].
+    """
+
+    def __init__(self, buckets, *, mu=0.95, precision="bf16", orth_mode="auto",
+                 kernel_path="tensor", fallback_cond=1e3, orth_tol=2e-5,
+                 max_wait_spins=1 << 26, scales=None):
+        self.shapes = [Shape(*map(int, b)) for b in buckets]
+        n = len(self.shapes)
+        descs = (BucketDesc * max(n, 1))()
+        for i, s in enumerate(self.shapes):
+            descs[i].m, descs[i].n, descs[i].r, descs[i].count = s.m, s.n, s.r, s.count
+            descs[i].scale = float(scales[i]) if scales is not None else 0.0
+        o = default_options()
+        o.mu = mu
+        o.precision = PRECISIONS[precision]
+        o.orth_mode = ORTH_MODES[orth_mode]
+        o.kernel_path = KERNEL_PATHS[kernel_path]
+        o.fallback_cond = fallback_cond
+        o.orth_tol = orth_tol
+        o.max_wait_spins = max_wait_spins
+        self.options = o
+        h = c_void_p()
+        ws = c_size_t()
+        _check(dion_init(descs, n, ctypes.byref(o), ctypes.byref(h), ctypes.byref(ws)),
+               "dion_init")
+        self._h = h
+        self.workspace_bytes = ws.value
+        self.num_matrices = dion_num_matrices(h)
+
+    # ------------------------------------------------------------ memory helpers
+    def alloc_workspace(self, device=None):
+        import torch
+        return torch.empty(self.workspace_bytes, dtype=torch.uint8, device=device or "cuda")
+
+    def alloc_status(self, device=None):
+        import torch
+        return torch.zeros(self.num_matrices, dtype=torch.int32, device=device or "cuda")
+
+    def _ptrs(self, X, M, G, Q):
+        import torch
+        n = len(self.shapes)
+        if not (len(X) == len(M) == len(G) == len(Q) == n):
+            raise ValueError(f"expected {n} tensors each for X, M, G and Q")
+        arr = (BucketPtrs * n)()
+        for i, s in enumerate(self.shapes):
+            for name, t, shape in (("X", X[i], (s.count, s.m, s.n)), ("M", M[i], (s.count, s.m, s.n)),
+                                   ("G", G[i], (s.count, s.m, s.n)), ("Q", Q[i], (s.count, s.n, s.r))):
+                if not isinstance(t, torch.Tensor) or not t.is_cuda:
+                    raise ValueError(f"bucket {i}: {name} must be a CUDA tensor")
+                if t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != shape:
+                    raise ValueError(f"bucket {i}: {name} must be contiguous fp32 {shape}, "
+                                     f"got {t.dtype} {tuple(t.shape)}")
+            arr[i].X, arr[i].M = X[i].data_ptr(), M[i].data_ptr()
+            arr[i].G, arr[i].Q = G[i].data_ptr(), Q[i].data_ptr()
+        return arr
+
+    @staticmethod
+    def _stream(stream):
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream()
+        return c_void_p(stream.cuda_stream)
+
+    def step(self, X, M, G, Q, lr: float, workspace, status=None, stream=None):
+        """One Dion step over all buckets, enqueued on ``stream`` (default: current)."""
+        arr = self._ptrs(X, M, G, Q)
+        _check(dion_step_batched(self._h, arr, len(self.shapes), float(lr),
+                                 c_void_p(workspace.data_ptr()), workspace.numel(),
+                                 c_void_p(status.data_ptr()) if status is not None else None,
+                                 self._stream(stream)),
+               "dion_step_batched")
+
+    def step_from_host(self, X, M, G_dev, Q, G_host, lr: float, workspace, status, host_status,
+                       stream=None):
+        """Upload the host gradients G_host into G_dev, step, return the host status."""
+        arr = self._ptrs(X, M, G_dev, Q)
+        hg = (c_void_p * len(self.shapes))(*[g.data_ptr() for g in G_host])
+        _check(dion_step_batched_from_host(self._h, arr, hg, len(self.shapes), float(lr),
+                                           c_void_p(workspace.data_ptr()), workspace.numel(),
+                                           c_void_p(status.data_ptr()),
+                                           c_void_p(host_status.data_ptr()),
+                                           self._stream(stream)),
+               "dion_step_batched_from_host")
+        return host_status
+
+    def view(self, bucket: int, which: int, workspace):
+        """P ([count, m, r]) or R ([count, n, r]) of the last step, as a view of the workspace."""
+        import torch
+        ptr, nbytes = c_void_p(), c_size_t()
+        _check(dion_workspace_view(self._h, bucket, which, c_void_p(workspace.data_ptr()),
+                                   ctypes.byref(ptr), ctypes.byref(nbytes)), "dion_workspace_view")
+        off = ptr.value - workspace.data_ptr()
+        s = self.shapes[bucket]
+        shape = (s.count, s.m, s.r) if which == VIEW_P else (s.count, s.n, s.r)
+        return workspace[off:off + nbytes.value].view(torch.float32).view(*shape)
+
+    @property
+    def last_launch_count(self) -> int:
+        return dion_last_launch_count(self._h)
+
+    def profile_enable(self, on: bool = True):
+        _check(dion_profile_enable(self._h, int(on)), "dion_profile_enable")
+
+    def profile_read(self):
+        """{class: (milliseconds, launches)} summed since profile_enable."""
+        n = len(KERNEL_CLASSES)
+        ms = (ctypes.c_double * n)()
+        nl = (c_int64 * n)()
+        _check(dion_profile_read(self._h, ms, nl, n), "dion_profile_read")
+        return {k: (ms[i], nl[i]) for i, k in enumerate(KERNEL_CLASSES)}
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            dion_free(self._h)
+            self._h = c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,556 @@
+// C ABI of the batched Dion step (include/dion.h): argument checks, the
+// shape-bucket plan and workspace layout, and the launch sequence of one step.
+//
+// Buckets stack same-shape matrices into [count, m, n] tensors so each kernel
+// runs once per bucket over all of its matrices, as "DASH: Faster Shampoo via
+// Batched Block Preconditioning and Efficient Inverse-Root Solvers"
+// (Methodologie, section 1) stacks preconditioner blocks instead of looping.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/dion.h"
+#include "internal.h"
+#include "tc.h"
+
+namespace {
+
+thread_local std::string tl_error;
+
+dion_status fail(dion_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  tl_error = buf;
+  return s;
+}
+
+constexpr uint64_t kMagic = 0x44494f4e42323030ull;  // "DIONB200"
+constexpr int64_t kMaxElems = int64_t(1) << 40;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Plan {
+  int64_t m, n, r;
+  int count;
+  float scale;
+  int64_t mat0;
+  int nsplit;
+  size_t off_Bg, off_Qg, off_P0, off_P, off_P2, off_Pg, off_W, off_Linv, off_dinv, off_R, off_Rg,
+      off_Qng, off_part, off_flags, off_stats;
+};
+
+struct EventPair {
+  cudaEvent_t a, b;
+  int cls;
+  int launches;  // kernel launches between the two records
+};
+
+}  // namespace
+
+struct dion_ctx {
+  uint64_t magic;
+  dion_options opt;
+  std::vector<Plan> plans;
+  size_t ws_bytes;
+  int64_t total_mats;
+  int32_t last_launches;
+  int device_checked;  // device id verified as sm_100, -1 before
+  bool profiling;
+  std::vector<EventPair> events;
+  size_t events_used;
+  double prof_ms[DION_KCLASS_COUNT];
+  int64_t prof_launches[DION_KCLASS_COUNT];
+};
+
+namespace {
+
+bool valid(dion_handle h) { return h != nullptr && h->magic == kMagic; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dion_status check_options(const dion_options& o) {
+  if (!(o.mu >= 0.f && o.mu < 1.f)) return fail(DION_ERR_INVALID_ARG, "mu must be in [0, 1), got %g", o.mu);
+  if (o.precision != DION_PREC_FP32 && o.precision != DION_PREC_BF16)
+    return fail(DION_ERR_INVALID_ARG, "unknown precision %d", o.precision);
+  if (o.orth_mode < DION_ORTH_AUTO || o.orth_mode > DION_ORTH_HOUSEHOLDER)
+    return fail(DION_ERR_INVALID_ARG, "unknown orth_mode %d", o.orth_mode);
+  if (!(o.fallback_cond > 1.f)) return fail(DION_ERR_INVALID_ARG, "fallback_cond must exceed 1");
+  if (!(o.orth_tol >= 0.f)) return fail(DION_ERR_INVALID_ARG, "orth_tol must be >= 0");
+  if (o.kernel_path != DION_PATH_TENSOR && o.kernel_path != DION_PATH_SIMT)
+    return fail(DION_ERR_INVALID_ARG, "unknown kernel_path %d", o.kernel_path);
+  if (o.max_wait_spins < 1) return fail(DION_ERR_INVALID_ARG, "max_wait_spins must be >= 1");
+  return DION_OK;
+}
+
+// Per-step record of kernel launches (host counter) and optional events.
+struct StepCtx {
+  dion_handle h;
+  cudaStream_t s;
+  int launches;
+  int cur_cls;
+  EventPair* open;
+  int open_at;
+};
+
+void begin_cls(StepCtx& c, int cls) {
+  c.cur_cls = cls;
+  c.open = nullptr;
+  if (!c.h->profiling) return;
+  dion_handle h = c.h;
+  if (h->events_used == h->events.size()) {
+    EventPair ep{};
+    if (cudaEventCreate(&ep.a) != cudaSuccess || cudaEventCreate(&ep.b) != cudaSuccess) return;
+    h->events.push_back(ep);
+  }
+  EventPair& ep = h->events[h->events_used++];
+  ep.cls = cls;
+  ep.launches = 0;
+  cudaEventRecord(ep.a, c.s);
+  c.open = &ep;
+  c.open_at = c.launches;
+}
+
+void end_cls(StepCtx& c) {
+  if (c.open) {
+    cudaEventRecord(c.open->b, c.s);
+    c.open->launches = c.launches - c.open_at;
+  }
+  c.open = nullptr;
+}
+
+#define DION_LAUNCH(ctx, n, expr)                                                       \
+  do {                                                                                  \
+    cudaError_t e_ = (expr);                                                            \
+    (ctx).launches += (n);                                                              \
+    if (e_ != cudaSuccess) return fail(DION_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+  } while (0)
+
+dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, float lr,
+                       char* ws, int32_t* d_status) {
+  const dion_options& o = c.h->opt;
+  const bool bf = o.precision == DION_PREC_BF16;
+  const bool tensor = o.kernel_path == DION_PATH_TENSOR;
+  const int ge = bf ? 2 : 4;
+  (void)ge;
+  void* Bg = ws + p.off_Bg;
+  void* Qg = ws + p.off_Qg;
+  float* P0 = reinterpret_cast<float*>(ws + p.off_P0);
+  float* P = reinterpret_cast<float*>(ws + p.off_P);
+  float* P2 = reinterpret_cast<float*>(ws + p.off_P2);
+  void* Pg = bf ? (void*)(ws + p.off_Pg) : (void*)P;
+  float* W = reinterpret_cast<float*>(ws + p.off_W);
+  float* Linv = reinterpret_cast<float*>(ws + p.off_Linv);
+  float* dinv = reinterpret_cast<float*>(ws + p.off_dinv);
+  float* R = reinterpret_cast<float*>(ws + p.off_R);
+  void* Rg = bf ? (void*)(ws + p.off_Rg) : (void*)R;
+  void* Qng = bf ? (void*)(ws + p.off_Qng) : (void*)bp.Q;
+  float* part = reinterpret_cast<float*>(ws + p.off_part);
+  int32_t* flags = reinterpret_cast<int32_t*>(ws + p.off_flags);
+  float* stats = reinterpret_cast<float*>(ws + p.off_stats);
+  const int64_t m = p.m, n = p.n, r = p.r;
+  const int cnt = p.count;
+  cudaStream_t s = c.s;
+
+  DION_LAUNCH(c, 1, dion::launch_init_flags(flags, stats, cnt,
+                                            o.orth_mode == DION_ORTH_HOUSEHOLDER ? DION_MAT_FALLBACK : 0,
+                                            s));
+
+  // step 1: B = M + G in the precision of the contractions
+  begin_cls(c, DION_KCLASS_FORM_B);
+  DION_LAUNCH(c, 1, dion::launch_form_b(bp.M, bp.G, Bg, bf, (int64_t)cnt * m * n, s));
+  end_cls(c);
+
+  begin_cls(c, DION_KCLASS_PREP_Q);
+  DION_LAUNCH(c, 1, dion::launch_prep_q(bp.Q, Qg, bf, cnt, n, r, s));
+  end_cls(c);
+
+  // step 2: P0 = B Q
+  begin_cls(c, DION_KCLASS_GEMM_BQ);
+  {
+    bool done = false;
+    if (tensor && bf) {
+      int nl = 0;
+      cudaError_t e = dion::tc_gemm_bq(Bg, Qg, P0, cnt, m, n, r, o.max_wait_spins, flags, s, &nl, &done);
+      c.launches += nl;
+      if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_gemm_bq: %s", cudaGetErrorString(e));
+    }
+    if (!done) {
+      dion::GemmDesc d{};
+      d.A = {Bg, m * n, n, 1};
+      d.B = {Qg, n * r, n, 1};
+      d.C = P0; d.sCb = m * r; d.sCi = r; d.sCj = 1;
+      d.M = (int)m; d.N = (int)r; d.K = (int)n; d.batch = cnt; d.alpha = 1.f;
+      DION_LAUNCH(c, (cnt + 65534) / 65535, dion::launch_gemm_simt(d, bf, s));
+    }
+  }
+  end_cls(c);
+
+  // step 3: P = orth(P0) -- Cholesky-QR, optional second pass, Householder fallback
+  begin_cls(c, DION_KCLASS_ORTH);
+  {
+    auto gram = [&](const float* src) {
+      dion::GemmDesc d{};
+      d.A = {src, m * r, 1, r};
+      d.B = {src, m * r, 1, r};
+      d.C = W; d.sCb = r * r; d.sCi = r; d.sCj = 1;
+      d.M = (int)r; d.N = (int)r; d.K = (int)m; d.batch = cnt; d.alpha = 1.f;
+      d.flags = flags; d.need_mask = 0; d.skip_mask = DION_MAT_FALLBACK;
+      return d;
+    };
+    auto apply = [&](const float* src, float* dst, int32_t need) {
+      dion::GemmDesc d{};
+      d.A = {src, m * r, r, 1};
+      d.B = {Linv, r * r, r, 1};
+      d.C = dst; d.sCb = m * r; d.sCi = r; d.sCj = 1;
+      d.M = (int)m; d.N = (int)r; d.K = (int)r; d.batch = cnt; d.alpha = 1.f;
+      d.flags = flags; d.need_mask = need; d.skip_mask = DION_MAT_FALLBACK;
+      return d;
+    };
+    const int gl = (cnt + 65534) / 65535;
+    dion::CholArgs ca{};
+    ca.W = W; ca.Linv = Linv; ca.dinv = dinv; ca.flags = flags; ca.stats = stats;
+    ca.count = cnt; ca.r = r; ca.fallback_cond = o.fallback_cond;
+    const int chol_launches = r <= 256 ? 1 : (int)(2 + 3 * ((r + 31) / 32) + (r + 31) / 32);
+    if (o.orth_mode != DION_ORTH_HOUSEHOLDER) {
+      DION_LAUNCH(c, gl, dion::launch_gemm_simt(gram(P0), false, s));
+      ca.pass = 1; ca.orth_tol = o.orth_tol;
+      DION_LAUNCH(c, chol_launches, dion::launch_chol_inv(ca, s));
+      DION_LAUNCH(c, gl, dion::launch_gemm_simt(apply(P0, P, 0), false, s));
+      if (o.orth_mode != DION_ORTH_CHOLQR) {
+        DION_LAUNCH(c, gl, dion::launch_gemm_simt(gram(P), false, s));
+        ca.pass = 2;
+        ca.orth_tol = o.orth_mode == DION_ORTH_CHOLQR2 ? -1.f : o.orth_tol;
+        DION_LAUNCH(c, chol_launches, dion::launch_chol_inv(ca, s));
+        DION_LAUNCH(c, gl, dion::launch_gemm_simt(apply(P, P2, DION_MAT_CHOLQR2), false, s));
+      }
+    }
+    DION_LAUNCH(c, 1, dion::launch_householder(P0, P2, P0, P, flags, cnt, m, r, s));
+    DION_LAUNCH(c, 1, dion::launch_finalize_p(P, P2, Pg, bf, flags, cnt, m, r, P, s));
+  }
+  end_cls(c);
+
+  // step 4: R = B^T P
+  begin_cls(c, DION_KCLASS_GEMM_BTP);
+  {
+    bool done = false;
+    if (tensor && bf) {
+      int nl = 0;
+      cudaError_t e = dion::tc_gemm_btp(Bg, Pg, R, cnt, m, n, r, o.max_wait_spins, flags, s, &nl, &done);
+      c.launches += nl;
+      if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_gemm_btp: %s", cudaGetErrorString(e));
+    }
+    if (!done) {
+      dion::GemmDesc d{};
+      d.A = {Bg, m * n, 1, n};
+      d.B = {Pg, m * r, 1, r};
+      d.C = R; d.sCb = n * r; d.sCi = r; d.sCj = 1;
+      d.M = (int)n; d.N = (int)r; d.K = (int)m; d.batch = cnt; d.alpha = 1.f;
+      DION_LAUNCH(c, (cnt + 65534) / 65535, dion::launch_gemm_simt(d, bf, s));
+    }
+  }
+  end_cls(c);
+
+  // step 6: Q = colnorm(R), plus the GEMM copies of R and Q for the update
+  begin_cls(c, DION_KCLASS_COLNORM);
+  DION_LAUNCH(c, 2, dion::launch_colnorm(R, bp.Q, Rg, Qng, bf, part, p.nsplit, flags, cnt, n, r, s));
+  end_cls(c);
+
+  // steps 5 and 7: M <- B - (1 - mu) P R^T and X <- X - lr s P Q^T in one pass
+  begin_cls(c, DION_KCLASS_UPDATE);
+  {
+    bool done = false;
+    const float lrs = lr * p.scale;
+    if (tensor && bf) {
+      int nl = 0;
+      cudaError_t e = dion::tc_update(Pg, Rg, Qng, bp.G, bp.M, bp.X, cnt, m, n, r, o.mu, lrs,
+                                      o.max_wait_spins, flags, s, &nl, &done);
+      c.launches += nl;
+      if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_update: %s", cudaGetErrorString(e));
+    }
+    if (!done)
+      DION_LAUNCH(c, (cnt + 65534) / 65535,
+                  dion::launch_update_simt(Pg, Rg, Qng, bf, bp.G, bp.M, bp.X, cnt, m, n, r, o.mu,
+                                           lrs, s));
+  }
+  end_cls(c);
+
+  if (d_status) DION_LAUNCH(c, 1, dion::launch_write_status(flags, d_status + p.mat0, cnt, s));
+  return DION_OK;
+}
+
+dion_status check_device(dion_handle h) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(DION_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (h->device_checked == dev) return DION_OK;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(DION_ERR_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a (B200)",
+                dev, major, minor);
+  h->device_checked = dev;
+  return DION_OK;
+}
+
+dion_status check_step_args(dion_handle h, const dion_bucket_ptrs* ptrs, int32_t nbuckets,
+                            void* ws, size_t ws_bytes, int32_t* d_status) {
+  if (!valid(h)) return fail(DION_ERR_NOT_INITIALIZED, "invalid or freed handle");
+  if (ptrs == nullptr) return fail(DION_ERR_INVALID_ARG, "ptrs is NULL");
+  if (nbuckets != (int32_t)h->plans.size())
+    return fail(DION_ERR_INVALID_ARG, "nbuckets %d does not match the plan (%zu)", nbuckets,
+                h->plans.size());
+  if (ws == nullptr) return fail(DION_ERR_INVALID_ARG, "workspace is NULL");
+  if (ws_bytes < h->ws_bytes)
+    return fail(DION_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes, %zu needed", ws_bytes,
+                h->ws_bytes);
+  if (!aligned16(ws)) return fail(DION_ERR_MISALIGNED, "workspace is not 16-byte aligned");
+  if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u))
+    return fail(DION_ERR_MISALIGNED, "d_status is not 4-byte aligned");
+  for (int32_t b = 0; b < nbuckets; ++b) {
+    const dion_bucket_ptrs& p = ptrs[b];
+    if (!p.X || !p.M || !p.G || !p.Q)
+      return fail(DION_ERR_INVALID_ARG, "bucket %d: a NULL device pointer", b);
+    if (!aligned16(p.X) || !aligned16(p.M) || !aligned16(p.G) || !aligned16(p.Q))
+      return fail(DION_ERR_MISALIGNED, "bucket %d: X, M, G and Q must be 16-byte aligned", b);
+  }
+  return check_device(h);
+}
+
+}  // namespace
+
+extern "C" {
+
+dion_status dion_default_options(dion_options* opt) {
+  if (!opt) return fail(DION_ERR_INVALID_ARG, "opt is NULL");
+  opt->mu = 0.95f;
+  opt->precision = DION_PREC_BF16;
+  opt->orth_mode = DION_ORTH_AUTO;
+  opt->fallback_cond = 1e3f;
+  opt->orth_tol = 2e-5f;
+  opt->kernel_path = DION_PATH_TENSOR;
+  opt->max_wait_spins = int64_t(1) << 26;
+  return DION_OK;
+}
+
+dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const dion_options* opt,
+                      dion_handle* out, size_t* workspace_bytes) {
+  if (!out || !workspace_bytes) return fail(DION_ERR_INVALID_ARG, "out or workspace_bytes is NULL");
+  *out = nullptr;
+  *workspace_bytes = 0;
+  if (!buckets || nbuckets < 1) return fail(DION_ERR_INVALID_ARG, "need at least one bucket");
+  dion_options o;
+  if (opt) o = *opt; else dion_default_options(&o);
+  dion_status st = check_options(o);
+  if (st != DION_OK) return st;
+  const bool bf = o.precision == DION_PREC_BF16;
+  const size_t ge = bf ? 2 : 4;
+  std::vector<Plan> plans;
+  size_t off = 0;
+  int64_t mats = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 1024);
+    return at;
+  };
+  for (int32_t b = 0; b < nbuckets; ++b) {
+    const dion_bucket_desc& d = buckets[b];
+    if (d.count < 1) return fail(DION_ERR_INVALID_ARG, "bucket %d: count %d < 1", b, d.count);
+    if (d.m < 1 || d.n < 1 || d.r < 1)
+      return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: m, n, r must be positive", b);
+    if (d.r > d.m || d.r > d.n)
+      return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: r=%lld exceeds min(m, n)", b, (long long)d.r);
+    if (d.r % 16 != 0)
+      return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: r=%lld is not a multiple of 16", b, (long long)d.r);
+    if (d.n % 8 != 0)
+      return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: n=%lld is not a multiple of 8", b, (long long)d.n);
+    if (d.m > (int64_t(1) << 30) || d.n > (int64_t(1) << 30) ||
+        (int64_t)d.count * d.m > kMaxElems / d.n || (int64_t)d.count * d.n > kMaxElems / d.r ||
+        (int64_t)d.count * d.m > kMaxElems / d.r)
+      return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: too large", b);
+    if (!(std::isfinite(d.scale)))
+      return fail(DION_ERR_INVALID_ARG, "bucket %d: scale is not finite", b);
+    Plan p{};
+    p.m = d.m; p.n = d.n; p.r = d.r; p.count = d.count;
+    p.scale = d.scale > 0.f ? d.scale : (float)std::sqrt((double)d.m / (double)d.n);
+    p.mat0 = mats;
+    mats += d.count;
+    {
+      int64_t ns = (2 * 148 + d.count - 1) / d.count;
+      if (ns > 64) ns = 64;
+      if (ns > (d.n + 31) / 32) ns = (d.n + 31) / 32;
+      if (ns < 1) ns = 1;
+      p.nsplit = (int)ns;
+    }
+    const size_t c = (size_t)d.count;
+    p.off_Bg = take(c * d.m * d.n * ge);
+    p.off_Qg = take(c * d.n * d.r * ge);
+    p.off_P0 = take(c * d.m * d.r * 4);
+    p.off_P = take(c * d.m * d.r * 4);
+    p.off_P2 = take(c * d.m * d.r * 4);
+    p.off_Pg = bf ? take(c * d.m * d.r * 2) : 0;
+    p.off_W = take(c * d.r * d.r * 4);
+    p.off_Linv = take(c * d.r * d.r * 4);
+    p.off_dinv = take(dion::chol_dinv_floats(d.count, d.r) * 4);
+    p.off_R = take(c * d.n * d.r * 4);
+    p.off_Rg = bf ? take(c * d.n * d.r * 2) : 0;
+    p.off_Qng = bf ? take(c * d.n * d.r * 2) : 0;
+    p.off_part = take(c * p.nsplit * d.r * 4);
+    p.off_flags = take(c * 4);
+    p.off_stats = take(c * 8);
+    plans.push_back(p);
+  }
+  dion_ctx* h = new (std::nothrow) dion_ctx();
+  if (!h) return fail(DION_ERR_INVALID_ARG, "out of host memory");
+  h->magic = kMagic;
+  h->opt = o;
+  h->plans = std::move(plans);
+  h->ws_bytes = off;
+  h->total_mats = mats;
+  h->last_launches = 0;
+  h->device_checked = -1;
+  h->profiling = false;
+  h->events_used = 0;
+  for (int i = 0; i < DION_KCLASS_COUNT; ++i) { h->prof_ms[i] = 0; h->prof_launches[i] = 0; }
+  *out = h;
+  *workspace_bytes = off;
+  return DION_OK;
+}
+
+dion_status dion_step_batched(dion_handle h, const dion_bucket_ptrs* ptrs, int32_t nbuckets,
+                              float lr, void* d_workspace, size_t workspace_bytes,
+                              int32_t* d_status, void* stream) {
+  dion_status st = check_step_args(h, ptrs, nbuckets, d_workspace, workspace_bytes, d_status);
+  if (st != DION_OK) return st;
+  if (!std::isfinite(lr)) return fail(DION_ERR_INVALID_ARG, "lr is not finite");
+  StepCtx c{h, reinterpret_cast<cudaStream_t>(stream), 0, -1, nullptr, 0};
+  for (int32_t b = 0; b < nbuckets; ++b) {
+    st = run_bucket(c, h->plans[b], ptrs[b], lr, static_cast<char*>(d_workspace), d_status);
+    if (st != DION_OK) {
+      end_cls(c);
+      h->last_launches = c.launches;
+      return st;
+    }
+  }
+  h->last_launches = c.launches;
+  return DION_OK;
+}
+
+dion_status dion_step_batched_from_host(dion_handle h, const dion_bucket_ptrs* ptrs,
+                                        const float* const* host_grads, int32_t nbuckets,
+                                        float lr, void* d_workspace, size_t workspace_bytes,
+                                        int32_t* d_status, int32_t* host_status, void* stream) {
+  dion_status st = check_step_args(h, ptrs, nbuckets, d_workspace, workspace_bytes, d_status);
+  if (st != DION_OK) return st;
+  if (!host_grads || !host_status || !d_status)
+    return fail(DION_ERR_INVALID_ARG, "host_grads, host_status and d_status are required");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  for (int32_t b = 0; b < nbuckets; ++b) {
+    if (!host_grads[b]) return fail(DION_ERR_INVALID_ARG, "host_grads[%d] is NULL", b);
+    const Plan& p = h->plans[b];
+    const size_t bytes = (size_t)p.count * p.m * p.n * sizeof(float);
+    cudaError_t e = cudaMemcpyAsync(const_cast<float*>(ptrs[b].G), host_grads[b], bytes,
+                                    cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return fail(DION_ERR_CUDA, "gradient upload: %s", cudaGetErrorString(e));
+  }
+  st = dion_step_batched(h, ptrs, nbuckets, lr, d_workspace, workspace_bytes, d_status, stream);
+  if (st != DION_OK) return st;
+  cudaError_t e = cudaMemcpyAsync(host_status, d_status, (size_t)h->total_mats * sizeof(int32_t),
+                                  cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return fail(DION_ERR_CUDA, "status download: %s", cudaGetErrorString(e));
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(DION_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+  return DION_OK;
+}
+
+dion_status dion_free(dion_handle h) {
+  if (!h) return DION_OK;
+  if (!valid(h)) return fail(DION_ERR_NOT_INITIALIZED, "invalid or freed handle");
+  for (auto& ep : h->events) {
+    cudaEventDestroy(ep.a);
+    cudaEventDestroy(ep.b);
+  }
+  h->magic = 0;
+  delete h;
+  return DION_OK;
+}
+
+const char* dion_status_string(dion_status s) {
+  switch (s) {
+    case DION_OK: return "ok";
+    case DION_ERR_INVALID_ARG: return "invalid argument";
+    case DION_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case DION_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case DION_ERR_CUDA: return "CUDA error";
+    case DION_ERR_NOT_INITIALIZED: return "handle not initialized";
+    case DION_ERR_DEVICE: return "unsupported device";
+    case DION_ERR_MISALIGNED: return "misaligned pointer";
+  }
+  return "unknown status";
+}
+
+const char* dion_last_error(void) { return tl_error.c_str(); }
+
+int64_t dion_num_matrices(dion_handle h) { return valid(h) ? h->total_mats : -1; }
+
+int32_t dion_last_launch_count(dion_handle h) { return valid(h) ? h->last_launches : -1; }
+
+dion_status dion_workspace_view(dion_handle h, int32_t bucket, int32_t which, void* d_workspace,
+                                void** d_ptr, size_t* bytes) {
+  if (!valid(h)) return fail(DION_ERR_NOT_INITIALIZED, "invalid or freed handle");
+  if (!d_ptr || !bytes || !d_workspace) return fail(DION_ERR_INVALID_ARG, "NULL argument");
+  if (bucket < 0 || bucket >= (int32_t)h->plans.size())
+    return fail(DION_ERR_INVALID_ARG, "bucket %d out of range", bucket);
+  const Plan& p = h->plans[bucket];
+  char* ws = static_cast<char*>(d_workspace);
+  if (which == DION_VIEW_P) {
+    *d_ptr = ws + p.off_P;
+    *bytes = (size_t)p.count * p.m * p.r * 4;
+  } else if (which == DION_VIEW_R) {
+    *d_ptr = ws + p.off_R;
+    *bytes = (size_t)p.count * p.n * p.r * 4;
+  } else {
+    return fail(DION_ERR_INVALID_ARG, "unknown view %d", which);
+  }
+  return DION_OK;
+}
+
+dion_status dion_profile_enable(dion_handle h, int32_t on) {
+  if (!valid(h)) return fail(DION_ERR_NOT_INITIALIZED, "invalid or freed handle");
+  h->profiling = on != 0;
+  h->events_used = 0;
+  for (int i = 0; i < DION_KCLASS_COUNT; ++i) { h->prof_ms[i] = 0; h->prof_launches[i] = 0; }
+  return DION_OK;
+}
+
+dion_status dion_profile_read(dion_handle h, double* ms, int64_t* launches, int32_t nclasses) {
+  if (!valid(h)) return fail(DION_ERR_NOT_INITIALIZED, "invalid or freed handle");
+  if (!ms || nclasses < 1) return fail(DION_ERR_INVALID_ARG, "ms is NULL or nclasses < 1");
+  for (size_t i = 0; i < h->events_used; ++i) {
+    EventPair& ep = h->events[i];
+    cudaError_t e = cudaEventSynchronize(ep.b);
+    if (e != cudaSuccess) return fail(DION_ERR_CUDA, "cudaEventSynchronize: %s", cudaGetErrorString(e));
+    float t = 0.f;
+    e = cudaEventElapsedTime(&t, ep.a, ep.b);
+    if (e != cudaSuccess) return fail(DION_ERR_CUDA, "cudaEventElapsedTime: %s", cudaGetErrorString(e));
+    h->prof_ms[ep.cls] += t;
+    h->prof_launches[ep.cls] += ep.launches;
+  }
+  h->events_used = 0;
+  for (int i = 0; i < nclasses && i < DION_KCLASS_COUNT; ++i) {
+    ms[i] = h->prof_ms[i];
+    if (launches) launches[i] = h->prof_launches[i];
+  }
+  return DION_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// Internal interface between the host planner (dion_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace dion {
+
+// Generic strided batched operand: element (i, k) of matrix b sits at
+// base + b*sb + i*si + k*sk (in elements).
+struct Operand {
+  const void* ptr;
+  int64_t sb, si, sk;
+};
+
+// C[b] = alpha * A[b] (M x K) * B[b] (K x N), fp32 accumulation, fp32 output.
+// A matrix b is skipped when flags != nullptr and
+// (flags[b] & need_mask) != need_mask or (flags[b] & skip_mask) != 0.
+struct GemmDesc {
+  Operand A, B;
+  float* C;
+  int64_t sCb, sCi, sCj;
+  int M, N, K, batch;
+  float alpha;
+  const int32_t* flags;
+  int32_t need_mask, skip_mask;
+};
+
+// ---- elementwise / layout kernels (k_elementwise.cu)
+cudaError_t launch_form_b(const float* M, const float* G, void* Bg, bool use_bf16, int64_t elems,
+                          cudaStream_t s);
+cudaError_t launch_prep_q(const float* Q, void* Qg, bool use_bf16, int count, int64_t n, int64_t r,
+                          cudaStream_t s);
+cudaError_t launch_init_flags(int32_t* flags, float* stats, int count, int32_t init_bits,
+                              cudaStream_t s);
+cudaError_t launch_finalize_p(const float* P, const float* P2, void* Pg, bool use_bf16,
+                              const int32_t* flags, int count, int64_t m, int64_t r,
+                              float* P_out, cudaStream_t s);
+cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, bool use_bf16,
+                           float* part, int nsplit, int32_t* flags, int count, int64_t n,
+                           int64_t r, cudaStream_t s);
+cudaError_t launch_write_status(const int32_t* flags, int32_t* d_status, int count,
+                                cudaStream_t s);
+
+// ---- SIMT contractions (k_gemm_simt.cu)
+cudaError_t launch_gemm_simt(const GemmDesc& d, bool bf16_operands, cudaStream_t s);
+cudaError_t launch_update_simt(const void* Pg, const void* Rg, const void* Qg, bool use_bf16,
+                               const float* G, float* M, float* X, int count, int64_t m,
+                               int64_t n, int64_t r, float mu, float lr_scale, cudaStream_t s);
+
+// ---- orthonormalisation (k_orth.cu)
+// pass 1: Cholesky of W = P0^T P0; pass 2: checks W = P1^T P1 first.
+struct CholArgs {
+  float* W;            // [count, r, r] Gram on entry (lower part overwritten by L)
+  float* Linv;         // [count, r, r] receives L^-1 (upper part zero)
+  float* dinv;         // [count, r, 32] scratch: inverses of 32x32 diagonal blocks
+  int32_t* flags;      // [count]
+  float* stats;        // [count, 2] min and max of diag(L) (positive floats)
+  int count;
+  int64_t r;
+  int pass;            // 1 or 2
+  float fallback_cond; // pass 1: diag ratio limit
+  float orth_tol;      // pass 2: skip the second pass when max|W - I| <= orth_tol
+};
+cudaError_t launch_chol_inv(const CholArgs& a, cudaStream_t s);
+cudaError_t launch_householder(const float* P0, float* work_cm, float* q_cm, float* P,
+                               int32_t* flags, int count, int64_t m, int64_t r,
+                               cudaStream_t s);
+size_t chol_dinv_floats(int count, int64_t r);
+
+}  // namespace dion

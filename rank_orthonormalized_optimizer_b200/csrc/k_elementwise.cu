@@ -1,0 +1,268 @@
+// Streaming and layout kernels of the batched Dion step: B = M + G in GEMM
+// precision, the previous Q in GEMM layout, the final P and its GEMM copy,
+// Q = colnorm(R) with the update operands, and the per-matrix status words.
+#include "common.cuh"
+#include "internal.h"
+
+namespace dion {
+
+static int g_sms = 0;
+static int sm_count() {
+  if (g_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_sms <= 0) g_sms = 148;
+  }
+  return g_sms;
+}
+
+// ---------------------------------------------------------------- B = M + G
+// Step 1 of the Dion step (error-feedback buffer plus this step's gradient),
+// written once in the precision the contractions read.  Pure HBM stream:
+// 8 bytes read and 2 (bf16) or 4 (fp32) bytes written per element.
+template <bool BF16, int U>
+__global__ void __launch_bounds__(256) k_form_b(const float4* __restrict__ M,
+                                                 const float4* __restrict__ G,
+                                                 void* __restrict__ B, int64_t n4) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < n4;
+       base += stride * U) {
+    float4 a[U], g[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = base + u * stride;
+      if (i < n4) {
+        a[u] = __ldcs(M + i);
+        g[u] = __ldcs(G + i);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = base + u * stride;
+      if (i < n4) {
+        float4 c = make_float4(a[u].x + g[u].x, a[u].y + g[u].y, a[u].z + g[u].z,
+                               a[u].w + g[u].w);
+        if (BF16) {
+          __nv_bfloat162 lo = __floats2bfloat162_rn(c.x, c.y);
+          __nv_bfloat162 hi = __floats2bfloat162_rn(c.z, c.w);
+          uint2 pk;
+          pk.x = *reinterpret_cast<uint32_t*>(&lo);
+          pk.y = *reinterpret_cast<uint32_t*>(&hi);
+          reinterpret_cast<uint2*>(B)[i] = pk;
+        } else {
+          reinterpret_cast<float4*>(B)[i] = c;
+        }
+      }
+    }
+  }
+}
+
+cudaError_t launch_form_b(const float* M, const float* G, void* Bg, bool use_bf16, int64_t elems,
+                          cudaStream_t s) {
+  const int64_t n4 = elems / 4;
+  int64_t want = (n4 + 255) / 256;
+  int64_t grid = (int64_t)sm_count() * 4;
+  if (want < grid) grid = want < 1 ? 1 : want;
+  if (use_bf16)
+    k_form_b<true, 4><<<(unsigned)grid, 256, 0, s>>>((const float4*)M, (const float4*)G, Bg, n4);
+  else
+    k_form_b<false, 4><<<(unsigned)grid, 256, 0, s>>>((const float4*)M, (const float4*)G, Bg, n4);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------- previous Q into GEMM layout
+// Qg[b][j][i] = Q[b][i][j]: the n x r factor transposed to r x n so that the
+// contraction B Q reads both operands along n (the reduction axis).
+template <typename T>
+__global__ void k_prep_q(const float* __restrict__ Q, T* __restrict__ Qg, int64_t n, int64_t r) {
+  __shared__ float tile[32][33];
+  const int64_t b = blockIdx.z;
+  const float* q = Q + b * n * r;
+  T* qg = Qg + b * n * r;
+  const int64_t j0 = (int64_t)blockIdx.x * 32, i0 = (int64_t)blockIdx.y * 32;
+  for (int y = threadIdx.y; y < 32; y += 8) {
+    const int64_t i = i0 + y, j = j0 + threadIdx.x;
+    tile[y][threadIdx.x] = (i < n && j < r) ? q[i * r + j] : 0.f;
+  }
+  __syncthreads();
+  for (int y = threadIdx.y; y < 32; y += 8) {
+    const int64_t j = j0 + y, i = i0 + threadIdx.x;
+    if (i < n && j < r) qg[j * n + i] = Cvt<T>::from_f(tile[threadIdx.x][y]);
+  }
+}
+
+cudaError_t launch_prep_q(const float* Q, void* Qg, bool use_bf16, int count, int64_t n, int64_t r,
+                          cudaStream_t s) {
+  dim3 grid((unsigned)((r + 31) / 32), (unsigned)((n + 31) / 32), (unsigned)count);
+  dim3 block(32, 8);
+  if (use_bf16)
+    k_prep_q<bf16><<<grid, block, 0, s>>>(Q, (bf16*)Qg, n, r);
+  else
+    k_prep_q<float><<<grid, block, 0, s>>>(Q, (float*)Qg, n, r);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------- flags and status
+__global__ void k_init_flags(int32_t* flags, float* stats, int count, int32_t init_bits) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < count) {
+    flags[b] = init_bits;
+    stats[2 * b] = 3.0e38f;  // running min of diag(L)
+    stats[2 * b + 1] = 0.f;  // running max of diag(L)
+  }
+}
+
+cudaError_t launch_init_flags(int32_t* flags, float* stats, int count, int32_t init_bits,
+                              cudaStream_t s) {
+  k_init_flags<<<(count + 255) / 256, 256, 0, s>>>(flags, stats, count, init_bits);
+  return cudaGetLastError();
+}
+
+__global__ void k_write_status(const int32_t* flags, int32_t* st, int count) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < count) st[b] = flags[b];
+}
+
+cudaError_t launch_write_status(const int32_t* flags, int32_t* d_status, int count,
+                                cudaStream_t s) {
+  k_write_status<<<(count + 255) / 256, 256, 0, s>>>(flags, d_status, count);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------- final P
+// P holds the first Cholesky-QR pass or the Householder result; P2 the
+// second pass.  Picks per matrix, then writes the GEMM copy Pg (bf16 mode).
+template <bool BF16>
+__global__ void k_finalize_p(float* __restrict__ P, const float* __restrict__ P2,
+                             void* __restrict__ Pg, const int32_t* __restrict__ flags,
+                             int64_t mr4) {
+  const int64_t b = blockIdx.y;
+  const int32_t f = flags[b];
+  const bool take2 = (f & F_CHOLQR2) && !(f & F_FALLBACK);
+  if (!take2 && !BF16) return;
+  float4* p = reinterpret_cast<float4*>(P) + b * mr4;
+  const float4* p2 = reinterpret_cast<const float4*>(P2) + b * mr4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < mr4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float4 v = take2 ? p2[i] : p[i];
+    if (take2) p[i] = v;
+    if (BF16) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(Pg)[b * mr4 + i] = pk;
+    }
+  }
+}
+
+cudaError_t launch_finalize_p(const float* P, const float* P2, void* Pg, bool use_bf16,
+                              const int32_t* flags, int count, int64_t m, int64_t r,
+                              float* P_out, cudaStream_t s) {
+  (void)P;
+  const int64_t mr4 = m * r / 4;
+  int64_t gx = (mr4 + 255) / 256;
+  if (gx > 64) gx = 64;
+  dim3 grid((unsigned)gx, (unsigned)count);
+  if (use_bf16)
+    k_finalize_p<true><<<grid, 256, 0, s>>>(P_out, P2, Pg, flags, mr4);
+  else
+    k_finalize_p<false><<<grid, 256, 0, s>>>(P_out, P2, Pg, flags, mr4);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------- Q = colnorm(R)
+// Step 6: each column of R (n x r) divided by its 2-norm over the n rows.
+// Deterministic two-stage reduction: fixed row splits, then a fixed-order
+// sum of the splits.  A zero column gives a zero Q column and F_ZERO_COL.
+__global__ void __launch_bounds__(256) k_colnorm_partial(const float* __restrict__ R,
+                                                          float* __restrict__ part, int64_t n,
+                                                          int64_t r, int nsplit) {
+  const int64_t b = blockIdx.y;
+  const int split = blockIdx.x;
+  const int64_t rows = (n + nsplit - 1) / nsplit;
+  const int64_t i0 = split * rows, i1 = (i0 + rows < n) ? i0 + rows : n;
+  const float* rb = R + b * n * r;
+  for (int64_t j = threadIdx.x; j < r; j += blockDim.x) {
+    float acc = 0.f;
+#pragma unroll 8
+    for (int64_t i = i0; i < i1; ++i) {
+      const float v = rb[i * r + j];
+      acc = fmaf(v, v, acc);
+    }
+    part[(b * nsplit + split) * r + j] = acc;
+  }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_colnorm_apply(const float* __restrict__ R,
+                                                        float* __restrict__ Q,
+                                                        void* __restrict__ Rg,
+                                                        void* __restrict__ Qg,
+                                                        const float* __restrict__ part,
+                                                        int32_t* __restrict__ flags, int64_t n,
+                                                        int64_t r, int nsplit,
+                                                        int64_t rows_per_block) {
+  extern __shared__ float norm_s[];  // r floats
+  const int64_t b = blockIdx.y;
+  bool zero = false;
+  for (int64_t j = threadIdx.x; j < r; j += blockDim.x) {
+    float ss = 0.f;
+    for (int s2 = 0; s2 < nsplit; ++s2) ss += part[(b * nsplit + s2) * r + j];
+    const float nrm = sqrtf(ss);
+    norm_s[j] = nrm;
+    zero |= !(nrm > 0.f);
+  }
+  zero = __syncthreads_or(zero);
+  if (zero && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(flags + b, F_ZERO_COL);
+  const int64_t i0 = blockIdx.x * rows_per_block;
+  const int64_t i1 = (i0 + rows_per_block < n) ? i0 + rows_per_block : n;
+  const int64_t base = b * n * r;
+  for (int64_t i = i0; i < i1; ++i) {
+    for (int64_t j = threadIdx.x; j < r; j += blockDim.x) {
+      const int64_t e = base + i * r + j;
+      const float rv = R[e];
+      const float nrm = norm_s[j];
+      const float qv = nrm > 0.f ? rv / nrm : 0.f;
+      Q[e] = qv;
+      if (BF16) {
+        reinterpret_cast<bf16*>(Rg)[e] = __float2bfloat16_rn(rv);
+        reinterpret_cast<bf16*>(Qg)[e] = __float2bfloat16_rn(qv);
+      }
+    }
+  }
+}
+
+cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, bool use_bf16, float* part,
+                           int nsplit, int32_t* flags, int count, int64_t n, int64_t r,
+                           cudaStream_t s) {
+  k_colnorm_partial<<<dim3((unsigned)nsplit, (unsigned)count), 256, 0, s>>>(R, part, n, r,
+                                                                            nsplit);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t target_blocks = 2 * (int64_t)sm_count();
+  int64_t per_mat = (target_blocks + count - 1) / count;
+  int64_t rows = (n + per_mat - 1) / per_mat;
+  if (rows < 8) rows = 8;
+  const int64_t gx = (n + rows - 1) / rows;
+  const size_t smem = (size_t)r * sizeof(float);
+  if (smem > 48 * 1024) {
+    if (use_bf16)
+      cudaFuncSetAttribute(k_colnorm_apply<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+    else
+      cudaFuncSetAttribute(k_colnorm_apply<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  }
+  if (use_bf16)
+    k_colnorm_apply<true><<<dim3((unsigned)gx, (unsigned)count), 256, smem, s>>>(
+        R, Q, Rg, Qg, part, flags, n, r, nsplit, rows);
+  else
+    k_colnorm_apply<false><<<dim3((unsigned)gx, (unsigned)count), 256, smem, s>>>(
+        R, Q, Rg, Qg, part, flags, n, r, nsplit, rows);
+  return cudaGetLastError();
+}
+
+}  // namespace dion

@@ -1,0 +1,25 @@
+// Tensor-core (tcgen05 + TMEM, fed by TMA) kernels of the batched Dion step.
+// Each entry sets *done when it handled the call; otherwise the caller runs
+// the SIMT kernel for the same contraction.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dion {
+
+// P0[b] (m x r, fp32) = Bg[b] (m x n, bf16) * Qg[b]^T (Qg: r x n, bf16).
+cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, int count, int64_t m,
+                       int64_t n, int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s,
+                       int* nlaunch, bool* done);
+// R[b] (n x r, fp32) = Bg[b]^T (n x m) * Pg[b] (m x r, bf16).
+cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, int count, int64_t m,
+                        int64_t n, int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s,
+                        int* nlaunch, bool* done);
+// M <- (M + G) - (1 - mu) Pg Rg^T and X <- X - lr_scale Pg Qg^T (Pg: m x r, Rg, Qg: n x r, bf16).
+cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, const float* G, float* M,
+                      float* X, int count, int64_t m, int64_t n, int64_t r, float mu,
+                      float lr_scale, int64_t max_spins, int32_t* flags, cudaStream_t s,
+                      int* nlaunch, bool* done);
+
+}  // namespace dion

@@ -1,16 +1,29 @@
+import importlib.util
 import os
 import sys
 
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-if ROOT not in sys.path:
-    sys.path.insert(0, ROOT)
+for p in (ROOT, os.path.dirname(os.path.abspath(__file__))):
+    if p not in sys.path:
+        sys.path.insert(0, p)
+
+
+def _ensure_library():
+    """Build the CUDA library if it is missing (the package refuses to import without it)."""
+    path = os.path.join(ROOT, "rank_orthonormalized_optimizer_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_dion_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    if not os.path.exists(mod.LIB):
+        mod.build()
 
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running case")
+    _ensure_library()
 
 
 def pytest_collection_modifyitems(config, items):

@@ -1,0 +1,150 @@
+"""The C-ABI library loads and exports every entry point include/dion.h declares,
+and its host-side checks return the documented status codes (no GPU needed: these
+calls stop before any device work)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import rank_orthonormalized_optimizer_b200 as dion
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dion.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dion_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_what_binding_wraps():
+    assert declared_functions() == sorted(dion.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported():
+    out = subprocess.run(["nm", "-D", "--defined-only", dion.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (dion_[a-z_]+)$", out, flags=re.M))
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(dion.LIB_PATH)
+    for f in declared_functions():
+        assert getattr(lib, f) is not None
+
+
+def test_library_needs_no_driver_to_load():
+    out = subprocess.run(["ldd", dion.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out          # the runtime is linked statically
+    assert "libtorch" not in out
+
+
+def test_build_targets_sm100a_only():
+    from rank_orthonormalized_optimizer_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def _init(buckets, **kw):
+    descs = (dion.BucketDesc * len(buckets))()
+    for i, (c, m, n, r) in enumerate(buckets):
+        descs[i].count, descs[i].m, descs[i].n, descs[i].r, descs[i].scale = c, m, n, r, 0.0
+    o = dion.default_options()
+    for k, v in kw.items():
+        setattr(o, k, v)
+    h = ctypes.c_void_p()
+    ws = ctypes.c_size_t()
+    code = dion.dion_init(descs, len(buckets), ctypes.byref(o), ctypes.byref(h), ctypes.byref(ws))
+    return code, h, ws.value
+
+
+def test_defaults():
+    o = dion.default_options()
+    assert abs(o.mu - 0.95) < 1e-7 and o.precision == 1 and o.orth_mode == 0
+    assert o.kernel_path == 0 and o.max_wait_spins == 1 << 26
+
+
+@pytest.mark.parametrize("bucket,code", [
+    ((1, 256, 128, 32), dion.OK),
+    ((0, 256, 128, 32), dion.ERR_INVALID_ARG),
+    ((1, 256, 128, 24), dion.ERR_UNSUPPORTED_SHAPE),     # r % 16
+    ((1, 256, 132, 32), dion.ERR_UNSUPPORTED_SHAPE),     # n % 8
+    ((1, 16, 128, 32), dion.ERR_UNSUPPORTED_SHAPE),      # r > m
+    ((1, 256, 16, 32), dion.ERR_UNSUPPORTED_SHAPE),      # r > n
+    ((1, 256, 128, 0), dion.ERR_UNSUPPORTED_SHAPE),
+    ((1, 1 << 31, 128, 32), dion.ERR_UNSUPPORTED_SHAPE),  # too large
+])
+def test_init_shape_checks(bucket, code):
+    c, h, ws = _init([bucket])
+    assert c == code, dion.dion_last_error()
+    if c == dion.OK:
+        assert ws > 0
+        dion.dion_free(h)
+    else:
+        assert not h.value and dion.dion_last_error()
+
+
+@pytest.mark.parametrize("field,value", [("mu", 1.0), ("mu", -0.1), ("precision", 7),
+                                         ("orth_mode", 9), ("fallback_cond", 0.5),
+                                         ("kernel_path", 3), ("max_wait_spins", 0)])
+def test_init_option_checks(field, value):
+    c, h, _ = _init([(1, 256, 128, 32)], **{field: value})
+    assert c == dion.ERR_INVALID_ARG
+
+
+def test_workspace_covers_the_layout():
+    c4 = [(128, 4096, 4096, 256), (64, 4096, 11008, 256), (32, 11008, 4096, 256)]
+    c, h, ws = _init(c4)
+    assert c == dion.OK
+    bf16_b = sum(k * m * n * 2 for k, m, n, r in c4)
+    factors = sum(k * (m * r * (4 * 3 + 2) + n * r * (4 + 2 + 2 + 2) + r * r * 8) for k, m, n, r in c4)
+    assert bf16_b + factors <= ws < 1.1 * (bf16_b + factors) + (1 << 24)
+    assert dion.dion_num_matrices(h) == 224
+    dion.dion_free(h)
+    c, h, ws32 = _init(c4, precision=0)
+    assert ws32 > ws                         # fp32 B copy
+    dion.dion_free(h)
+
+
+def test_step_argument_checks_without_device():
+    c, h, ws = _init([(2, 256, 128, 32)])
+    assert c == dion.OK
+    fake = 1 << 20                           # aligned, never dereferenced
+    ptrs = (dion.BucketPtrs * 1)()
+    ptrs[0].X = ptrs[0].M = ptrs[0].G = ptrs[0].Q = fake
+    step = dion.dion_step_batched
+    assert step(None, ptrs, 1, 0.01, fake, ws, None, None) == dion.ERR_NOT_INITIALIZED
+    assert step(h, None, 1, 0.01, fake, ws, None, None) == dion.ERR_INVALID_ARG
+    assert step(h, ptrs, 2, 0.01, fake, ws, None, None) == dion.ERR_INVALID_ARG
+    assert step(h, ptrs, 1, 0.01, None, ws, None, None) == dion.ERR_INVALID_ARG
+    assert step(h, ptrs, 1, 0.01, fake, ws - 1, None, None) == dion.ERR_WORKSPACE_TOO_SMALL
+    assert step(h, ptrs, 1, 0.01, fake + 8, ws, None, None) == dion.ERR_MISALIGNED
+    assert step(h, ptrs, 1, 0.01, fake, ws, fake + 2, None) == dion.ERR_MISALIGNED
+    ptrs[0].Q = fake + 4
+    assert step(h, ptrs, 1, 0.01, fake, ws, None, None) == dion.ERR_MISALIGNED
+    ptrs[0].Q = None
+    assert step(h, ptrs, 1, 0.01, fake, ws, None, None) == dion.ERR_INVALID_ARG
+    ptrs[0].Q = fake
+    try:
+        import torch
+        no_gpu = not torch.cuda.is_available()
+    except Exception:
+        no_gpu = True
+    if no_gpu:                               # valid arguments reach the device check
+        assert step(h, ptrs, 1, 0.01, fake, ws, None, None) in (dion.ERR_CUDA, dion.ERR_DEVICE)
+    assert dion.dion_free(h) == dion.OK
+
+
+def test_status_strings_and_views():
+    for code in range(8):
+        assert dion.dion_status_string(code)
+    c, h, ws = _init([(3, 64, 32, 16)])
+    ptr, nb = ctypes.c_void_p(), ctypes.c_size_t()
+    assert dion.dion_workspace_view(h, 0, dion.VIEW_P, 1 << 20, ctypes.byref(ptr),
+                                    ctypes.byref(nb)) == dion.OK
+    assert nb.value == 3 * 64 * 16 * 4 and ptr.value >= 1 << 20
+    assert dion.dion_workspace_view(h, 1, dion.VIEW_P, 1 << 20, ctypes.byref(ptr),
+                                    ctypes.byref(nb)) == dion.ERR_INVALID_ARG
+    assert dion.dion_last_launch_count(h) == 0
+    dion.dion_free(h)

@@ -1,0 +1,76 @@
+"""Host logic of bench.py: rank reduction over gloo (world size 2), roofline figures,
+and the oracle arm's JSON line."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import workloads as W  # noqa: E402
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, w = bench.dist_setup("gloo")
+    bench.barrier()
+    got = bench.max_over_ranks(1.5 + r)
+    rate = bench.whole_job_rate(100.0, w, got)
+    out.put((r, w, got, rate))
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[2] for r in res] == [2.5, 2.5]          # the slowest rank's time on both
+    assert [r[3] for r in res] == [80.0, 80.0]        # 2 ranks x 100 units / 2.5 s
+
+
+def test_single_process_reduction_is_identity():
+    assert bench.max_over_ranks(3.25) == 3.25
+    assert bench.whole_job_rate(10.0, 1, 2.0) == 5.0
+
+
+def test_algorithmic_figures_of_7b_shapes():
+    wl = W.WORKLOADS[W.HEADLINE]
+    flops, bytes_, upd = bench.algorithmic(wl)
+    assert wl.params == 6_476_005_376
+    assert abs(flops / 1.35e13 - 1) < 0.01
+    assert abs(bytes_ / 219.1e9 - 1) < 0.01
+    assert upd == 20 * wl.params
+
+
+def test_reference_arm_prints_one_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "single_256x128_r32", "--steps", "2", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "params/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "single_256x128_r32", "--steps", "1", "--warmup", "0"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert out.returncode == 0 and out.stdout.strip() == ""

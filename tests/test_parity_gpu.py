@@ -1,0 +1,229 @@
+"""Parity of the CUDA Dion step with the fp64 oracle on every workload (GPU).
+
+Tolerances (relative Frobenius error per matrix, max over the checked matrices):
+  fp32 contractions   X and M <= 1e-4 after the step count of the workload
+  bf16-input GEMMs    X and M <= 2e-2
+  every matrix        max |P^T P - I| <= 1e-4 on the GPU's own P
+The weight change dX = X_T - X_0 is checked too, since X_0 dominates X.  Its bound
+follows from the operand rounding: bf16 operands carry a relative error up to 2^-8 per
+product, and fp32 ones 2^-23 amplified by the subspace conditioning (fp32: 1e-3,
+bf16: 6e-2 on the full step count).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from parity_harness import GpuRun, compare, oracle_slot, update_norm_error
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"fp32": 1e-4, "bf16": 2e-2}
+TOL_DX = {"fp32": 1e-3, "bf16": 6e-2}
+ORTH_TOL = 1e-4
+
+
+def _check(rep, precision, dx=True):
+    print(rep)
+    assert rep.rel_x <= TOL[precision], rep
+    assert rep.rel_m <= TOL[precision], rep
+    assert rep.orth_gpu <= ORTH_TOL, rep
+    if dx:
+        assert rep.rel_dx <= TOL_DX[precision], rep
+    assert not rep.status_or & (4 | 8), rep      # no non-finite Gram, no timeout
+
+
+@pytest.mark.parametrize("path", ["tensor", "simt"])
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_single_256x128_r32(path, precision):
+    wl = W.WORKLOADS["single_256x128_r32"]
+    run = GpuRun(wl, precision=precision, kernel_path=path)
+    rep = compare(run, wl.steps)
+    _check(rep, precision)
+
+
+@pytest.mark.parametrize("path", ["tensor", "simt"])
+def test_fullrank_16x1024_polar(path):
+    """Full rank on a fixed B: M' = mu B exactly, and the distance of P Q^T to the polar
+    factor U V^T follows the oracle's curve over 50 steps."""
+    wl = W.WORKLOADS["fullrank_16x1024x1024"]
+    run = GpuRun(wl, kernel_path=path)
+    checkpoints = [1, 5, 10, 20, 50]
+    slots = [0, 15]
+    svd = {s: W.fixed_b_svd(wl, 0, s) for s in slots}
+    polar = {s: (u @ v.T) for s, (u, _, v) in svd.items()}
+    gpu_curve = {s: [] for s in slots}
+    done = 0
+    for c in checkpoints:
+        run.step(c - done)
+        done = c
+        P = run.P(0)
+        for s in slots:
+            pq = P[s].double().cpu() @ run.Q[0][s].double().cpu().T
+            gpu_curve[s].append((torch.linalg.norm(pq - polar[s]) / torch.linalg.norm(polar[s])).item())
+        if c == 10:
+            for s in slots:
+                B = W.gradient(wl, 0, 0, run.gen, slots=[s])[0].double()
+                rel = (torch.linalg.norm(run.M[0][s].double().cpu() - wl.mu * B) /
+                       torch.linalg.norm(wl.mu * B)).item()
+                assert rel <= TOL["fp32"], rel
+    for s in slots:
+        X0 = W.weights(wl, 0, run.gen, slots=[s])[0].double().numpy()
+        Q = W.right_factor(wl, 0, run.gen, slots=[s])[0].double().numpy()
+        B = W.gradient(wl, 0, 0, run.gen, slots=[s])[0].double().numpy()
+        X, M = X0, np.zeros_like(B)
+        curve, t = [], 0
+        for c in checkpoints:
+            while t < c:
+                X, M, Q, P, R = oracle.dion_step(X, np.zeros_like(B), B, Q, wl.mu, wl.lr)
+                t += 1
+            curve.append(np.linalg.norm(P @ Q.T - polar[s].numpy()) / np.linalg.norm(polar[s].numpy()))
+        print("slot", s, "oracle", np.round(curve, 6), "gpu", np.round(gpu_curve[s], 6))
+        assert np.abs(np.array(curve) - np.array(gpu_curve[s])).max() <= 1e-4
+        assert oracle.rel_fro(run.X[0][s].double().cpu().numpy(), X) <= TOL["fp32"]
+        assert oracle.rel_fro(run.M[0][s].double().cpu().numpy(), M) <= TOL["fp32"]
+    assert run.orth_error() <= ORTH_TOL
+
+
+@pytest.mark.parametrize("path", ["tensor", "simt"])
+def test_transformer_h2048_l24(path):
+    wl = W.WORKLOADS["transformer_h2048_l24_r256"]
+    run = GpuRun(wl, kernel_path=path)
+    rep = compare(run, wl.steps, slots_per_bucket=wl.sample_slots)
+    _check(rep, "bf16")
+
+
+def test_transformer_h4096_l32_ff11008():
+    """The 7B-like workload at full size (224 matrices, 6.48e9 parameters)."""
+    wl = W.WORKLOADS["transformer_h4096_l32_ff11008_r256"]
+    run = GpuRun(wl, kernel_path="tensor")
+    rep = compare(run, wl.steps, slots_per_bucket=wl.sample_slots)
+    _check(rep, "bf16")
+
+
+@pytest.mark.parametrize("r,steps", [(64, 10), (512, 10), (2048, 3)])
+def test_square_8x8192_rank_sweep(r, steps):
+    wl = W.WORKLOADS[f"square_8x8192_r{r}"]
+    run = GpuRun(wl)
+    rep = compare(run, steps, slots_per_bucket=(0,))
+    _check(rep, "fp32")
+
+
+# ------------------------------------------------------------------ edge cases
+
+EDGE = [
+    ("ragged", [(3, 200, 136, 16), (2, 130, 72, 48)]),
+    ("tall_thin", [(2, 1000, 24, 16)]),
+    ("full_rank_square", [(2, 64, 64, 64)]),
+    ("wide", [(2, 48, 520, 32)]),
+    ("many_small", [(300, 32, 16, 16)]),
+]
+
+
+@pytest.mark.parametrize("path", ["tensor", "simt"])
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+@pytest.mark.parametrize("name,buckets", EDGE, ids=[e[0] for e in EDGE])
+def test_edge_shapes(name, buckets, precision, path):
+    wl = W.custom(f"edge_{name}", buckets, precision=precision, steps=4)
+    run = GpuRun(wl, kernel_path=path)
+    X_before = [x.clone() for x in run.X]
+    rep = compare(run, 4)
+    _check(rep, precision, dx=False)
+
+
+@pytest.mark.parametrize("mode,bit", [("householder", 1), ("cholqr2", 2), ("cholqr", 0)])
+def test_orth_modes(mode, bit):
+    wl = W.custom(f"orth_{mode}", [(3, 256, 128, 32), (2, 300, 64, 48)], precision="fp32", steps=5)
+    run = GpuRun(wl, orth_mode=mode)
+    rep = compare(run, 5)
+    _check(rep, "fp32")
+    st = run.status.cpu().numpy()
+    if bit:
+        assert np.all(st & bit), st
+
+
+def test_update_norm_is_lr_s_sqrt_r():
+    """||X' - X||_F = lr sqrt(m/n) sqrt(r) for orthonormal P and unit-column Q."""
+    for precision, tol in (("fp32", 1e-5), ("bf16", 1e-2)):
+        wl = W.custom(f"norm_{precision}", [(4, 512, 256, 64), (2, 256, 512, 32)],
+                      precision=precision, steps=1)
+        run = GpuRun(wl)
+        for _ in range(3):
+            before = [x.clone() for x in run.X]
+            run.step(1)
+            assert update_norm_error(run, before) <= tol
+
+
+def test_zero_gradient_gives_zero_update():
+    wl = W.custom("zero", [(2, 128, 64, 16)], precision="fp32", steps=1)
+    run = GpuRun(wl)
+    X0 = run.X[0].clone()
+    run.step(1, G_override=[torch.zeros_like(run.X[0])])
+    assert torch.equal(run.X[0], X0)
+    assert torch.count_nonzero(run.M[0]) == 0 and torch.count_nonzero(run.Q[0]) == 0
+    st = run.status.cpu().numpy()
+    assert np.all(st & 16), st            # zero columns reported
+    assert not np.any(st & 8)
+
+
+def test_nonfinite_gradient_is_reported_and_contained():
+    wl = W.custom("nan", [(3, 128, 64, 16)], precision="fp32", steps=1)
+    run = GpuRun(wl)
+    G = W.gradient(wl, 0, 0).cuda()
+    G[1, 5, 7] = float("nan")
+    X_ok = run.X[0][[0, 2]].clone()
+    run.step(1, G_override=[G])
+    st = run.status.cpu().numpy()
+    assert st[1] & 4 and not (st[0] & 4) and not (st[2] & 4), st
+    for s in (0, 2):
+        X0, X, M, Q, P = oracle_slot(wl, 0, s, 1, "cpu")
+        assert oracle.rel_fro(run.X[0][s].double().cpu().numpy(), X) <= TOL["fp32"]
+
+
+def test_deterministic_and_resumable():
+    """Two runs are bitwise equal, and 3 + 3 steps through a saved state equal 6 steps."""
+    wl = W.custom("det", [(4, 384, 256, 32), (3, 256, 512, 48)], precision="bf16", steps=6)
+    a = GpuRun(wl)
+    a.step(6)
+    b = GpuRun(wl)
+    b.step(6)
+    for i in range(2):
+        assert torch.equal(a.X[i], b.X[i]) and torch.equal(a.M[i], b.M[i])
+        assert torch.equal(a.Q[i], b.Q[i])
+    c = GpuRun(wl)
+    c.step(3)
+    saved = [(x.cpu(), m.cpu(), q.cpu()) for x, m, q in zip(c.X, c.M, c.Q)]
+    del c
+    d = GpuRun(wl)
+    for i, (x, m, q) in enumerate(saved):
+        d.X[i].copy_(x); d.M[i].copy_(m); d.Q[i].copy_(q)
+    d.t = 3
+    d.step(3)
+    for i in range(2):
+        assert torch.equal(a.X[i], d.X[i]) and torch.equal(a.M[i], d.M[i])
+
+
+def test_tensor_and_simt_paths_agree():
+    wl = W.custom("paths", [(6, 1024, 512, 64), (4, 512, 1024, 128)], precision="bf16", steps=3)
+    a = GpuRun(wl, kernel_path="tensor")
+    b = GpuRun(wl, kernel_path="simt")
+    a.step(3)
+    b.step(3)
+    for i in range(2):
+        dm = (a.M[i] - b.M[i]).norm() / b.M[i].norm()
+        dx = ((a.X[i] - a.X0[i]) - (b.X[i] - b.X0[i])).norm() / (b.X[i] - b.X0[i]).norm()
+        print(i, dm.item(), dx.item())
+        assert dm <= 1e-3 and dx <= 1e-2
+
+
+def test_launch_count_and_profile():
+    wl = W.custom("prof", [(2, 256, 128, 32), (1, 128, 256, 16)], precision="bf16", steps=1)
+    run = GpuRun(wl)
+    run.opt.profile_enable(True)
+    run.step(2)
+    prof = run.opt.profile_read()
+    assert run.opt.last_launch_count > 0
+    assert all(v[0] > 0 and v[1] > 0 for v in prof.values()), prof
