@@ -1,26 +1,629 @@
-// Tensor-core kernels (placeholder entries until the tcgen05 kernels land).
+// Tensor-core kernels of the batched Dion step for sm_100a: tcgen05.mma with
+// accumulators in TMEM, operands staged in shared memory by TMA (128-byte
+// swizzle), persistent CTAs over all tiles of a bucket, warp-specialised:
+//   warp 0        TMA producer of the MMA operands
+//   warp 1        MMA issuer (one thread)
+//   warp 2        TMEM allocator; in the update kernel also the TMA producer
+//                 of the M, G, X slabs
+//   warps 4..7    epilogue (TMEM lanes 0..127)
+// Two TMEM accumulators let the epilogue of one tile overlap the MMAs of the
+// next.  Every wait is bounded (max_spins); on give-up the CTA drains what it
+// issued, marks DION_MAT_TIMEOUT on the matrices it did not finish, frees its
+// TMEM and returns.
+//
+// gemm (step 2 and 4 of the Dion step, the two halves of one power-iteration
+// step, rivista.ai Dion article paragraph 5):
+//   P0[b] = B[b] Q[b]     A = B (m x n, K-major),   B-operand = Q^T (r x n, K-major)
+//   R[b]  = B[b]^T P[b]   A = B^T (MN-major view),  B-operand = P (m x r, MN-major)
+// update (steps 5 and 7, error feedback of paragraph 3 and the weight step):
+//   acc = P [R | Q]^T per 128 x 128 tile (one N = 256 MMA), then
+//   M <- (M + G) - (1 - mu) acc_R,  X <- X - lr s acc_Q, with M, G, X streamed
+//   through shared memory by TMA in 128 x 32 slabs and M, X stored by TMA.
+#include <cuda.h>
+
+#include "common.cuh"
 #include "tc.h"
+#include "tc_ptx.cuh"
 
 namespace dion {
+namespace tc {
 
-cudaError_t tc_gemm_bq(const void*, const void*, float*, int, int64_t, int64_t, int64_t, int64_t,
-                       int32_t*, cudaStream_t, int* nlaunch, bool* done) {
-  *nlaunch = 0;
-  *done = false;
-  return cudaSuccess;
+constexpr int BM = 128;       // tile rows = TMEM lanes
+constexpr int BK = 64;        // bf16 elements per 128-byte swizzle row
+constexpr int NT = 256;       // threads per CTA
+constexpr int UPD_BN = 128;   // update tile columns (acc uses 2 * UPD_BN TMEM columns)
+constexpr int SLAB = 32;      // update epilogue slab width (fp32: 128 bytes)
+constexpr int SLAB_STAGES = 2;
+constexpr int UPD_STAGES = 2;
+
+// ------------------------------------------------------------------ host: tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
 }
-cudaError_t tc_gemm_btp(const void*, const void*, float*, int, int64_t, int64_t, int64_t, int64_t,
-                        int32_t*, cudaStream_t, int* nlaunch, bool* done) {
-  *nlaunch = 0;
-  *done = false;
-  return cudaSuccess;
+
+// 3-D map over a stack [d2][d1][d0] of row-major matrices, box {b0, b1, 1}.
+static bool map3d(CUtensorMap* m, const void* base, bool bf16, uint64_t d0, uint64_t d1,
+                  uint64_t d2, uint32_t b0, uint32_t b1) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  const uint64_t es = bf16 ? 2 : 4;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * es, d0 * d1 * es};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return f(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+           const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-cudaError_t tc_update(const void*, const void*, const void*, const float*, float*, float*, int,
-                      int64_t, int64_t, int64_t, float, float, int64_t, int32_t*, cudaStream_t,
-                      int* nlaunch, bool* done) {
+
+static int sm_count() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
+// ------------------------------------------------------------------ device: timeouts
+// Mark DION_MAT_TIMEOUT on every matrix owning a tile from `t` on (this CTA's share).
+__device__ void mark_unfinished(int32_t* flags, int t, int ntiles, int tiles_per_mat) {
+  int last = -1;
+  for (; t < ntiles; t += gridDim.x) {
+    const int b = t / tiles_per_mat;
+    if (b != last) {
+      atomicOr(flags + b, F_TIMEOUT);
+      last = b;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ batched GEMM
+struct GemmP {
+  int64_t M, N, K;
+  int batch, tiles_m, tiles_n, num_kb, block_n, stages;
+  uint32_t idesc, a_bytes, b_bytes, tmem_cols, acc_stride;
+  float* C;
+  int64_t ldc, c_bs;
+  int32_t* flags;
+  int64_t max_spins;
+};
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(NT, 1)
+    k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const GemmP p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + (size_t)p.stages * p.a_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + (size_t)p.stages * p.b_bytes);
+  uint64_t* empty = full + p.stages;
+  uint64_t* tfull = empty + p.stages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_per_mat = p.tiles_m * p.tiles_n;
+  const int ntiles = p.batch * tiles_per_mat;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull + a, 1);
+      mbar_init(tempty + a, 4);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    prefetch_map(&tmA);
+    prefetch_map(&tmB);
+    int stage = 0;
+    uint32_t phase = 0;
+    int used = 0;  // stages issued at least once
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const int b = t / tiles_per_mat;
+      const int rem = t % tiles_per_mat;
+      const int m0 = (rem / p.tiles_n) * BM;
+      const int n0 = (rem % p.tiles_n) * p.block_n;
+      bool ok = true;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!wait_bounded(empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
+        mbar_expect_tx(full + stage, p.a_bytes + p.b_bytes);
+        uint8_t* a_dst = sA + (size_t)stage * p.a_bytes;
+        uint8_t* b_dst = sB + (size_t)stage * p.b_bytes;
+        const int k0 = kb * BK;
+        if (A_MN) {  // A = B^T: boxes of 64 (M, along n) x 64 (K, along m)
+          tma_load_3d(a_dst, &tmA, full + stage, m0, k0, b);
+          tma_load_3d(a_dst + 8192, &tmA, full + stage, m0 + 64, k0, b);
+        } else {     // A rows along M, 64 K elements each
+          tma_load_3d(a_dst, &tmA, full + stage, k0, m0, b);
+        }
+        if (B_MN) {  // B-operand = P (K x N): boxes of 64 N x 64 K
+          for (int j = 0; j < p.block_n / 64; ++j)
+            tma_load_3d(b_dst + j * 8192, &tmB, full + stage, n0 + 64 * j, k0, b);
+        } else {     // B-operand rows along N, 64 K elements each
+          tma_load_3d(b_dst, &tmB, full + stage, k0, n0, b);
+        }
+        if (used < p.stages) ++used;
+        if (++stage == p.stages) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+    if (*abort) {
+      // let every load already issued land before the CTA goes away
+      for (int i = 0; i < used; ++i) {
+        stage = (stage + p.stages - 1) % p.stages;
+        if (stage == p.stages - 1) phase ^= 1;
+        wait_drain(full + stage, phase);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int lt = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      const uint32_t acc_phase = (lt >> 1) & 1;
+      if (!wait_bounded(tempty + acc, acc_phase ^ 1, p.max_spins, abort)) break;
+      tc_fence_after();
+      const uint32_t d = tmem + acc * p.acc_stride;
+      bool ok = true;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!wait_bounded(full + stage, phase, p.max_spins, abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + (size_t)stage * p.a_bytes);
+        const uint32_t b_base = smem_u32(sB + (size_t)stage * p.b_bytes);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          const uint64_t ad = A_MN ? sw128_desc(a_base + k * 2048, 8192, 1024)
+                                   : sw128_desc(a_base + k * 32, 16, 1024);
+          const uint64_t bd = B_MN ? sw128_desc(b_base + k * 2048, 8192, 1024)
+                                   : sw128_desc(b_base + k * 32, 16, 1024);
+          mma_bf16(d, ad, bd, p.idesc, (kb | k) != 0);
+        }
+        mma_commit(empty + stage);
+        if (++stage == p.stages) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      mma_commit(tfull + acc);
+    }
+    mma_commit(drain);
+    wait_drain(drain, 0);
+  } else if (warp >= 4) {
+    // ---------------- epilogue: TMEM -> registers -> global fp32
+    const int ew = warp - 4;
+    int lt = 0;
+    int t = blockIdx.x;
+    for (; t < ntiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      const uint32_t acc_phase = (lt >> 1) & 1;
+      if (!wait_bounded(tfull + acc, acc_phase, p.max_spins, abort)) break;
+      tc_fence_after();
+      const int b = t / tiles_per_mat;
+      const int rem = t % tiles_per_mat;
+      const int64_t row = (int64_t)(rem / p.tiles_n) * BM + ew * 32 + lane;
+      const int64_t n0 = (int64_t)(rem % p.tiles_n) * p.block_n;
+      float* crow = p.C + (int64_t)b * p.c_bs + row * p.ldc;
+      const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * p.acc_stride;
+      for (int c = 0; c < p.block_n; c += 16) {
+        float v[16];
+        tmem_ld16(tbase + c, v);
+        tmem_wait_ld();
+        if (row < p.M && n0 + c < p.N) {
+          float4* dst = reinterpret_cast<float4*>(crow + n0 + c);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty + acc);
+    }
+    if (t < ntiles && lane == 0) mark_unfinished(p.flags, t, ntiles, tiles_per_mat);
+  }
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+static uint32_t pow2_cols(uint32_t c) {
+  uint32_t v = 32;
+  while (v < c) v <<= 1;
+  return v;
+}
+
+template <bool A_MN, bool B_MN>
+static cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, GemmP p,
+                               cudaStream_t s) {
+  p.a_bytes = BM * BK * 2;
+  p.b_bytes = (uint32_t)p.block_n * BK * 2;
+  const size_t stage_bytes = p.a_bytes + p.b_bytes;
+  int stages = (int)((200 * 1024) / stage_bytes);
+  if (stages > 8) stages = 8;
+  if (stages < 2) stages = 2;
+  p.stages = stages;
+  p.acc_stride = (uint32_t)p.block_n;
+  p.tmem_cols = pow2_cols(2 * p.block_n);
+  const size_t smem = 1024 + stages * stage_bytes + (2 * stages + 5) * 8 + 16;
+  auto kern = k_tc_gemm<A_MN, B_MN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int ntiles = p.batch * p.tiles_m * p.tiles_n;
+  const int grid = ntiles < sm_count() ? ntiles : sm_count();
+  kern<<<grid, NT, smem, s>>>(ma, mb, p);
+  return cudaGetLastError();
+}
+
+static int pick_block_n(int64_t r, int mult) {
+  const int64_t tiles = (r + 255) / 256;
+  int64_t bn = (r + tiles - 1) / tiles;
+  bn = (bn + mult - 1) / mult * mult;
+  return (int)bn;
+}
+
+}  // namespace tc
+
+cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, int count, int64_t m, int64_t n,
+                       int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
+                       bool* done) {
+  using namespace tc;
   *nlaunch = 0;
   *done = false;
-  return cudaSuccess;
+  const int bn = pick_block_n(r, 16);
+  CUtensorMap ma, mb;
+  if (!map3d(&ma, Bg, true, n, m, count, BK, BM)) return cudaSuccess;
+  if (!map3d(&mb, Qg, true, n, r, count, BK, bn)) return cudaSuccess;
+  GemmP p{};
+  p.M = m; p.N = r; p.K = n;
+  p.batch = count;
+  p.block_n = bn;
+  p.tiles_m = (int)((m + BM - 1) / BM);
+  p.tiles_n = (int)((r + bn - 1) / bn);
+  p.num_kb = (int)((n + BK - 1) / BK);
+  p.idesc = idesc_bf16(BM, bn, false, false);
+  p.C = P0; p.ldc = r; p.c_bs = m * r;
+  p.flags = flags;
+  p.max_spins = max_spins;
+  cudaError_t e = launch_gemm<false, false>(ma, mb, p, s);
+  if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
+  return e;
+}
+
+cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, int count, int64_t m, int64_t n,
+                        int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
+                        bool* done) {
+  using namespace tc;
+  *nlaunch = 0;
+  *done = false;
+  const int bn = pick_block_n(r, 64);
+  if (r % 64 != 0 || bn % 64 != 0) return cudaSuccess;  // MN-major B needs whole 64-wide atoms
+  CUtensorMap ma, mb;
+  if (!map3d(&ma, Bg, true, n, m, count, 64, BK)) return cudaSuccess;
+  if (!map3d(&mb, Pg, true, r, m, count, 64, BK)) return cudaSuccess;
+  GemmP p{};
+  p.M = n; p.N = r; p.K = m;
+  p.batch = count;
+  p.block_n = bn;
+  p.tiles_m = (int)((n + BM - 1) / BM);
+  p.tiles_n = (int)((r + bn - 1) / bn);
+  p.num_kb = (int)((m + BK - 1) / BK);
+  p.idesc = idesc_bf16(BM, bn, true, true);
+  p.C = R; p.ldc = r; p.c_bs = n * r;
+  p.flags = flags;
+  p.max_spins = max_spins;
+  cudaError_t e = launch_gemm<true, true>(ma, mb, p, s);
+  if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
+  return e;
+}
+
+namespace tc {
+
+// ------------------------------------------------------------------ fused update
+struct UpdP {
+  int64_t m, n;
+  int batch, tiles_m, tiles_n, num_kb;
+  float omm, lrs;  // 1 - mu, lr * s
+  int32_t* flags;
+  int64_t max_spins;
+};
+
+constexpr uint32_t UPD_A_BYTES = BM * BK * 2;           // 16 KB
+constexpr uint32_t UPD_B_BYTES = 2 * UPD_BN * BK * 2;   // 32 KB (R rows then Q rows)
+constexpr uint32_t SLAB_BYTES = BM * SLAB * 4;          // 16 KB per tensor
+constexpr size_t UPD_SMEM = 1024 + UPD_STAGES * (UPD_A_BYTES + UPD_B_BYTES) +
+                            SLAB_STAGES * 3 * SLAB_BYTES + 256;
+
+__global__ void __launch_bounds__(NT, 1)
+    k_tc_update(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmR,
+                const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmM,
+                const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmX,
+                const __grid_constant__ CUtensorMap tmMs, const __grid_constant__ CUtensorMap tmXs,
+                const UpdP p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + UPD_STAGES * UPD_A_BYTES;
+  uint8_t* sS = sB + UPD_STAGES * UPD_B_BYTES;  // [stage][M | G | X] slabs
+  uint64_t* full = reinterpret_cast<uint64_t*>(sS + SLAB_STAGES * 3 * SLAB_BYTES);
+  uint64_t* empty = full + UPD_STAGES;
+  uint64_t* sfull = empty + UPD_STAGES;
+  uint64_t* sempty = sfull + SLAB_STAGES;
+  uint64_t* tfull = sempty + SLAB_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_per_mat = p.tiles_m * p.tiles_n;
+  const int ntiles = p.batch * tiles_per_mat;
+  constexpr int NSLAB = UPD_BN / SLAB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < UPD_STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int s = 0; s < SLAB_STAGES; ++s) {
+      mbar_init(sfull + s, 1);
+      mbar_init(sempty + s, 4);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull + a, 1);
+      mbar_init(tempty + a, 4);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 3) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- operand producer: P tile and the R, Q rows of the tile
+    prefetch_map(&tmP);
+    prefetch_map(&tmR);
+    prefetch_map(&tmQ);
+    int stage = 0, used = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const int b = t / tiles_per_mat;
+      const int rem = t % tiles_per_mat;
+      const int m0 = (rem / p.tiles_n) * BM;
+      const int n0 = (rem % p.tiles_n) * UPD_BN;
+      bool ok = true;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!wait_bounded(empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
+        mbar_expect_tx(full + stage, UPD_A_BYTES + UPD_B_BYTES);
+        uint8_t* a_dst = sA + stage * UPD_A_BYTES;
+        uint8_t* b_dst = sB + stage * UPD_B_BYTES;
+        tma_load_3d(a_dst, &tmP, full + stage, kb * BK, m0, b);
+        tma_load_3d(b_dst, &tmR, full + stage, kb * BK, n0, b);
+        tma_load_3d(b_dst + UPD_BN * BK * 2, &tmQ, full + stage, kb * BK, n0, b);
+        if (used < UPD_STAGES) ++used;
+        if (++stage == UPD_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+    if (*abort)
+      for (int i = 0; i < used; ++i) {
+        stage = (stage + UPD_STAGES - 1) % UPD_STAGES;
+        if (stage == UPD_STAGES - 1) phase ^= 1;
+        wait_drain(full + stage, phase);
+      }
+  } else if (warp == 2 && lane == 0) {
+    // ---------------- slab producer: M, G, X in 128 x 32 fp32 slabs
+    prefetch_map(&tmM);
+    prefetch_map(&tmG);
+    prefetch_map(&tmX);
+    int stage = 0, used = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const int b = t / tiles_per_mat;
+      const int rem = t % tiles_per_mat;
+      const int m0 = (rem / p.tiles_n) * BM;
+      const int n0 = (rem % p.tiles_n) * UPD_BN;
+      bool ok = true;
+      for (int sl = 0; sl < NSLAB; ++sl) {
+        if (!wait_bounded(sempty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
+        mbar_expect_tx(sfull + stage, 3 * SLAB_BYTES);
+        uint8_t* dst = sS + stage * 3 * SLAB_BYTES;
+        const int c0 = n0 + sl * SLAB;
+        tma_load_3d(dst, &tmM, sfull + stage, c0, m0, b);
+        tma_load_3d(dst + SLAB_BYTES, &tmG, sfull + stage, c0, m0, b);
+        tma_load_3d(dst + 2 * SLAB_BYTES, &tmX, sfull + stage, c0, m0, b);
+        if (used < SLAB_STAGES) ++used;
+        if (++stage == SLAB_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+    if (*abort)
+      for (int i = 0; i < used; ++i) {
+        stage = (stage + SLAB_STAGES - 1) % SLAB_STAGES;
+        if (stage == SLAB_STAGES - 1) phase ^= 1;
+        wait_drain(sfull + stage, phase);
+      }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer: acc = P [R | Q]^T, M = 128, N = 256
+    constexpr uint32_t idesc = idesc_bf16(BM, 2 * UPD_BN, false, false);
+    int stage = 0;
+    uint32_t phase = 0;
+    int lt = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      if (!wait_bounded(tempty + acc, ((lt >> 1) & 1) ^ 1, p.max_spins, abort)) break;
+      tc_fence_after();
+      const uint32_t d = tmem + acc * 256;
+      bool ok = true;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!wait_bounded(full + stage, phase, p.max_spins, abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + stage * UPD_A_BYTES);
+        const uint32_t b_base = smem_u32(sB + stage * UPD_B_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          mma_bf16(d, sw128_desc(a_base + k * 32, 16, 1024), sw128_desc(b_base + k * 32, 16, 1024),
+                   idesc, (kb | k) != 0);
+        mma_commit(empty + stage);
+        if (++stage == UPD_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      mma_commit(tfull + acc);
+    }
+    mma_commit(drain);
+    wait_drain(drain, 0);
+  } else if (warp >= 4) {
+    // ---------------- epilogue: one TMEM lane (tile row) per thread
+    const int ew = warp - 4;
+    const int row = ew * 32 + lane;  // row inside the tile
+    int stage = 0;
+    uint32_t phase = 0;
+    int lt = 0;
+    int t = blockIdx.x;
+    bool ok = true;
+    for (; t < ntiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      if (!wait_bounded(tfull + acc, (lt >> 1) & 1, p.max_spins, abort)) break;
+      tc_fence_after();
+      const int b = t / tiles_per_mat;
+      const int rem = t % tiles_per_mat;
+      const int m0 = (rem / p.tiles_n) * BM;
+      const int n0 = (rem % p.tiles_n) * UPD_BN;
+      const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * 256;
+      for (int sl = 0; sl < NSLAB; ++sl) {
+        float ar[32], aq[32];
+        tmem_ld32(tbase + sl * SLAB, ar);
+        tmem_ld32(tbase + UPD_BN + sl * SLAB, aq);
+        tmem_wait_ld();
+        if (!wait_bounded(sfull + stage, phase, p.max_spins, abort)) { ok = false; break; }
+        uint8_t* slab = sS + stage * 3 * SLAB_BYTES;
+        uint8_t* rm = slab + row * 128;
+        uint8_t* rg = slab + SLAB_BYTES + row * 128;
+        uint8_t* rx = slab + 2 * SLAB_BYTES + row * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int off = ((c ^ (row & 7)) << 4);
+          float4 mv = *reinterpret_cast<float4*>(rm + off);
+          const float4 gv = *reinterpret_cast<const float4*>(rg + off);
+          float4 xv = *reinterpret_cast<float4*>(rx + off);
+          mv.x = (mv.x + gv.x) - p.omm * ar[4 * c + 0];
+          mv.y = (mv.y + gv.y) - p.omm * ar[4 * c + 1];
+          mv.z = (mv.z + gv.z) - p.omm * ar[4 * c + 2];
+          mv.w = (mv.w + gv.w) - p.omm * ar[4 * c + 3];
+          xv.x = xv.x - p.lrs * aq[4 * c + 0];
+          xv.y = xv.y - p.lrs * aq[4 * c + 1];
+          xv.z = xv.z - p.lrs * aq[4 * c + 2];
+          xv.w = xv.w - p.lrs * aq[4 * c + 3];
+          *reinterpret_cast<float4*>(rm + off) = mv;
+          *reinterpret_cast<float4*>(rx + off) = xv;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tmMs, slab + ew * 32 * 128, n0 + sl * SLAB, m0 + ew * 32, b);
+          tma_store_3d(&tmXs, slab + 2 * SLAB_BYTES + ew * 32 * 128, n0 + sl * SLAB, m0 + ew * 32, b);
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(sempty + stage);
+        }
+        __syncwarp();
+        if (++stage == SLAB_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;  // t stays on the unfinished tile
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty + acc);
+    }
+    if (lane == 0) bulk_wait0();
+    if (t < ntiles && lane == 0) mark_unfinished(p.flags, t, ntiles, tiles_per_mat);
+  }
+  __syncthreads();
+  if (warp == 3) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace tc
+
+cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, const float* G, float* M,
+                      float* X, int count, int64_t m, int64_t n, int64_t r, float mu, float lr_scale,
+                      int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch, bool* done) {
+  using namespace tc;
+  *nlaunch = 0;
+  *done = false;
+  if (r % 16 != 0) return cudaSuccess;
+  CUtensorMap mP, mR, mQ, mM, mG, mX, mMs, mXs;
+  bool ok = map3d(&mP, Pg, true, r, m, count, BK, BM) && map3d(&mR, Rg, true, r, n, count, BK, UPD_BN) &&
+            map3d(&mQ, Qg, true, r, n, count, BK, UPD_BN) &&
+            map3d(&mM, M, false, n, m, count, SLAB, BM) && map3d(&mG, G, false, n, m, count, SLAB, BM) &&
+            map3d(&mX, X, false, n, m, count, SLAB, BM) &&
+            map3d(&mMs, M, false, n, m, count, SLAB, 32) && map3d(&mXs, X, false, n, m, count, SLAB, 32);
+  if (!ok) return cudaSuccess;
+  UpdP p{};
+  p.m = m; p.n = n;
+  p.batch = count;
+  p.tiles_m = (int)((m + BM - 1) / BM);
+  p.tiles_n = (int)((n + UPD_BN - 1) / UPD_BN);
+  p.num_kb = (int)((r + BK - 1) / BK);
+  p.omm = 1.f - mu;
+  p.lrs = lr_scale;
+  p.flags = flags;
+  p.max_spins = max_spins;
+  cudaError_t e = cudaFuncSetAttribute(k_tc_update, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)UPD_SMEM);
+  if (e != cudaSuccess) return e;
+  const int ntiles = count * p.tiles_m * p.tiles_n;
+  const int grid = ntiles < sm_count() ? ntiles : sm_count();
+  k_tc_update<<<grid, NT, UPD_SMEM, s>>>(mP, mR, mQ, mM, mG, mX, mMs, mXs, p);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
+  return e;
 }
 
 }  // namespace dion

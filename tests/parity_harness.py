@@ -25,13 +25,14 @@ class Report:
     rel_m: float = 0.0
     rel_q: float = 0.0
     rel_dx: float = 0.0
+    dx_floor: float = 0.0          # fp32 rounding of the stored X, relative to ||dX||
     orth_gpu: float = 0.0          # max |P^T P - I| over every matrix of the GPU run
     status_or: int = 0
     per_slot: list = field(default_factory=list)
 
     def __str__(self):
         return (f"rel_F X {self.rel_x:.3e}  M {self.rel_m:.3e}  Q {self.rel_q:.3e}  "
-                f"dX {self.rel_dx:.3e}  |P^T P - I| {self.orth_gpu:.3e}  status {self.status_or}")
+                f"dX {self.rel_dx:.3e} (fp32 floor {self.dx_floor:.1e})  |P^T P - I| {self.orth_gpu:.3e}  status {self.status_or}")
 
 
 class GpuRun:
@@ -108,13 +109,19 @@ def compare(run: GpuRun, steps: int, slots_per_bucket=None) -> Report:
             gx = run.X[bi][s].double().cpu().numpy()
             gm = run.M[bi][s].double().cpu().numpy()
             gq = run.Q[bi][s].double().cpu().numpy()
+            # X is fp32 state: each step rounds every element by up to half an ulp, a noise
+            # floor of about 2^-24 ||X||_F sqrt(steps) in dX that no kernel can remove
+            floor = 2.0 ** -24 * np.linalg.norm(X0) * math.sqrt(steps) / max(
+                np.linalg.norm(X - X0), 1e-300)
             one = dict(bucket=bi, slot=s, rel_x=oracle.rel_fro(gx, X), rel_m=oracle.rel_fro(gm, M),
-                       rel_q=oracle.rel_fro(gq, Q), rel_dx=oracle.rel_fro(gx - X0, X - X0))
+                       rel_q=oracle.rel_fro(gq, Q), rel_dx=oracle.rel_fro(gx - X0, X - X0),
+                       dx_floor=floor)
             rep.per_slot.append(one)
             rep.rel_x = max(rep.rel_x, one["rel_x"])
             rep.rel_m = max(rep.rel_m, one["rel_m"])
             rep.rel_q = max(rep.rel_q, one["rel_q"])
             rep.rel_dx = max(rep.rel_dx, one["rel_dx"])
+            rep.dx_floor = max(rep.dx_floor, one["dx_floor"])
     rep.orth_gpu = run.orth_error()
     rep.status_or = int(np.bitwise_or.reduce(run.status.cpu().numpy()))
     return rep

@@ -5,9 +5,10 @@ Tolerances (relative Frobenius error per matrix, max over the checked matrices):
   bf16-input GEMMs    X and M <= 2e-2
   every matrix        max |P^T P - I| <= 1e-4 on the GPU's own P
 The weight change dX = X_T - X_0 is checked too, since X_0 dominates X.  Its bound
-follows from the operand rounding: bf16 operands carry a relative error up to 2^-8 per
-product, and fp32 ones 2^-23 amplified by the subspace conditioning (fp32: 1e-3,
-bf16: 6e-2 on the full step count).
+has two parts: the operand rounding (bf16 operands carry a relative error up to 2^-8
+per product, fp32 ones 2^-23 amplified by the subspace conditioning: fp32 1e-3, bf16
+6e-2 over the step count), plus the rounding of the fp32 state X itself, which every
+step perturbs by up to half an ulp per element: 3 x 2^-24 ||X_0||_F sqrt(T) / ||dX||_F.
 """
 import math
 
@@ -32,7 +33,7 @@ def _check(rep, precision, dx=True):
     assert rep.rel_m <= TOL[precision], rep
     assert rep.orth_gpu <= ORTH_TOL, rep
     if dx:
-        assert rep.rel_dx <= TOL_DX[precision], rep
+        assert rep.rel_dx <= TOL_DX[precision] + 3 * rep.dx_floor, rep
     assert not rep.status_or & (4 | 8), rep      # no non-finite Gram, no timeout
 
 

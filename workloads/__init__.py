@@ -89,6 +89,13 @@ WORKLOADS = {
             note="7B-like: 32 layers, hidden 4096, MLP 11008 (Wq/Wk/Wv/Wo, W_gate/W_up, W_down), "
                  "rank fraction 1/16",
             sample_slots=(0, -1)),
+        Workload(
+            name="stack_16x4096x4096_r256",
+            buckets=(Bucket(16, 4096, 4096, 256),),
+            precision="bf16", mu=0.95, lr=0.01, steps=3, grad="gaussian_1e-3",
+            note="16 attention-sized 4096x4096 matrices, rank 256: a 3 GB case for profiling "
+                 "(inputs larger than L2)",
+            sample_slots=(0, 15)),
     ] + [_sweep(r) for r in (64, 128, 256, 512, 1024, 2048, 4096, 8192)]
 }
 
