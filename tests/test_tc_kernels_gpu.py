@@ -2,8 +2,11 @@
 
 One step through each kernel path from the same state: P isolates B Q (the
 orthonormalisation that follows is the same code on both paths), R isolates B^T P,
-and M, X isolate the fused update.  Both paths round the same operands to bf16, so
-they differ only by fp32 accumulation order.
+and M, X isolate the fused update.  Both paths round B, Q, P, R to bf16 and differ by
+fp32 accumulation order, ~1e-6 relative in P.  Rounding P to bf16 then flips a
+fraction ~delta / 2^-8 of its entries by one bf16 ulp, which moves R, M and dX by about
+sqrt(delta * 2^-8) ~ 1e-4 (dX also inherits the flips of the bf16 R and Q).  A wrong
+tile, descriptor or swizzle gives errors of order 1.
 """
 import numpy as np
 import pytest
@@ -45,9 +48,9 @@ def test_tensor_views_match_simt(buckets):
         ex = _rel(a.X[i] - a.X0[i], b.X[i] - b.X0[i])
         print(bk, f"P {ep:.2e} R {er:.2e} M {em:.2e} dX {ex:.2e}")
         assert ep < 1e-4, ("B Q", ep)
-        assert er < 1e-4, ("B^T P", er)
-        assert em < 1e-5, ("update M", em)
-        assert ex < 1e-4, ("update X", ex)
+        assert er < 1e-3, ("B^T P", er)
+        assert em < 2e-4, ("update M", em)
+        assert ex < 2e-3, ("update X", ex)
     assert int(a.status.max()) & 12 == 0
 
 
