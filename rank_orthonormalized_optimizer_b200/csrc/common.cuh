@@ -33,6 +33,15 @@ template <> struct Cvt<bf16> {
 
 __device__ __forceinline__ bool finitef(float v) { return isfinite(v); }
 
+// x = h + m + l with h, m, l bf16: each part is the bf16 rounding of what the
+// earlier parts left over, so h + m + l carries about 24 significant bits of x.
+__device__ __forceinline__ void split3_bf16(float v, bf16& h, bf16& m, bf16& l) {
+  h = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(h);
+  m = __float2bfloat16_rn(r1);
+  l = __float2bfloat16_rn(r1 - __bfloat162float(m));
+}
+
 // Positive floats order like their bit patterns; used for atomic min/max.
 __device__ __forceinline__ void atomic_max_pos(float* a, float v) {
   atomicMax(reinterpret_cast<int*>(a), __float_as_int(v));

@@ -5,6 +5,7 @@
 // runs once per bucket over all of its matrices, as "DASH: Faster Shampoo via
 // Batched Block Preconditioning and Efficient Inverse-Root Solvers"
 // (Methodologie, section 1) stacks preconditioner blocks instead of looping.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -45,7 +46,7 @@ struct Plan {
   int64_t mat0;
   int nsplit;
   size_t off_Bg, off_Qg, off_P0, off_P, off_P2, off_Pg, off_W, off_Linv, off_dinv, off_R, off_Rg,
-      off_Qng, off_part, off_flags, off_stats;
+      off_Qng, off_part, off_flags, off_stats, off_P0s, off_Ps, off_Linvs;
 };
 
 struct EventPair {
@@ -156,6 +157,10 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
   float* part = reinterpret_cast<float*>(ws + p.off_part);
   int32_t* flags = reinterpret_cast<int32_t*>(ws + p.off_flags);
   float* stats = reinterpret_cast<float*>(ws + p.off_stats);
+  __nv_bfloat16* P0s = reinterpret_cast<__nv_bfloat16*>(ws + p.off_P0s);
+  __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ps);
+  __nv_bfloat16* Linvs = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Linvs);
+  bool p0s_ready = false;
   const int64_t m = p.m, n = p.n, r = p.r;
   const int cnt = p.count;
   cudaStream_t s = c.s;
@@ -179,9 +184,11 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
     bool done = false;
     if (tensor && bf) {
       int nl = 0;
-      cudaError_t e = dion::tc_gemm_bq(Bg, Qg, P0, cnt, m, n, r, o.max_wait_spins, flags, s, &nl, &done);
+      cudaError_t e = dion::tc_gemm_bq(Bg, Qg, P0, P0s, cnt, m, n, r, o.max_wait_spins, flags, s,
+                                       &nl, &done);
       c.launches += nl;
       if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_gemm_bq: %s", cudaGetErrorString(e));
+      p0s_ready = done;
     }
     if (!done) {
       dion::GemmDesc d{};
@@ -220,7 +227,42 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
     ca.W = W; ca.Linv = Linv; ca.dinv = dinv; ca.flags = flags; ca.stats = stats;
     ca.count = cnt; ca.r = r; ca.fallback_cond = o.fallback_cond;
     const int chol_launches = r <= 256 ? 1 : (int)(2 + 3 * ((r + 31) / 32) + (r + 31) / 32);
-    if (o.orth_mode != DION_ORTH_HOUSEHOLDER) {
+    const int64_t mr = (int64_t)cnt * m * r, rr = (int64_t)cnt * r * r;
+    // tensor cores: Gram and triangular apply from three-way bf16 splits (fp32-accurate)
+    auto tc_call = [&](cudaError_t e, int nl, bool done, const char* what) -> dion_status {
+      c.launches += nl;
+      if (e != cudaSuccess) return fail(DION_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+      if (!done) return fail(DION_ERR_CUDA, "%s: tensor map encoding failed", what);
+      return DION_OK;
+    };
+    if (o.orth_mode != DION_ORTH_HOUSEHOLDER && tensor) {
+      int nl = 0;
+      bool done = false;
+      dion_status st;
+      if (!p0s_ready) DION_LAUNCH(c, 1, dion::launch_split3(P0, P0s, mr, mr, s));
+      st = tc_call(dion::tc_gram(P0s, W, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins,
+                                 s, &nl, &done), nl, done, "tc_gram");
+      if (st != DION_OK) return st;
+      ca.pass = 1; ca.orth_tol = o.orth_tol;
+      DION_LAUNCH(c, chol_launches, dion::launch_chol_inv(ca, s));
+      DION_LAUNCH(c, 1, dion::launch_split3(Linv, Linvs, rr, rr, s));
+      st = tc_call(dion::tc_apply(P0s, Linvs, P, Ps, cnt, m, r, flags, 0, DION_MAT_FALLBACK,
+                                  o.max_wait_spins, s, &nl, &done), nl, done, "tc_apply");
+      if (st != DION_OK) return st;
+      if (o.orth_mode != DION_ORTH_CHOLQR) {
+        st = tc_call(dion::tc_gram(Ps, W, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins,
+                                   s, &nl, &done), nl, done, "tc_gram");
+        if (st != DION_OK) return st;
+        ca.pass = 2;
+        ca.orth_tol = o.orth_mode == DION_ORTH_CHOLQR2 ? -1.f : o.orth_tol;
+        DION_LAUNCH(c, chol_launches, dion::launch_chol_inv(ca, s));
+        DION_LAUNCH(c, 1, dion::launch_split3(Linv, Linvs, rr, rr, s));
+        st = tc_call(dion::tc_apply(Ps, Linvs, P2, nullptr, cnt, m, r, flags, DION_MAT_CHOLQR2,
+                                    DION_MAT_FALLBACK, o.max_wait_spins, s, &nl, &done),
+                     nl, done, "tc_apply");
+        if (st != DION_OK) return st;
+      }
+    } else if (o.orth_mode != DION_ORTH_HOUSEHOLDER) {
       DION_LAUNCH(c, gl, dion::launch_gemm_simt(gram(P0), false, s));
       ca.pass = 1; ca.orth_tol = o.orth_tol;
       DION_LAUNCH(c, chol_launches, dion::launch_chol_inv(ca, s));
@@ -407,6 +449,10 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
     p.off_part = take(c * p.nsplit * d.r * 4);
     p.off_flags = take(c * 4);
     p.off_stats = take(c * 8);
+    // three-way bf16 splits for the tensor-core orthonormalisation
+    p.off_P0s = take(c * d.m * d.r * 6);
+    p.off_Ps = take(c * d.m * d.r * 6);
+    p.off_Linvs = take(c * d.r * d.r * 6);
     plans.push_back(p);
   }
   dion_ctx* h = new (std::nothrow) dion_ctx();

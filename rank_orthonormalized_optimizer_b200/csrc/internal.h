@@ -40,6 +40,8 @@ cudaError_t launch_finalize_p(const float* P, const float* P2, void* Pg, bool us
 cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, bool use_bf16,
                            float* part, int nsplit, int32_t* flags, int count, int64_t n,
                            int64_t r, cudaStream_t s);
+cudaError_t launch_split3(const float* src, void* dst, int64_t n, int64_t dst_stride,
+                          cudaStream_t s);
 cudaError_t launch_write_status(const int32_t* flags, int32_t* d_status, int count,
                                 cudaStream_t s);
 

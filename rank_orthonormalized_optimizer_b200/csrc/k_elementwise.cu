@@ -103,6 +103,31 @@ cudaError_t launch_prep_q(const float* Q, void* Qg, bool use_bf16, int count, in
   return cudaGetLastError();
 }
 
+// ------------------------------------------------ three-way bf16 split of fp32
+// dst[i], dst[i + stride], dst[i + 2 stride] = the bf16 parts of src[i], for the
+// split-operand tensor-core contractions of the orthonormalisation.
+__global__ void __launch_bounds__(256) k_split3(const float* __restrict__ src,
+                                                 bf16* __restrict__ dst, int64_t n,
+                                                 int64_t stride) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    bf16 h, m, l;
+    split3_bf16(src[i], h, m, l);
+    dst[i] = h;
+    dst[i + stride] = m;
+    dst[i + 2 * stride] = l;
+  }
+}
+
+cudaError_t launch_split3(const float* src, void* dst, int64_t n, int64_t dst_stride,
+                          cudaStream_t s) {
+  int64_t grid = (n + 255) / 256;
+  if (grid > (int64_t)sm_count() * 8) grid = (int64_t)sm_count() * 8;
+  if (grid < 1) grid = 1;
+  k_split3<<<(unsigned)grid, 256, 0, s>>>(src, (bf16*)dst, n, dst_stride);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------- flags and status
 __global__ void k_init_flags(int32_t* flags, float* stats, int count, int32_t init_bits) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;

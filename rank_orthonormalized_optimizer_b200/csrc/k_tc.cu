@@ -96,15 +96,35 @@ __device__ void mark_unfinished(int32_t* flags, int t, int ntiles, int tiles_per
 }
 
 // ------------------------------------------------------------------ batched GEMM
+// C[b] = sum over pairs (i, j) of A_i[b] B_j[b], fp32 accumulation in TMEM.
+// One pair is a plain bf16 GEMM.  With operands split into three bf16 parts
+// (x = x0 + x1 + x2, each the bf16 rounding of what the earlier parts left),
+// the six pairs (0,0) (0,1) (1,0) (1,1) (0,2) (2,0) reproduce an fp32 product to
+// about 2^-24 relative: this keeps the Gram matrix and the triangular apply of
+// Cholesky-QR fp32-accurate on bf16 tensor cores.  A split operand is stored as
+// [3 * batch][rows][cols]; split i of matrix b is matrix i * batch + b.
+constexpr int MAX_PAIRS = 6;
+
 struct GemmP {
   int64_t M, N, K;
   int batch, tiles_m, tiles_n, num_kb, block_n, stages;
   uint32_t idesc, a_bytes, b_bytes, tmem_cols, acc_stride;
-  float* C;
+  int npairs;
+  int pa[MAX_PAIRS], pb[MAX_PAIRS];  // split index of A and of B per pair
+  float* C;                          // fp32 result (may be null)
   int64_t ldc, c_bs;
+  bf16* Cs;                          // three-way bf16 split of the result (may be null)
+  int64_t cs_stride;                 // elements between the split parts
   int32_t* flags;
+  int32_t need_mask, skip_mask;      // matrices whose flags fail this are skipped
   int64_t max_spins;
 };
+
+__device__ __forceinline__ bool tile_active(const GemmP& p, int b) {
+  if (p.need_mask == 0 && p.skip_mask == 0) return true;
+  const int32_t f = p.flags[b];
+  return (f & p.need_mask) == p.need_mask && !(f & p.skip_mask);
+}
 
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(NT, 1)
@@ -125,6 +145,7 @@ __global__ void __launch_bounds__(NT, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_per_mat = p.tiles_m * p.tiles_n;
   const int ntiles = p.batch * tiles_per_mat;
+  const int kiters = p.num_kb * p.npairs;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -157,27 +178,30 @@ __global__ void __launch_bounds__(NT, 1)
     int used = 0;  // stages issued at least once
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       const int b = t / tiles_per_mat;
+      if (!tile_active(p, b)) continue;
       const int rem = t % tiles_per_mat;
       const int m0 = (rem / p.tiles_n) * BM;
       const int n0 = (rem % p.tiles_n) * p.block_n;
       bool ok = true;
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+      for (int it = 0; it < kiters; ++it) {
+        const int kb = it / p.npairs, pi = it % p.npairs;
+        const int za = p.pa[pi] * p.batch + b, zb = p.pb[pi] * p.batch + b;
         if (!wait_bounded(empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
         mbar_expect_tx(full + stage, p.a_bytes + p.b_bytes);
         uint8_t* a_dst = sA + (size_t)stage * p.a_bytes;
         uint8_t* b_dst = sB + (size_t)stage * p.b_bytes;
         const int k0 = kb * BK;
-        if (A_MN) {  // A = B^T: boxes of 64 (M, along n) x 64 (K, along m)
-          tma_load_3d(a_dst, &tmA, full + stage, m0, k0, b);
-          tma_load_3d(a_dst + 8192, &tmA, full + stage, m0 + 64, k0, b);
-        } else {     // A rows along M, 64 K elements each
-          tma_load_3d(a_dst, &tmA, full + stage, k0, m0, b);
+        if (A_MN) {  // A^T stored [K][M]: boxes of 64 (M) x 64 (K)
+          tma_load_3d(a_dst, &tmA, full + stage, m0, k0, za);
+          tma_load_3d(a_dst + 8192, &tmA, full + stage, m0 + 64, k0, za);
+        } else {     // A stored [M][K]: 128 rows of 64 K elements
+          tma_load_3d(a_dst, &tmA, full + stage, k0, m0, za);
         }
-        if (B_MN) {  // B-operand = P (K x N): boxes of 64 N x 64 K
+        if (B_MN) {  // B stored [K][N]: boxes of 64 (N) x 64 (K)
           for (int j = 0; j < p.block_n / 64; ++j)
-            tma_load_3d(b_dst + j * 8192, &tmB, full + stage, n0 + 64 * j, k0, b);
-        } else {     // B-operand rows along N, 64 K elements each
-          tma_load_3d(b_dst, &tmB, full + stage, k0, n0, b);
+            tma_load_3d(b_dst + j * 8192, &tmB, full + stage, n0 + 64 * j, k0, zb);
+        } else {     // B stored [N][K]: block_n rows of 64 K elements
+          tma_load_3d(b_dst, &tmB, full + stage, k0, n0, zb);
         }
         if (used < p.stages) ++used;
         if (++stage == p.stages) { stage = 0; phase ^= 1; }
@@ -197,14 +221,15 @@ __global__ void __launch_bounds__(NT, 1)
     int stage = 0;
     uint32_t phase = 0;
     int lt = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      if (!tile_active(p, t / tiles_per_mat)) continue;
       const int acc = lt & 1;
       const uint32_t acc_phase = (lt >> 1) & 1;
       if (!wait_bounded(tempty + acc, acc_phase ^ 1, p.max_spins, abort)) break;
       tc_fence_after();
       const uint32_t d = tmem + acc * p.acc_stride;
       bool ok = true;
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+      for (int it = 0; it < kiters; ++it) {
         if (!wait_bounded(full + stage, phase, p.max_spins, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_base = smem_u32(sA + (size_t)stage * p.a_bytes);
@@ -215,46 +240,66 @@ __global__ void __launch_bounds__(NT, 1)
                                    : sw128_desc(a_base + k * 32, 16, 1024);
           const uint64_t bd = B_MN ? sw128_desc(b_base + k * 2048, 8192, 1024)
                                    : sw128_desc(b_base + k * 32, 16, 1024);
-          mma_bf16(d, ad, bd, p.idesc, (kb | k) != 0);
+          mma_bf16(d, ad, bd, p.idesc, (it | k) != 0);
         }
         mma_commit(empty + stage);
         if (++stage == p.stages) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
       mma_commit(tfull + acc);
+      ++lt;
     }
     mma_commit(drain);
     wait_drain(drain, 0);
   } else if (warp >= 4) {
-    // ---------------- epilogue: TMEM -> registers -> global fp32
+    // ---------------- epilogue: TMEM -> registers -> global (fp32 and/or bf16 split)
     const int ew = warp - 4;
     int lt = 0;
     int t = blockIdx.x;
-    for (; t < ntiles; t += gridDim.x, ++lt) {
+    for (; t < ntiles; t += gridDim.x) {
+      const int b = t / tiles_per_mat;
+      if (!tile_active(p, b)) continue;
       const int acc = lt & 1;
       const uint32_t acc_phase = (lt >> 1) & 1;
       if (!wait_bounded(tfull + acc, acc_phase, p.max_spins, abort)) break;
       tc_fence_after();
-      const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
       const int64_t row = (int64_t)(rem / p.tiles_n) * BM + ew * 32 + lane;
       const int64_t n0 = (int64_t)(rem % p.tiles_n) * p.block_n;
-      float* crow = p.C + (int64_t)b * p.c_bs + row * p.ldc;
+      const int64_t off = (int64_t)b * p.c_bs + row * p.ldc;
       const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * p.acc_stride;
       for (int c = 0; c < p.block_n; c += 16) {
         float v[16];
         tmem_ld16(tbase + c, v);
         tmem_wait_ld();
         if (row < p.M && n0 + c < p.N) {
-          float4* dst = reinterpret_cast<float4*>(crow + n0 + c);
+          if (p.C) {
+            float4* dst = reinterpret_cast<float4*>(p.C + off + n0 + c);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          }
+          if (p.Cs) {
+            __align__(16) bf16 h[16], mi[16], lo[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) split3_bf16(v[q], h[q], mi[q], lo[q]);
+            bf16* base = p.Cs + off + n0 + c;
+            uint4* d0 = reinterpret_cast<uint4*>(base);
+            uint4* d1 = reinterpret_cast<uint4*>(base + p.cs_stride);
+            uint4* d2 = reinterpret_cast<uint4*>(base + 2 * p.cs_stride);
+            const uint4* sh = reinterpret_cast<const uint4*>(h);
+            const uint4* sm = reinterpret_cast<const uint4*>(mi);
+            const uint4* sl = reinterpret_cast<const uint4*>(lo);
+            d0[0] = sh[0]; d0[1] = sh[1];
+            d1[0] = sm[0]; d1[1] = sm[1];
+            d2[0] = sl[0]; d2[1] = sl[1];
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + acc);
+      ++lt;
     }
     if (t < ntiles && lane == 0) mark_unfinished(p.flags, t, ntiles, tiles_per_mat);
   }
@@ -300,11 +345,21 @@ static int pick_block_n(int64_t r, int mult) {
   return (int)bn;
 }
 
+static void set_pairs(GemmP& p, int npairs) {
+  static const int A6[6] = {2, 0, 1, 1, 0, 0};  // small terms first
+  static const int B6[6] = {0, 2, 1, 0, 1, 0};
+  p.npairs = npairs;
+  for (int i = 0; i < npairs; ++i) {
+    p.pa[i] = npairs == 1 ? 0 : A6[i];
+    p.pb[i] = npairs == 1 ? 0 : B6[i];
+  }
+}
+
 }  // namespace tc
 
-cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, int count, int64_t m, int64_t n,
-                       int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
-                       bool* done) {
+cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, bf16* P0s, int count, int64_t m,
+                       int64_t n, int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s,
+                       int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
@@ -319,8 +374,10 @@ cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, int count, int
   p.tiles_m = (int)((m + BM - 1) / BM);
   p.tiles_n = (int)((r + bn - 1) / bn);
   p.num_kb = (int)((n + BK - 1) / BK);
+  set_pairs(p, 1);
   p.idesc = idesc_bf16(BM, bn, false, false);
   p.C = P0; p.ldc = r; p.c_bs = m * r;
+  p.Cs = P0s; p.cs_stride = (int64_t)count * m * r;
   p.flags = flags;
   p.max_spins = max_spins;
   cudaError_t e = launch_gemm<false, false>(ma, mb, p, s);
@@ -334,8 +391,7 @@ cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, int count, int
   using namespace tc;
   *nlaunch = 0;
   *done = false;
-  const int bn = pick_block_n(r, 64);
-  if (r % 64 != 0 || bn % 64 != 0) return cudaSuccess;  // MN-major B needs whole 64-wide atoms
+  const int bn = pick_block_n(r, 64);  // MN-major B: whole 64-wide atoms (zero-filled past r)
   CUtensorMap ma, mb;
   if (!map3d(&ma, Bg, true, n, m, count, 64, BK)) return cudaSuccess;
   if (!map3d(&mb, Pg, true, r, m, count, 64, BK)) return cudaSuccess;
@@ -346,11 +402,67 @@ cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, int count, int
   p.tiles_m = (int)((n + BM - 1) / BM);
   p.tiles_n = (int)((r + bn - 1) / bn);
   p.num_kb = (int)((m + BK - 1) / BK);
+  set_pairs(p, 1);
   p.idesc = idesc_bf16(BM, bn, true, true);
   p.C = R; p.ldc = r; p.c_bs = n * r;
   p.flags = flags;
   p.max_spins = max_spins;
   cudaError_t e = launch_gemm<true, true>(ma, mb, p, s);
+  if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
+  return e;
+}
+
+cudaError_t tc_gram(const bf16* Xs, float* W, int count, int64_t m, int64_t r, int32_t* flags,
+                    int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s, int* nlaunch,
+                    bool* done) {
+  using namespace tc;
+  *nlaunch = 0;
+  *done = false;
+  const int bn = pick_block_n(r, 64);
+  CUtensorMap ma, mb;
+  if (!map3d(&ma, Xs, true, r, m, 3 * (uint64_t)count, 64, BK)) return cudaSuccess;
+  if (!map3d(&mb, Xs, true, r, m, 3 * (uint64_t)count, 64, BK)) return cudaSuccess;
+  GemmP p{};
+  p.M = r; p.N = r; p.K = m;
+  p.batch = count;
+  p.block_n = bn;
+  p.tiles_m = (int)((r + BM - 1) / BM);
+  p.tiles_n = (int)((r + bn - 1) / bn);
+  p.num_kb = (int)((m + BK - 1) / BK);
+  set_pairs(p, 6);
+  p.idesc = idesc_bf16(BM, bn, true, true);
+  p.C = W; p.ldc = r; p.c_bs = r * r;
+  p.flags = flags; p.need_mask = need; p.skip_mask = skip;
+  p.max_spins = max_spins;
+  cudaError_t e = launch_gemm<true, true>(ma, mb, p, s);
+  if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
+  return e;
+}
+
+cudaError_t tc_apply(const bf16* Xs, const bf16* Ls, float* Y, bf16* Ys, int count, int64_t m,
+                     int64_t r, int32_t* flags, int32_t need, int32_t skip, int64_t max_spins,
+                     cudaStream_t s, int* nlaunch, bool* done) {
+  using namespace tc;
+  *nlaunch = 0;
+  *done = false;
+  const int bn = pick_block_n(r, 16);
+  CUtensorMap ma, mb;
+  if (!map3d(&ma, Xs, true, r, m, 3 * (uint64_t)count, BK, BM)) return cudaSuccess;
+  if (!map3d(&mb, Ls, true, r, r, 3 * (uint64_t)count, BK, bn)) return cudaSuccess;
+  GemmP p{};
+  p.M = m; p.N = r; p.K = r;
+  p.batch = count;
+  p.block_n = bn;
+  p.tiles_m = (int)((m + BM - 1) / BM);
+  p.tiles_n = (int)((r + bn - 1) / bn);
+  p.num_kb = (int)((r + BK - 1) / BK);
+  set_pairs(p, 6);
+  p.idesc = idesc_bf16(BM, bn, false, false);
+  p.C = Y; p.ldc = r; p.c_bs = m * r;
+  p.Cs = Ys; p.cs_stride = (int64_t)count * m * r;
+  p.flags = flags; p.need_mask = need; p.skip_mask = skip;
+  p.max_spins = max_spins;
+  cudaError_t e = launch_gemm<false, false>(ma, mb, p, s);
   if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
   return e;
 }

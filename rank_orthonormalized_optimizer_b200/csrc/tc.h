@@ -3,15 +3,17 @@
 // the SIMT kernel for the same contraction.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace dion {
 
-// P0[b] (m x r, fp32) = Bg[b] (m x n, bf16) * Qg[b]^T (Qg: r x n, bf16).
-cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, int count, int64_t m,
-                       int64_t n, int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s,
-                       int* nlaunch, bool* done);
+// P0[b] (m x r, fp32) = Bg[b] (m x n, bf16) * Qg[b]^T (Qg: r x n, bf16); when P0s is
+// not null its three-way bf16 split ([3][count][m][r]) is written as well.
+cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, __nv_bfloat16* P0s, int count,
+                       int64_t m, int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
+                       cudaStream_t s, int* nlaunch, bool* done);
 // R[b] (n x r, fp32) = Bg[b]^T (n x m) * Pg[b] (m x r, bf16).
 cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, int count, int64_t m,
                         int64_t n, int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s,
@@ -21,5 +23,17 @@ cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, const floa
                       float* X, int count, int64_t m, int64_t n, int64_t r, float mu,
                       float lr_scale, int64_t max_spins, int32_t* flags, cudaStream_t s,
                       int* nlaunch, bool* done);
+
+// W[b] (r x r, fp32) = X[b]^T X[b] from the three-way split Xs ([3][count][m][r] bf16),
+// six split products; matrices failing (flags & need) == need && !(flags & skip) skipped.
+cudaError_t tc_gram(const __nv_bfloat16* Xs, float* W, int count, int64_t m, int64_t r,
+                    int32_t* flags, int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s,
+                    int* nlaunch, bool* done);
+// Y[b] (m x r, fp32) = X[b] L[b]^T from the splits Xs ([3][count][m][r]) and Ls
+// ([3][count][r][r], L lower triangular), optionally writing Y's split to Ys.
+cudaError_t tc_apply(const __nv_bfloat16* Xs, const __nv_bfloat16* Ls, float* Y,
+                     __nv_bfloat16* Ys, int count, int64_t m, int64_t r, int32_t* flags,
+                     int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s, int* nlaunch,
+                     bool* done);
 
 }  // namespace dion

@@ -98,7 +98,8 @@ def test_workspace_covers_the_layout():
     c, h, ws = _init(c4)
     assert c == dion.OK
     bf16_b = sum(k * m * n * 2 for k, m, n, r in c4)
-    factors = sum(k * (m * r * (4 * 3 + 2) + n * r * (4 + 2 + 2 + 2) + r * r * 8) for k, m, n, r in c4)
+    factors = sum(k * (m * r * (4 * 3 + 2 + 12) + n * r * (4 + 2 + 2 + 2) + r * r * 14)
+                  for k, m, n, r in c4)
     assert bf16_b + factors <= ws < 1.1 * (bf16_b + factors) + (1 << 24)
     assert dion.dion_num_matrices(h) == 224
     dion.dion_free(h)
