@@ -155,23 +155,27 @@ def measured_peaks():
             "source": "fallback"}
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_tc_update_traffic_stack16x4096_r256.json")
+
+
 def update_traffic():
-    """DRAM bytes per element of the fused update from the committed ncu summary, if any."""
-    p = os.path.join(ROOT, "profiles", "update_traffic.json")
-    if os.path.exists(p):
-        d = json.load(open(p))
+    """DRAM bytes per weight element of the fused update, from the committed ncu capture,
+    and the hash of the kernel source it was taken on."""
+    if os.path.exists(TRAFFIC_FILE):
+        d = json.load(open(TRAFFIC_FILE))
         return d.get("dram_bytes_per_element"), d.get("kernel_source_hash")
     return None, None
 
 
-def kernel_source_hash():
+def update_kernel_hash():
+    """Hash of the fused-update kernel's source (its section of k_tc.cu and the PTX
+    helpers): a captured traffic figure is only reported while this is unchanged."""
     import hashlib
-    h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rank_orthonormalized_optimizer_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, name), "rb").read())
-    return h.hexdigest()[:16]
+    src = open(os.path.join(csrc, "k_tc.cu")).read()
+    marker = "// ------------------------------------------------------------------ fused update"
+    upd = src[src.index(marker):] if marker in src else src
+    return hashlib.sha256((upd + open(os.path.join(csrc, "tc_ptx.cuh")).read()).encode()).hexdigest()[:16]
 
 
 # ------------------------------------------------------------------ oracle timing
@@ -264,7 +268,7 @@ def run_ours(args):
     achieved = upd_bytes / (upd_ms / 1e3) / 1e9
     traffic_per_elem, traffic_hash = update_traffic()
     traffic = None
-    if traffic_per_elem is not None and traffic_hash == kernel_source_hash():
+    if traffic_per_elem is not None and traffic_hash == update_kernel_hash():
         traffic = traffic_per_elem * sum(b.params for b in wl.buckets) / max(upd_launches, 1)
     roof_t = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_alg / (peaks["hbm_gbs"] * 1e9))
 

@@ -4,7 +4,7 @@ The arithmetic runs in the CUDA library ``lib/libdion_b200.so`` behind the C ABI
 of ``include/dion.h``; this module only marshals arguments (torch tensors to
 device pointers and the current CUDA stream).  PyTorch provides device memory
 and streams.  There is no CPU implementation: importing this module fails if
-the library has not been built (``python -m rank_orthonormalized_optimizer_b200.build``).
+the library has not been built (``python rank_orthonormalized_optimizer_b200/build.py``).
 
 One step, for every matrix of every bucket (see include/dion.h):
     B = M + G;  P = orth(B Q);  R = B^T P;  M <- B - (1 - mu) P R^T;
@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_PKG, "lib", "libdion_b200.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing: build the CUDA library first with "
-        "`python -m rank_orthonormalized_optimizer_b200.build` (nvcc, sm_100a)")
+        "`python rank_orthonormalized_optimizer_b200/build.py` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 

@@ -1,6 +1,8 @@
 """Build the CUDA library of the batched Dion step for sm_100a (B200), in-tree.
 
-    python -m rank_orthonormalized_optimizer_b200.build [--force] [-v]
+    python rank_orthonormalized_optimizer_b200/build.py [--force] [-v]
+
+(run as a script: importing the package would load the library being rebuilt)
 
 Compiles every ``csrc/*.cu`` with nvcc (``-gencode arch=compute_100a,code=sm_100a``)
 and links ``lib/libdion_b200.so`` with the CUDA runtime linked statically, so the

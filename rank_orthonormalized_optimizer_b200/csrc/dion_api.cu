@@ -188,6 +188,7 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
                                        &nl, &done);
       c.launches += nl;
       if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_gemm_bq: %s", cudaGetErrorString(e));
+      if (!done) return fail(DION_ERR_CUDA, "tc_gemm_bq: %s", dion::tc_map_error());
       p0s_ready = done;
     }
     if (!done) {
@@ -229,38 +230,39 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
     const int chol_launches = r <= 256 ? 1 : (int)(2 + 3 * ((r + 31) / 32) + (r + 31) / 32);
     const int64_t mr = (int64_t)cnt * m * r, rr = (int64_t)cnt * r * r;
     // tensor cores: Gram and triangular apply from three-way bf16 splits (fp32-accurate)
-    auto tc_call = [&](cudaError_t e, int nl, bool done, const char* what) -> dion_status {
+    int nl = 0;
+    bool done = false;
+    // checks the call that just returned e (nl and done were set by that call)
+    auto tc_check = [&](cudaError_t e, const char* what) -> dion_status {
       c.launches += nl;
       if (e != cudaSuccess) return fail(DION_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
-      if (!done) return fail(DION_ERR_CUDA, "%s: tensor map encoding failed", what);
+      if (!done) return fail(DION_ERR_CUDA, "%s: %s", what, dion::tc_map_error());
       return DION_OK;
     };
     if (o.orth_mode != DION_ORTH_HOUSEHOLDER && tensor) {
-      int nl = 0;
-      bool done = false;
       dion_status st;
+      cudaError_t e;
       if (!p0s_ready) DION_LAUNCH(c, 1, dion::launch_split3(P0, P0s, mr, mr, s));
-      st = tc_call(dion::tc_gram(P0s, W, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins,
-                                 s, &nl, &done), nl, done, "tc_gram");
-      if (st != DION_OK) return st;
+      e = dion::tc_gram(P0s, W, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s, &nl,
+                        &done);
+      if ((st = tc_check(e, "tc_gram")) != DION_OK) return st;
       ca.pass = 1; ca.orth_tol = o.orth_tol;
       DION_LAUNCH(c, chol_launches, dion::launch_chol_inv(ca, s));
       DION_LAUNCH(c, 1, dion::launch_split3(Linv, Linvs, rr, rr, s));
-      st = tc_call(dion::tc_apply(P0s, Linvs, P, Ps, cnt, m, r, flags, 0, DION_MAT_FALLBACK,
-                                  o.max_wait_spins, s, &nl, &done), nl, done, "tc_apply");
-      if (st != DION_OK) return st;
+      e = dion::tc_apply(P0s, Linvs, P, Ps, cnt, m, r, flags, 0, DION_MAT_FALLBACK,
+                         o.max_wait_spins, s, &nl, &done);
+      if ((st = tc_check(e, "tc_apply")) != DION_OK) return st;
       if (o.orth_mode != DION_ORTH_CHOLQR) {
-        st = tc_call(dion::tc_gram(Ps, W, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins,
-                                   s, &nl, &done), nl, done, "tc_gram");
-        if (st != DION_OK) return st;
+        e = dion::tc_gram(Ps, W, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s, &nl,
+                          &done);
+        if ((st = tc_check(e, "tc_gram")) != DION_OK) return st;
         ca.pass = 2;
         ca.orth_tol = o.orth_mode == DION_ORTH_CHOLQR2 ? -1.f : o.orth_tol;
         DION_LAUNCH(c, chol_launches, dion::launch_chol_inv(ca, s));
         DION_LAUNCH(c, 1, dion::launch_split3(Linv, Linvs, rr, rr, s));
-        st = tc_call(dion::tc_apply(Ps, Linvs, P2, nullptr, cnt, m, r, flags, DION_MAT_CHOLQR2,
-                                    DION_MAT_FALLBACK, o.max_wait_spins, s, &nl, &done),
-                     nl, done, "tc_apply");
-        if (st != DION_OK) return st;
+        e = dion::tc_apply(Ps, Linvs, P2, nullptr, cnt, m, r, flags, DION_MAT_CHOLQR2,
+                           DION_MAT_FALLBACK, o.max_wait_spins, s, &nl, &done);
+        if ((st = tc_check(e, "tc_apply")) != DION_OK) return st;
       }
     } else if (o.orth_mode != DION_ORTH_HOUSEHOLDER) {
       DION_LAUNCH(c, gl, dion::launch_gemm_simt(gram(P0), false, s));
@@ -289,6 +291,7 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
       cudaError_t e = dion::tc_gemm_btp(Bg, Pg, R, cnt, m, n, r, o.max_wait_spins, flags, s, &nl, &done);
       c.launches += nl;
       if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_gemm_btp: %s", cudaGetErrorString(e));
+      if (!done) return fail(DION_ERR_CUDA, "tc_gemm_btp: %s", dion::tc_map_error());
     }
     if (!done) {
       dion::GemmDesc d{};
@@ -317,6 +320,7 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
                                       o.max_wait_spins, flags, s, &nl, &done);
       c.launches += nl;
       if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_update: %s", cudaGetErrorString(e));
+      if (!done) return fail(DION_ERR_CUDA, "tc_update: %s", dion::tc_map_error());
     }
     if (!done)
       DION_LAUNCH(c, (cnt + 65534) / 65535,

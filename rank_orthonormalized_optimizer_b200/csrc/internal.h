@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/dion.h"
+
 namespace dion {
 
 // Generic strided batched operand: element (i, k) of matrix b sits at

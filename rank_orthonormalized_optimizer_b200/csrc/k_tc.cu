@@ -21,6 +21,8 @@
 //   through shared memory by TMA in 128 x 32 slabs and M, X stored by TMA.
 #include <cuda.h>
 
+#include <cstdio>
+
 #include "common.cuh"
 #include "tc.h"
 #include "tc_ptx.cuh"
@@ -55,21 +57,40 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
+static thread_local char tl_map_error[256];
+
 // 3-D map over a stack [d2][d1][d0] of row-major matrices, box {b0, b1, 1}.
 static bool map3d(CUtensorMap* m, const void* base, bool bf16, uint64_t d0, uint64_t d1,
                   uint64_t d2, uint32_t b0, uint32_t b1) {
   EncodeTiledFn f = encode_fn();
-  if (!f) return false;
+  if (!f) {
+    snprintf(tl_map_error, sizeof(tl_map_error), "cuTensorMapEncodeTiled unavailable");
+    return false;
+  }
   const uint64_t es = bf16 ? 2 : 4;
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {d0 * es, d0 * d1 * es};
   cuuint32_t box[3] = {b0, b1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return f(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
-           const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = f(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                       3, const_cast<void*>(base), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(tl_map_error, sizeof(tl_map_error),
+             "cuTensorMapEncodeTiled -> %d (base %p, dims %llu x %llu x %llu, box %u x %u, %s)",
+             (int)r, base, (unsigned long long)d0, (unsigned long long)d1, (unsigned long long)d2,
+             b0, b1, bf16 ? "bf16" : "fp32");
+    return false;
+  }
+  return true;
 }
+
+}  // namespace tc
+
+const char* tc_map_error() { return tc::tl_map_error; }
+
+namespace tc {
 
 static int sm_count() {
   static int sms = 0;
@@ -709,7 +730,6 @@ cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, const floa
   using namespace tc;
   *nlaunch = 0;
   *done = false;
-  if (r % 16 != 0) return cudaSuccess;
   CUtensorMap mP, mR, mQ, mM, mG, mX, mMs, mXs;
   bool ok = map3d(&mP, Pg, true, r, m, count, BK, BM) && map3d(&mR, Rg, true, r, n, count, BK, UPD_BN) &&
             map3d(&mQ, Qg, true, r, n, count, BK, UPD_BN) &&

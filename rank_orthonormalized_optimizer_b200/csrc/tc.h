@@ -1,6 +1,7 @@
 // Tensor-core (tcgen05 + TMEM, fed by TMA) kernels of the batched Dion step.
-// Each entry sets *done when it handled the call; otherwise the caller runs
-// the SIMT kernel for the same contraction.
+// Each entry sets *done when it launched its kernel; *done stays false only when a
+// tensor map could not be encoded (tc_map_error() says why), which the caller
+// reports as an error.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -8,6 +9,9 @@
 #include <stdint.h>
 
 namespace dion {
+
+// Text of the last tensor-map encoding failure on this thread.
+const char* tc_map_error();
 
 // P0[b] (m x r, fp32) = Bg[b] (m x n, bf16) * Qg[b]^T (Qg: r x n, bf16); when P0s is
 // not null its three-way bf16 split ([3][count][m][r]) is written as well.

@@ -16,7 +16,7 @@ def _ensure_library():
     spec = importlib.util.spec_from_file_location("_dion_build", path)
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
-    if not os.path.exists(mod.LIB):
+    if mod.stale():
         mod.build()
 
 
