@@ -171,6 +171,36 @@ dion_status dion_step_batched_from_host(dion_handle h, const dion_bucket_ptrs* p
                                         int32_t* d_status, int32_t* host_status,
                                         void* stream);
 
+/*
+ * Size of the scratch array built into the library for dion_step_batched_noalloc:
+ * 16 MiB of device memory on every GPU the library is used on, held until the
+ * process exits.
+ */
+#define DION_STATIC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * dion_step_batched without a caller workspace, for callers that cannot allocate
+ * device memory: code running while a stream is being captured into a CUDA graph
+ * (where cudaMalloc is not allowed), plug-ins that are handed only the model's
+ * buffers by a host program whose allocator they cannot reach, or loops that must
+ * not allocate after start-up.  The pages describe nothing like it; it is a
+ * convenience of this library.  Arguments are those of dion_step_batched; X, M, G,
+ * Q and d_status remain caller buffers.
+ *  - Scratch comes from one array of DION_STATIC_SCRATCH_BYTES inside the library.
+ *    A plan whose workspace (from dion_init) is larger is rejected with
+ *    DION_ERR_WORKSPACE_TOO_SMALL and nothing runs.
+ *  - The first call on a device looks the array's device address up once (with
+ *    that device current); make that first call outside any stream capture.
+ *  - Every call on a device shares the array.  It keeps whatever the last call
+ *    left in it; the step writes every scratch word it reads, so nothing needs
+ *    clearing.  Calls whose work overlaps on the GPU (two streams, two threads, two
+ *    handles) race on it: serialise them.
+ *  - The library allocates and frees no device memory in this call.
+ */
+dion_status dion_step_batched_noalloc(dion_handle h, const dion_bucket_ptrs* ptrs,
+                                      int32_t nbuckets, float lr, int32_t* d_status,
+                                      void* stream);
+
 /* Release the handle (host memory only).  NULL is accepted. */
 dion_status dion_free(dion_handle h);
 

@@ -38,6 +38,7 @@ ORTH_MODES = {"auto": 0, "cholqr": 1, "cholqr2": 2, "householder": 3}
 KERNEL_PATHS = {"tensor": 0, "simt": 1}
 KERNEL_CLASSES = ["form_b", "prep_q", "gemm_bq", "orth", "gemm_btp", "colnorm", "update"]
 VIEW_P, VIEW_R = 0, 1
+STATIC_SCRATCH_BYTES = 16 << 20   # DION_STATIC_SCRATCH_BYTES of include/dion.h
 
 
 class BucketDesc(ctypes.Structure):
@@ -70,6 +71,8 @@ dion_step_batched = _sig("dion_step_batched", c_int32, c_void_p, ctypes.POINTER(
 dion_step_batched_from_host = _sig("dion_step_batched_from_host", c_int32, c_void_p,
                                    ctypes.POINTER(BucketPtrs), ctypes.POINTER(c_void_p), c_int32,
                                    c_float, c_void_p, c_size_t, c_void_p, c_void_p, c_void_p)
+dion_step_batched_noalloc = _sig("dion_step_batched_noalloc", c_int32, c_void_p,
+                                 ctypes.POINTER(BucketPtrs), c_int32, c_float, c_void_p, c_void_p)
 dion_free = _sig("dion_free", c_int32, c_void_p)
 dion_status_string = _sig("dion_status_string", ctypes.c_char_p, c_int32)
 dion_last_error = _sig("dion_last_error", ctypes.c_char_p)
@@ -83,7 +86,7 @@ dion_profile_read = _sig("dion_profile_read", c_int32, c_void_p, ctypes.POINTER(
 
 #: every entry point include/dion.h declares
 EXPORTED = ["dion_default_options", "dion_init", "dion_step_batched",
-            "dion_step_batched_from_host", "dion_free", "dion_status_string", "dion_last_error",
+            "dion_step_batched_from_host", "dion_step_batched_noalloc", "dion_free", "dion_status_string", "dion_last_error",
             "dion_num_matrices", "dion_last_launch_count", "dion_workspace_view",
             "dion_profile_enable", "dion_profile_read"]
 
@@ -191,6 +194,14 @@ class DionB200:
                                  c_void_p(status.data_ptr()) if status is not None else None,
                                  self._stream(stream)),
                "dion_step_batched")
+
+    def step_noalloc(self, X, M, G, Q, lr: float, status=None, stream=None):
+        """The step with the library's built-in scratch instead of a workspace."""
+        arr = self._ptrs(X, M, G, Q)
+        _check(dion_step_batched_noalloc(self._h, arr, len(self.shapes), float(lr),
+                                         c_void_p(status.data_ptr()) if status is not None else None,
+                                         self._stream(stream)),
+               "dion_step_batched_noalloc")
 
     def step_from_host(self, X, M, G_dev, Q, G_host, lr: float, workspace, status, host_status,
                        stream=None):

@@ -374,6 +374,26 @@ dion_status check_step_args(dion_handle h, const dion_bucket_ptrs* ptrs, int32_t
 
 }  // namespace
 
+namespace dion {
+
+dion_status set_error(dion_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  tl_error = buf;
+  return s;
+}
+
+dion_status plan_workspace_bytes(dion_handle h, size_t* bytes) {
+  if (!valid(h)) return fail(DION_ERR_NOT_INITIALIZED, "invalid or freed handle");
+  *bytes = h->ws_bytes;
+  return DION_OK;
+}
+
+}  // namespace dion
+
 extern "C" {
 
 dion_status dion_default_options(dion_options* opt) {

@@ -9,6 +9,11 @@
 
 namespace dion {
 
+// Record a message for dion_last_error() on this thread and return `s`.
+dion_status set_error(dion_status s, const char* fmt, ...);
+// Workspace size of a valid handle's plan.
+dion_status plan_workspace_bytes(dion_handle h, size_t* bytes);
+
 // Generic strided batched operand: element (i, k) of matrix b sits at
 // base + b*sb + i*si + k*sk (in elements).
 struct Operand {
