@@ -128,8 +128,8 @@ dion_status dion_default_options(dion_options* opt);
 
 /*
  * Plan a step over `nbuckets` buckets (host only; touches no device).
- * Supported shapes: count >= 1, 1 <= r <= min(m, n), r % 16 == 0, n % 8 == 0,
- * m >= 1, and every buffer below 2^40 elements; otherwise
+ * Supported shapes: 1 <= count <= 65535, 1 <= r <= min(m, n), r % 16 == 0,
+ * n % 8 == 0, m >= 1, and every buffer below 2^40 elements; otherwise
  * DION_ERR_UNSUPPORTED_SHAPE.  opt may be NULL (defaults).
  * On success *out receives a handle (host memory owned by the library until
  * dion_free) and *workspace_bytes the size of the device workspace that

@@ -184,8 +184,9 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
     bool done = false;
     if (tensor && bf) {
       int nl = 0;
-      cudaError_t e = dion::tc_gemm_bq(Bg, Qg, P0, P0s, cnt, m, n, r, o.max_wait_spins, flags, s,
-                                       &nl, &done);
+      // only the split of P0 is written: the orthonormalisation reads nothing else
+      cudaError_t e = dion::tc_gemm_bq(Bg, Qg, nullptr, P0s, cnt, m, n, r, o.max_wait_spins, flags,
+                                       s, &nl, &done);
       c.launches += nl;
       if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_gemm_bq: %s", cudaGetErrorString(e));
       if (!done) return fail(DION_ERR_CUDA, "tc_gemm_bq: %s", dion::tc_map_error());
@@ -277,7 +278,8 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
         DION_LAUNCH(c, gl, dion::launch_gemm_simt(apply(P, P2, DION_MAT_CHOLQR2), false, s));
       }
     }
-    DION_LAUNCH(c, 1, dion::launch_householder(P0, P2, P0, P, flags, cnt, m, r, s));
+    DION_LAUNCH(c, 1, dion::launch_householder(P0, p0s_ready ? P0s : nullptr, P2, P0, P, flags,
+                                               cnt, m, r, s));
     DION_LAUNCH(c, 1, dion::launch_finalize_p(P, P2, Pg, bf, flags, cnt, m, r, P, s));
   }
   end_cls(c);
@@ -431,6 +433,9 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
   for (int32_t b = 0; b < nbuckets; ++b) {
     const dion_bucket_desc& d = buckets[b];
     if (d.count < 1) return fail(DION_ERR_INVALID_ARG, "bucket %d: count %d < 1", b, d.count);
+    if (d.count > 65535)
+      return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: count %d exceeds 65535 (split the bucket)",
+                  b, d.count);
     if (d.m < 1 || d.n < 1 || d.r < 1)
       return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: m, n, r must be positive", b);
     if (d.r > d.m || d.r > d.n)
@@ -450,13 +455,7 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
     p.scale = d.scale > 0.f ? d.scale : (float)std::sqrt((double)d.m / (double)d.n);
     p.mat0 = mats;
     mats += d.count;
-    {
-      int64_t ns = (2 * 148 + d.count - 1) / d.count;
-      if (ns > 64) ns = 64;
-      if (ns > (d.n + 31) / 32) ns = (d.n + 31) / 32;
-      if (ns < 1) ns = 1;
-      p.nsplit = (int)ns;
-    }
+    p.nsplit = dion::colnorm_splits(d.count, d.n);
     const size_t c = (size_t)d.count;
     p.off_Bg = take(c * d.m * d.n * ge);
     p.off_Qg = take(c * d.n * d.r * ge);

@@ -44,6 +44,7 @@ cudaError_t launch_init_flags(int32_t* flags, float* stats, int count, int32_t i
 cudaError_t launch_finalize_p(const float* P, const float* P2, void* Pg, bool use_bf16,
                               const int32_t* flags, int count, int64_t m, int64_t r,
                               float* P_out, cudaStream_t s);
+int colnorm_splits(int count, int64_t n);
 cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, bool use_bf16,
                            float* part, int nsplit, int32_t* flags, int count, int64_t n,
                            int64_t r, cudaStream_t s);
@@ -73,8 +74,9 @@ struct CholArgs {
   float orth_tol;      // pass 2: skip the second pass when max|W - I| <= orth_tol
 };
 cudaError_t launch_chol_inv(const CholArgs& a, cudaStream_t s);
-cudaError_t launch_householder(const float* P0, float* work_cm, float* q_cm, float* P,
-                               int32_t* flags, int count, int64_t m, int64_t r,
+// P0 fp32, or (when P0s is not null) its three-way bf16 split [3][count][m][r].
+cudaError_t launch_householder(const float* P0, const void* P0s, float* work_cm, float* q_cm,
+                               float* P, int32_t* flags, int count, int64_t m, int64_t r,
                                cudaStream_t s);
 size_t chol_dinv_floats(int count, int64_t r);
 

@@ -73,33 +73,58 @@ cudaError_t launch_form_b(const float* M, const float* G, void* Bg, bool use_bf1
 
 // ------------------------------------------------- previous Q into GEMM layout
 // Qg[b][j][i] = Q[b][i][j]: the n x r factor transposed to r x n so that the
-// contraction B Q reads both operands along n (the reduction axis).
+// contraction B Q reads both operands along n (the reduction axis).  64 x 64 tiles:
+// float4 loads along r, 4-element stores along n.
 template <typename T>
-__global__ void k_prep_q(const float* __restrict__ Q, T* __restrict__ Qg, int64_t n, int64_t r) {
-  __shared__ float tile[32][33];
+__global__ void __launch_bounds__(256) k_prep_q(const float* __restrict__ Q, T* __restrict__ Qg,
+                                                 int64_t n, int64_t r) {
+  __shared__ float tile[64][65];
   const int64_t b = blockIdx.z;
   const float* q = Q + b * n * r;
   T* qg = Qg + b * n * r;
-  const int64_t j0 = (int64_t)blockIdx.x * 32, i0 = (int64_t)blockIdx.y * 32;
-  for (int y = threadIdx.y; y < 32; y += 8) {
-    const int64_t i = i0 + y, j = j0 + threadIdx.x;
-    tile[y][threadIdx.x] = (i < n && j < r) ? q[i * r + j] : 0.f;
+  const int64_t j0 = (int64_t)blockIdx.x * 64, i0 = (int64_t)blockIdx.y * 64;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < 64 * 16; e += 256) {       // 64 rows (i) x 16 float4 (j)
+    const int y = e / 16, x4 = e % 16;
+    const int64_t i = i0 + y, j = j0 + 4 * x4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < n && j < r) v = *reinterpret_cast<const float4*>(q + i * r + j);  // r % 16 == 0
+    tile[4 * x4 + 0][y] = v.x;
+    tile[4 * x4 + 1][y] = v.y;
+    tile[4 * x4 + 2][y] = v.z;
+    tile[4 * x4 + 3][y] = v.w;
   }
   __syncthreads();
-  for (int y = threadIdx.y; y < 32; y += 8) {
-    const int64_t j = j0 + y, i = i0 + threadIdx.x;
-    if (i < n && j < r) qg[j * n + i] = Cvt<T>::from_f(tile[threadIdx.x][y]);
+  for (int e = tid; e < 64 * 16; e += 256) {       // 64 rows (j) x 16 groups of 4 (i)
+    const int y = e / 16, x4 = e % 16;
+    const int64_t j = j0 + y, i = i0 + 4 * x4;
+    if (j >= r || i >= n) continue;
+    T* dst = qg + j * n + i;
+    if (i + 3 < n) {
+      if (sizeof(T) == 2) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(tile[y][4 * x4], tile[y][4 * x4 + 1]);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(tile[y][4 * x4 + 2], tile[y][4 * x4 + 3]);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(dst) = pk;  // n % 8 == 0: 8-byte aligned
+      } else {
+        *reinterpret_cast<float4*>(dst) =
+            make_float4(tile[y][4 * x4], tile[y][4 * x4 + 1], tile[y][4 * x4 + 2], tile[y][4 * x4 + 3]);
+      }
+    } else {
+      for (int q2 = 0; q2 < 4 && i + q2 < n; ++q2) dst[q2] = Cvt<T>::from_f(tile[y][4 * x4 + q2]);
+    }
   }
 }
 
 cudaError_t launch_prep_q(const float* Q, void* Qg, bool use_bf16, int count, int64_t n, int64_t r,
                           cudaStream_t s) {
-  dim3 grid((unsigned)((r + 31) / 32), (unsigned)((n + 31) / 32), (unsigned)count);
-  dim3 block(32, 8);
+  dim3 grid((unsigned)((r + 63) / 64), (unsigned)((n + 63) / 64), (unsigned)count);
   if (use_bf16)
-    k_prep_q<bf16><<<grid, block, 0, s>>>(Q, (bf16*)Qg, n, r);
+    k_prep_q<bf16><<<grid, 256, 0, s>>>(Q, (bf16*)Qg, n, r);
   else
-    k_prep_q<float><<<grid, block, 0, s>>>(Q, (float*)Qg, n, r);
+    k_prep_q<float><<<grid, 256, 0, s>>>(Q, (float*)Qg, n, r);
   return cudaGetLastError();
 }
 
@@ -200,24 +225,47 @@ cudaError_t launch_finalize_p(const float* P, const float* P2, void* Pg, bool us
 
 // ------------------------------------------------------------- Q = colnorm(R)
 // Step 6: each column of R (n x r) divided by its 2-norm over the n rows.
-// Deterministic two-stage reduction: fixed row splits, then a fixed-order
-// sum of the splits.  A zero column gives a zero Q column and F_ZERO_COL.
+// Deterministic two-stage reduction: every block sums the squares of a fixed
+// row range in a fixed order, then the per-range sums are added in range order.
+// A zero column gives a zero Q column and F_ZERO_COL.
+// Vectorised by 4 columns (r % 16 == 0); 256 threads = (256 / (r/4)) row lanes.
 __global__ void __launch_bounds__(256) k_colnorm_partial(const float* __restrict__ R,
                                                           float* __restrict__ part, int64_t n,
                                                           int64_t r, int nsplit) {
+  extern __shared__ float4 red4[];  // [lanes][r/4]
   const int64_t b = blockIdx.y;
   const int split = blockIdx.x;
+  const int vc = (int)(r / 4);
   const int64_t rows = (n + nsplit - 1) / nsplit;
   const int64_t i0 = split * rows, i1 = (i0 + rows < n) ? i0 + rows : n;
-  const float* rb = R + b * n * r;
-  for (int64_t j = threadIdx.x; j < r; j += blockDim.x) {
-    float acc = 0.f;
-#pragma unroll 8
-    for (int64_t i = i0; i < i1; ++i) {
-      const float v = rb[i * r + j];
-      acc = fmaf(v, v, acc);
+  const float4* rb = reinterpret_cast<const float4*>(R + b * n * r);
+  const int lanes = vc >= 256 ? 1 : 256 / vc;  // row lanes
+  for (int c0 = 0; c0 < vc; c0 += 256) {
+    const int t = threadIdx.x;
+    const int col = c0 + (vc >= 256 ? t : t % vc);
+    const int lane = vc >= 256 ? 0 : t / vc;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (col < vc && lane < lanes) {
+#pragma unroll 4
+      for (int64_t i = i0 + lane; i < i1; i += lanes) {
+        const float4 v = __ldcs(rb + i * vc + col);
+        acc.x = fmaf(v.x, v.x, acc.x);
+        acc.y = fmaf(v.y, v.y, acc.y);
+        acc.z = fmaf(v.z, v.z, acc.z);
+        acc.w = fmaf(v.w, v.w, acc.w);
+      }
     }
-    part[(b * nsplit + split) * r + j] = acc;
+    if (lane < lanes && col < vc) red4[lane * (vc >= 256 ? 256 : vc) + (col - c0)] = acc;
+    __syncthreads();
+    if (lane == 0 && col < vc) {
+      float4 s4 = red4[col - c0];
+      for (int l = 1; l < lanes; ++l) {
+        const float4 o = red4[l * vc + (col - c0)];
+        s4.x += o.x; s4.y += o.y; s4.z += o.z; s4.w += o.w;
+      }
+      reinterpret_cast<float4*>(part + (b * nsplit + split) * r)[col] = s4;
+    }
+    __syncthreads();
   }
 }
 
@@ -242,35 +290,56 @@ __global__ void __launch_bounds__(256) k_colnorm_apply(const float* __restrict__
   }
   zero = __syncthreads_or(zero);
   if (zero && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(flags + b, F_ZERO_COL);
+  const int64_t vc = r / 4;
   const int64_t i0 = blockIdx.x * rows_per_block;
   const int64_t i1 = (i0 + rows_per_block < n) ? i0 + rows_per_block : n;
-  const int64_t base = b * n * r;
-  for (int64_t i = i0; i < i1; ++i) {
-    for (int64_t j = threadIdx.x; j < r; j += blockDim.x) {
-      const int64_t e = base + i * r + j;
-      const float rv = R[e];
-      const float nrm = norm_s[j];
-      const float qv = nrm > 0.f ? rv / nrm : 0.f;
-      Q[e] = qv;
-      if (BF16) {
-        reinterpret_cast<bf16*>(Rg)[e] = __float2bfloat16_rn(rv);
-        reinterpret_cast<bf16*>(Qg)[e] = __float2bfloat16_rn(qv);
-      }
+  const int64_t e0 = (b * n + i0) * vc, e1 = (b * n + i1) * vc;
+  const float4* R4 = reinterpret_cast<const float4*>(R);
+  float4* Q4 = reinterpret_cast<float4*>(Q);
+  for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+    const int j = (int)((e - e0) % vc) * 4;
+    const float4 rv = R4[e];
+    const float n0 = norm_s[j], n1 = norm_s[j + 1], n2 = norm_s[j + 2], n3 = norm_s[j + 3];
+    float4 qv;
+    qv.x = n0 > 0.f ? rv.x / n0 : 0.f;
+    qv.y = n1 > 0.f ? rv.y / n1 : 0.f;
+    qv.z = n2 > 0.f ? rv.z / n2 : 0.f;
+    qv.w = n3 > 0.f ? rv.w / n3 : 0.f;
+    Q4[e] = qv;
+    if (BF16) {
+      __nv_bfloat162 r01 = __floats2bfloat162_rn(rv.x, rv.y), r23 = __floats2bfloat162_rn(rv.z, rv.w);
+      __nv_bfloat162 q01 = __floats2bfloat162_rn(qv.x, qv.y), q23 = __floats2bfloat162_rn(qv.z, qv.w);
+      uint2 rp, qp;
+      rp.x = *reinterpret_cast<uint32_t*>(&r01); rp.y = *reinterpret_cast<uint32_t*>(&r23);
+      qp.x = *reinterpret_cast<uint32_t*>(&q01); qp.y = *reinterpret_cast<uint32_t*>(&q23);
+      reinterpret_cast<uint2*>(Rg)[e] = rp;
+      reinterpret_cast<uint2*>(Qg)[e] = qp;
     }
   }
+}
+
+int colnorm_splits(int count, int64_t n) {
+  // planned on the host before any device is touched: sized for B200's 148 SMs
+  int64_t ns = (8 * 148 + count - 1) / count;
+  if (ns > 256) ns = 256;
+  if (ns > (n + 15) / 16) ns = (n + 15) / 16;
+  if (ns < 1) ns = 1;
+  return (int)ns;
 }
 
 cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, bool use_bf16, float* part,
                            int nsplit, int32_t* flags, int count, int64_t n, int64_t r,
                            cudaStream_t s) {
-  k_colnorm_partial<<<dim3((unsigned)nsplit, (unsigned)count), 256, 0, s>>>(R, part, n, r,
-                                                                            nsplit);
+  const int64_t vc = r / 4;
+  const size_t red_bytes = (size_t)(vc >= 256 ? 256 : 256 / vc * vc) * sizeof(float4);
+  k_colnorm_partial<<<dim3((unsigned)nsplit, (unsigned)count), 256, red_bytes, s>>>(R, part, n, r,
+                                                                                  nsplit);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int64_t target_blocks = 2 * (int64_t)sm_count();
+  const int64_t target_blocks = 8 * (int64_t)sm_count();
   int64_t per_mat = (target_blocks + count - 1) / count;
   int64_t rows = (n + per_mat - 1) / per_mat;
-  if (rows < 8) rows = 8;
+  if (rows < 4) rows = 4;
   const int64_t gx = (n + rows - 1) / rows;
   const size_t smem = (size_t)r * sizeof(float);
   if (smem > 48 * 1024) {

@@ -115,6 +115,218 @@ __global__ void __launch_bounds__(NT) k_chol_small(CholArgs a) {
   if (a.pass == 2 && tid == 0) atomicOr(a.flags + b, F_CHOLQR2);
 }
 
+// ------------------------------------ r <= 256: one CTA, 32 x 32 blocks in shared memory
+// Right-looking blocked Cholesky with the triangular inverse, all on chip:
+//   for each block column k: factor L_kk (one warp), D_k = L_kk^-1 (one warp),
+//   panel L_ik = W_ik D_k^T (a thread per row), trailing W_ij -= L_ik L_jk^T
+//   (a warp per block pair, a lane per row, the row of L_ik in registers);
+//   then L^-1 block row by block row: X_ij = -D_i sum_{k=j}^{i-1} L_ik X_kj, X_ii = D_i.
+// Rows and columns past r are padded with the identity, which factors and inverts
+// to itself.  Padded stride 33 keeps row-per-lane accesses free of bank conflicts.
+namespace {
+constexpr int CB = 32, CBS = 33, CBLK = CB * CBS;
+__device__ __forceinline__ float* blk_at(float* base, int i, int j) {
+  return base + (i * (i + 1) / 2 + j) * CBLK;
+}
+}  // namespace
+
+size_t chol_blocked_smem_bytes(int64_t r) {
+  const int T = (int)((r + CB - 1) / CB);
+  return (size_t)(T * (T + 1) / 2 + T + (T > 1 ? T - 1 : 1)) * CBLK * sizeof(float) + 64 * sizeof(float);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
+  extern __shared__ float sm[];
+  const int r = (int)a.r;
+  const int T = (r + CB - 1) / CB;
+  float* blk = sm;                                  // T(T+1)/2 lower blocks
+  float* dinv = blk + (T * (T + 1) / 2) * CBLK;     // T inverses of the diagonal blocks
+  float* tmp = dinv + T * CBLK;                     // T-1 blocks of partial sums
+  float* red = tmp + (T > 1 ? T - 1 : 1) * CBLK;    // 64 floats
+  __shared__ int s_fail;
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = NT / 32;
+  const int32_t f0 = a.flags[b];
+  if (f0 & F_FALLBACK) return;
+  const float* W = a.W + (int64_t)b * r * r;
+
+  // load the lower blocks, padding with the identity; check finiteness and |W - I|
+  float dev = 0.f;
+  bool nonfin = false;
+  const int nlow = T * (T + 1) / 2;
+  for (int e = tid; e < nlow * CB * CB; e += NT) {
+    const int bl = e / (CB * CB), w = e % (CB * CB), u = w / CB, v = w % CB;
+    int bi = 0;
+    while ((bi + 1) * (bi + 2) / 2 <= bl) ++bi;
+    const int bj = bl - bi * (bi + 1) / 2;
+    const int gi = bi * CB + u, gj = bj * CB + v;
+    float val;
+    if (gi < r && gj < r) {
+      val = W[(int64_t)gi * r + gj];
+      if (gj <= gi) {
+        nonfin |= !isfinite(val);
+        dev = fmaxf(dev, fabsf(val - (gi == gj ? 1.f : 0.f)));
+      }
+    } else {
+      val = (gi == gj) ? 1.f : 0.f;
+    }
+    blk[bl * CBLK + u * CBS + v] = val;
+  }
+  if (tid == 0) s_fail = 0;
+  nonfin = __syncthreads_or(nonfin);
+  if (nonfin) {
+    if (tid == 0) atomicOr(a.flags + b, F_NONFINITE | F_FALLBACK);
+    return;
+  }
+  if (a.pass == 2) {
+    dev = block_max<NT>(dev, red);
+    if (dev <= a.orth_tol) return;  // the first pass is orthonormal enough
+  }
+
+  float dmin = 3.0e38f, dmax = 0.f;  // meaningful in warp 0
+  for (int k = 0; k < T; ++k) {
+    float* Lkk = blk_at(blk, k, k);
+    float* Dk = dinv + k * CBLK;
+    if (warp == 0) {
+      // Cholesky of the diagonal block, lane = row
+      const int u = lane;
+      bool fail = false;
+      for (int j = 0; j < CB; ++j) {
+        const float d = Lkk[j * CBS + j];
+        if (!(d > 0.f) || !isfinite(d)) { fail = true; break; }
+        const float ljj = sqrtf(d);
+        if (k * CB + j < r) { dmin = fminf(dmin, ljj); dmax = fmaxf(dmax, ljj); }
+        __syncwarp();
+        if (u > j) Lkk[u * CBS + j] /= ljj;
+        __syncwarp();
+        if (u == j) Lkk[j * CBS + j] = ljj;
+        if (u > j) {
+          const float luj = Lkk[u * CBS + j];
+          for (int c = j + 1; c <= u; ++c) Lkk[u * CBS + c] -= luj * Lkk[c * CBS + j];
+        }
+        __syncwarp();
+      }
+      if (fail) {
+        if (lane == 0) s_fail = 1;
+      } else {
+        // D_k = L_kk^-1 by forward substitution, lane = column
+        const int v = lane;
+        for (int i = 0; i < CB; ++i) {
+          if (i < v) { Dk[i * CBS + v] = 0.f; continue; }
+          float sacc = (i == v) ? 1.f : 0.f;
+          for (int t = v; t < i; ++t) sacc -= Lkk[i * CBS + t] * Dk[t * CBS + v];
+          Dk[i * CBS + v] = sacc / Lkk[i * CBS + i];
+        }
+      }
+    }
+    __syncthreads();
+    if (s_fail) {
+      if (tid == 0) atomicOr(a.flags + b, F_FALLBACK);
+      return;
+    }
+    // panel: L_ik = W_ik D_k^T, one thread per row of the panel
+    const int prow = (T - 1 - k) * CB;
+    for (int rr = tid; rr < prow; rr += NT) {
+      float* row = blk_at(blk, k + 1 + rr / CB, k) + (rr % CB) * CBS;
+      float w[CB];
+#pragma unroll
+      for (int t = 0; t < CB; ++t) w[t] = row[t];
+#pragma unroll
+      for (int c = 0; c < CB; ++c) {
+        float sacc = 0.f;
+        for (int t = 0; t <= c; ++t) sacc = fmaf(w[t], Dk[c * CBS + t], sacc);
+        row[c] = sacc;
+      }
+    }
+    __syncthreads();
+    // trailing update: W_ij -= L_ik L_jk^T for k < j <= i
+    const int nt = T - 1 - k;
+    const int npairs = nt * (nt + 1) / 2;
+    for (int pi = warp; pi < npairs; pi += NW) {
+      int ii = 0;
+      while ((ii + 1) * (ii + 2) / 2 <= pi) ++ii;
+      const int jj = pi - ii * (ii + 1) / 2;
+      const int i = k + 1 + ii, j = k + 1 + jj;
+      const float* Lik = blk_at(blk, i, k) + lane * CBS;
+      const float* Ljk = blk_at(blk, j, k);
+      float* Wij = blk_at(blk, i, j) + lane * CBS;
+      float av[CB];
+#pragma unroll
+      for (int t = 0; t < CB; ++t) av[t] = Lik[t];
+      for (int c = 0; c < CB; ++c) {
+        float sacc = 0.f;
+#pragma unroll
+        for (int t = 0; t < CB; ++t) sacc = fmaf(av[t], Ljk[c * CBS + t], sacc);
+        Wij[c] -= sacc;
+      }
+    }
+    __syncthreads();
+  }
+
+  if (a.pass == 1 && dmax > a.fallback_cond * dmin) s_fail = 1;  // warp 0 only
+  __syncthreads();
+  if (s_fail) {
+    if (tid == 0) atomicOr(a.flags + b, F_FALLBACK);
+    return;
+  }
+  if (tid == 0) {
+    a.stats[2 * b] = dmin;
+    a.stats[2 * b + 1] = dmax;
+  }
+
+  // L^-1 block row by block row; X_ij overwrites L_ij once row i is done
+  for (int i = 1; i < T; ++i) {
+    for (int j = warp; j < i; j += NW) {
+      float acc[CB];
+#pragma unroll
+      for (int c = 0; c < CB; ++c) acc[c] = 0.f;
+      for (int k = j; k < i; ++k) {
+        const float* Lik = blk_at(blk, i, k) + lane * CBS;
+        const float* Xkj = (k == j) ? dinv + j * CBLK : blk_at(blk, k, j);
+        float av[CB];
+#pragma unroll
+        for (int t = 0; t < CB; ++t) av[t] = Lik[t];
+#pragma unroll
+        for (int t = 0; t < CB; ++t) {
+          const float* xr = Xkj + t * CBS;
+#pragma unroll
+          for (int c = 0; c < CB; ++c) acc[c] = fmaf(av[t], xr[c], acc[c]);
+        }
+      }
+      float* Sj = tmp + j * CBLK + lane * CBS;
+#pragma unroll
+      for (int c = 0; c < CB; ++c) Sj[c] = acc[c];
+    }
+    __syncthreads();
+    for (int j = warp; j < i; j += NW) {
+      const float* Di = dinv + i * CBLK + lane * CBS;
+      const float* Sj = tmp + j * CBLK;
+      float* Xij = blk_at(blk, i, j) + lane * CBS;
+      for (int c = 0; c < CB; ++c) {
+        float sacc = 0.f;
+        for (int t = 0; t <= lane; ++t) sacc = fmaf(Di[t], Sj[t * CBS + c], sacc);
+        Xij[c] = -sacc;
+      }
+    }
+    __syncthreads();
+  }
+
+  // write L^-1 (zeros above the diagonal)
+  float* Li = a.Linv + (int64_t)b * r * r;
+  for (int64_t e = tid; e < (int64_t)r * r; e += NT) {
+    const int gi = (int)(e / r), gj = (int)(e % r);
+    float val = 0.f;
+    if (gj <= gi) {
+      const int bi = gi / CB, bj = gj / CB, u = gi % CB, v = gj % CB;
+      val = (bi == bj) ? dinv[bi * CBLK + u * CBS + v] : blk_at(blk, bi, bj)[u * CBS + v];
+    }
+    Li[e] = val;
+  }
+  if (a.pass == 2 && tid == 0) atomicOr(a.flags + b, F_CHOLQR2);
+}
+
 // ---------------------------------------------- r > 256: blocked, multi-launch
 // Pass 2 entry: compare W with I; set F_CHOLQR2 when the second pass is needed.
 __global__ void __launch_bounds__(256) k_gram_check(CholArgs a) {
@@ -348,12 +560,12 @@ size_t chol_dinv_floats(int count, int64_t r) { return (size_t)count * r * NB; }
 
 cudaError_t launch_chol_inv(const CholArgs& a, cudaStream_t s) {
   if (a.r <= CHOL_SMALL_MAX) {
-    constexpr int NT = 1024;
-    const size_t smem = (size_t)(a.r * (a.r + 1) / 2 + a.r + 32) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(k_chol_small<NT>,
+    constexpr int NT = 512;
+    const size_t smem = chol_blocked_smem_bytes(a.r);
+    cudaError_t e = cudaFuncSetAttribute(k_chol_blocked<NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_chol_small<NT><<<a.count, NT, smem, s>>>(a);
+    k_chol_blocked<NT><<<a.count, NT, smem, s>>>(a);
     return cudaGetLastError();
   }
   k_gram_check<<<a.count, 256, 0, s>>>(a);
@@ -379,7 +591,8 @@ cudaError_t launch_chol_inv(const CholArgs& a, cudaStream_t s) {
 // q_cm are m x r column-major scratch (q_cm may alias P0: P0 is read first).
 // P receives the orthonormal factor with column signs fixed so that the
 // triangular factor has a non-negative diagonal.
-__global__ void __launch_bounds__(1024) k_householder(const float* P0, float* work_cm,
+__global__ void __launch_bounds__(1024) k_householder(const float* P0, const bf16* P0s,
+                                                      int64_t split_stride, float* work_cm,
                                                       float* q_cm, float* P,
                                                       const int32_t* flags, int64_t m,
                                                       int64_t r) {
@@ -401,7 +614,14 @@ __global__ void __launch_bounds__(1024) k_householder(const float* P0, float* wo
   for (int64_t ti = 0; ti < m; ti += 32)
     for (int64_t tj = 0; tj < r; tj += 32) {
       const int y = tid / 32, x = tid % 32;
-      tile[y][x] = (ti + y < m && tj + x < r) ? p0[(ti + y) * r + tj + x] : 0.f;
+      float v = 0.f;
+      if (ti + y < m && tj + x < r) {
+        const int64_t e = (int64_t)b * m * r + (ti + y) * r + tj + x;
+        v = P0s ? (__bfloat162float(P0s[e]) + __bfloat162float(P0s[e + split_stride])) +
+                      __bfloat162float(P0s[e + 2 * split_stride])
+                : p0[(ti + y) * r + tj + x];
+      }
+      tile[y][x] = v;
       __syncthreads();
       if (ti + x < m && tj + y < r) A[(tj + y) * m + ti + x] = tile[x][y];
       __syncthreads();
@@ -476,8 +696,8 @@ __global__ void __launch_bounds__(1024) k_householder(const float* P0, float* wo
     }
 }
 
-cudaError_t launch_householder(const float* P0, float* work_cm, float* q_cm, float* P,
-                               int32_t* flags, int count, int64_t m, int64_t r,
+cudaError_t launch_householder(const float* P0, const void* P0s, float* work_cm, float* q_cm,
+                               float* P, int32_t* flags, int count, int64_t m, int64_t r,
                                cudaStream_t s) {
   const size_t smem = (size_t)(2 * r + 32) * sizeof(float);
   if (smem > 48 * 1024) {
@@ -485,7 +705,8 @@ cudaError_t launch_householder(const float* P0, float* work_cm, float* q_cm, flo
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  k_householder<<<count, 1024, smem, s>>>(P0, work_cm, q_cm, P, flags, m, r);
+  k_householder<<<count, 1024, smem, s>>>(P0, (const bf16*)P0s, (int64_t)count * m * r, work_cm,
+                                          q_cm, P, flags, m, r);
   return cudaGetLastError();
 }
 

@@ -117,45 +117,49 @@ __device__ void mark_unfinished(int32_t* flags, int t, int ntiles, int tiles_per
 }
 
 // ------------------------------------------------------------------ batched GEMM
-// C[b] = sum over pairs (i, j) of A_i[b] B_j[b], fp32 accumulation in TMEM.
-// One pair is a plain bf16 GEMM.  With operands split into three bf16 parts
-// (x = x0 + x1 + x2, each the bf16 rounding of what the earlier parts left),
-// the six pairs (0,0) (0,1) (1,0) (1,1) (0,2) (2,0) reproduce an fp32 product to
-// about 2^-24 relative: this keeps the Gram matrix and the triangular apply of
-// Cholesky-QR fp32-accurate on bf16 tensor cores.  A split operand is stored as
-// [3 * batch][rows][cols]; split i of matrix b is matrix i * batch + b.
-constexpr int MAX_PAIRS = 6;
-
+// C[b] = A[b] B[b] with fp32 accumulation in TMEM (SPLIT = 1), or, with SPLIT = 3,
+// operands given as three bf16 parts (x = x0 + x1 + x2, each the bf16 rounding of
+// what the earlier parts left over) and C = sum of the six products
+// (0,0) (0,1) (1,0) (1,1) (0,2) (2,0), which reproduces an fp32 product to about
+// 2^-24 relative: this keeps the Gram matrix and the triangular apply of Cholesky-QR
+// fp32-accurate on bf16 tensor cores.  In split mode one pipeline stage holds the
+// three parts of the A tile and of the B tile, and the six products are issued from
+// shared memory.  A split operand is stored [3 * batch][rows][cols]: part i of
+// matrix b is matrix i * batch + b.
 struct GemmP {
   int64_t M, N, K;
   int batch, tiles_m, tiles_n, num_kb, block_n, stages;
   uint32_t idesc, a_bytes, b_bytes, tmem_cols, acc_stride;
-  int npairs;
-  int pa[MAX_PAIRS], pb[MAX_PAIRS];  // split index of A and of B per pair
   float* C;                          // fp32 result (may be null)
   int64_t ldc, c_bs;
   bf16* Cs;                          // three-way bf16 split of the result (may be null)
   int64_t cs_stride;                 // elements between the split parts
   int32_t* flags;
   int32_t need_mask, skip_mask;      // matrices whose flags fail this are skipped
+  int lower_only;                    // skip tiles above the diagonal (symmetric results)
   int64_t max_spins;
 };
 
-__device__ __forceinline__ bool tile_active(const GemmP& p, int b) {
+__device__ __forceinline__ bool tile_active(const GemmP& p, int t, int tiles_per_mat) {
+  if (p.lower_only) {
+    const int rem = t % tiles_per_mat;
+    if ((rem % p.tiles_n) * p.block_n > (rem / p.tiles_n) * BM) return false;
+  }
   if (p.need_mask == 0 && p.skip_mask == 0) return true;
-  const int32_t f = p.flags[b];
+  const int32_t f = p.flags[t / tiles_per_mat];
   return (f & p.need_mask) == p.need_mask && !(f & p.skip_mask);
 }
 
-template <bool A_MN, bool B_MN>
+template <bool A_MN, bool B_MN, int SPLIT>
 __global__ void __launch_bounds__(NT, 1)
     k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const GemmP p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
+  const uint32_t stage_a = SPLIT * p.a_bytes, stage_b = SPLIT * p.b_bytes;
   uint8_t* sA = smem;
-  uint8_t* sB = smem + (size_t)p.stages * p.a_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + (size_t)p.stages * p.b_bytes);
+  uint8_t* sB = smem + (size_t)p.stages * stage_a;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + (size_t)p.stages * stage_b);
   uint64_t* empty = full + p.stages;
   uint64_t* tfull = empty + p.stages;
   uint64_t* tempty = tfull + 2;
@@ -166,7 +170,6 @@ __global__ void __launch_bounds__(NT, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_per_mat = p.tiles_m * p.tiles_n;
   const int ntiles = p.batch * tiles_per_mat;
-  const int kiters = p.num_kb * p.npairs;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -198,31 +201,33 @@ __global__ void __launch_bounds__(NT, 1)
     uint32_t phase = 0;
     int used = 0;  // stages issued at least once
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      if (!tile_active(p, t, tiles_per_mat)) continue;
       const int b = t / tiles_per_mat;
-      if (!tile_active(p, b)) continue;
       const int rem = t % tiles_per_mat;
       const int m0 = (rem / p.tiles_n) * BM;
       const int n0 = (rem % p.tiles_n) * p.block_n;
       bool ok = true;
-      for (int it = 0; it < kiters; ++it) {
-        const int kb = it / p.npairs, pi = it % p.npairs;
-        const int za = p.pa[pi] * p.batch + b, zb = p.pb[pi] * p.batch + b;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
         if (!wait_bounded(empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
-        mbar_expect_tx(full + stage, p.a_bytes + p.b_bytes);
-        uint8_t* a_dst = sA + (size_t)stage * p.a_bytes;
-        uint8_t* b_dst = sB + (size_t)stage * p.b_bytes;
+        mbar_expect_tx(full + stage, stage_a + stage_b);
         const int k0 = kb * BK;
-        if (A_MN) {  // A^T stored [K][M]: boxes of 64 (M) x 64 (K)
-          tma_load_3d(a_dst, &tmA, full + stage, m0, k0, za);
-          tma_load_3d(a_dst + 8192, &tmA, full + stage, m0 + 64, k0, za);
-        } else {     // A stored [M][K]: 128 rows of 64 K elements
-          tma_load_3d(a_dst, &tmA, full + stage, k0, m0, za);
-        }
-        if (B_MN) {  // B stored [K][N]: boxes of 64 (N) x 64 (K)
-          for (int j = 0; j < p.block_n / 64; ++j)
-            tma_load_3d(b_dst + j * 8192, &tmB, full + stage, n0 + 64 * j, k0, zb);
-        } else {     // B stored [N][K]: block_n rows of 64 K elements
-          tma_load_3d(b_dst, &tmB, full + stage, k0, n0, zb);
+#pragma unroll
+        for (int part = 0; part < SPLIT; ++part) {
+          uint8_t* a_dst = sA + (size_t)stage * stage_a + part * p.a_bytes;
+          uint8_t* b_dst = sB + (size_t)stage * stage_b + part * p.b_bytes;
+          const int z = part * p.batch + b;
+          if (A_MN) {  // A^T stored [K][M]: boxes of 64 (M) x 64 (K)
+            tma_load_3d(a_dst, &tmA, full + stage, m0, k0, z);
+            tma_load_3d(a_dst + 8192, &tmA, full + stage, m0 + 64, k0, z);
+          } else {     // A stored [M][K]: 128 rows of 64 K elements
+            tma_load_3d(a_dst, &tmA, full + stage, k0, m0, z);
+          }
+          if (B_MN) {  // B stored [K][N]: boxes of 64 (N) x 64 (K)
+            for (int j = 0; j < p.block_n / 64; ++j)
+              tma_load_3d(b_dst + j * 8192, &tmB, full + stage, n0 + 64 * j, k0, z);
+          } else {     // B stored [N][K]: block_n rows of 64 K elements
+            tma_load_3d(b_dst, &tmB, full + stage, k0, n0, z);
+          }
         }
         if (used < p.stages) ++used;
         if (++stage == p.stages) { stage = 0; phase ^= 1; }
@@ -239,29 +244,38 @@ __global__ void __launch_bounds__(NT, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
+    // split products, smallest terms first: (2,0) (0,2) (1,1) (1,0) (0,1) (0,0)
+    constexpr int NPROD = SPLIT == 3 ? 6 : 1;
+    const int pa[6] = {2, 0, 1, 1, 0, 0};
+    const int pb[6] = {0, 2, 1, 0, 1, 0};
     int stage = 0;
     uint32_t phase = 0;
     int lt = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      if (!tile_active(p, t / tiles_per_mat)) continue;
+      if (!tile_active(p, t, tiles_per_mat)) continue;
       const int acc = lt & 1;
       const uint32_t acc_phase = (lt >> 1) & 1;
       if (!wait_bounded(tempty + acc, acc_phase ^ 1, p.max_spins, abort)) break;
       tc_fence_after();
       const uint32_t d = tmem + acc * p.acc_stride;
       bool ok = true;
-      for (int it = 0; it < kiters; ++it) {
+      for (int kb = 0; kb < p.num_kb; ++kb) {
         if (!wait_bounded(full + stage, phase, p.max_spins, abort)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(sA + (size_t)stage * p.a_bytes);
-        const uint32_t b_base = smem_u32(sB + (size_t)stage * p.b_bytes);
+        const uint32_t a_base = smem_u32(sA + (size_t)stage * stage_a);
+        const uint32_t b_base = smem_u32(sB + (size_t)stage * stage_b);
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k) {
-          const uint64_t ad = A_MN ? sw128_desc(a_base + k * 2048, 8192, 1024)
-                                   : sw128_desc(a_base + k * 32, 16, 1024);
-          const uint64_t bd = B_MN ? sw128_desc(b_base + k * 2048, 8192, 1024)
-                                   : sw128_desc(b_base + k * 32, 16, 1024);
-          mma_bf16(d, ad, bd, p.idesc, (it | k) != 0);
+#pragma unroll
+          for (int q = 0; q < NPROD; ++q) {
+            const uint32_t ab = a_base + (SPLIT == 3 ? pa[q] : 0) * p.a_bytes;
+            const uint32_t bb = b_base + (SPLIT == 3 ? pb[q] : 0) * p.b_bytes;
+            const uint64_t ad = A_MN ? sw128_desc(ab + k * 2048, 8192, 1024)
+                                     : sw128_desc(ab + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sw128_desc(bb + k * 2048, 8192, 1024)
+                                     : sw128_desc(bb + k * 32, 16, 1024);
+            mma_bf16(d, ad, bd, p.idesc, (kb | k | q) != 0);
+          }
         }
         mma_commit(empty + stage);
         if (++stage == p.stages) { stage = 0; phase ^= 1; }
@@ -278,8 +292,8 @@ __global__ void __launch_bounds__(NT, 1)
     int lt = 0;
     int t = blockIdx.x;
     for (; t < ntiles; t += gridDim.x) {
+      if (!tile_active(p, t, tiles_per_mat)) continue;
       const int b = t / tiles_per_mat;
-      if (!tile_active(p, b)) continue;
       const int acc = lt & 1;
       const uint32_t acc_phase = (lt >> 1) & 1;
       if (!wait_bounded(tfull + acc, acc_phase, p.max_spins, abort)) break;
@@ -337,20 +351,20 @@ static uint32_t pow2_cols(uint32_t c) {
   return v;
 }
 
-template <bool A_MN, bool B_MN>
+template <bool A_MN, bool B_MN, int SPLIT>
 static cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, GemmP p,
                                cudaStream_t s) {
   p.a_bytes = BM * BK * 2;
   p.b_bytes = (uint32_t)p.block_n * BK * 2;
-  const size_t stage_bytes = p.a_bytes + p.b_bytes;
+  const size_t stage_bytes = (size_t)SPLIT * (p.a_bytes + p.b_bytes);
   int stages = (int)((200 * 1024) / stage_bytes);
   if (stages > 8) stages = 8;
-  if (stages < 2) stages = 2;
+  if (stages < 1) return cudaErrorInvalidValue;
   p.stages = stages;
   p.acc_stride = (uint32_t)p.block_n;
   p.tmem_cols = pow2_cols(2 * p.block_n);
   const size_t smem = 1024 + stages * stage_bytes + (2 * stages + 5) * 8 + 16;
-  auto kern = k_tc_gemm<A_MN, B_MN>;
+  auto kern = k_tc_gemm<A_MN, B_MN, SPLIT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int ntiles = p.batch * p.tiles_m * p.tiles_n;
@@ -364,16 +378,6 @@ static int pick_block_n(int64_t r, int mult) {
   int64_t bn = (r + tiles - 1) / tiles;
   bn = (bn + mult - 1) / mult * mult;
   return (int)bn;
-}
-
-static void set_pairs(GemmP& p, int npairs) {
-  static const int A6[6] = {2, 0, 1, 1, 0, 0};  // small terms first
-  static const int B6[6] = {0, 2, 1, 0, 1, 0};
-  p.npairs = npairs;
-  for (int i = 0; i < npairs; ++i) {
-    p.pa[i] = npairs == 1 ? 0 : A6[i];
-    p.pb[i] = npairs == 1 ? 0 : B6[i];
-  }
 }
 
 }  // namespace tc
@@ -395,13 +399,12 @@ cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, bf16* P0s, int
   p.tiles_m = (int)((m + BM - 1) / BM);
   p.tiles_n = (int)((r + bn - 1) / bn);
   p.num_kb = (int)((n + BK - 1) / BK);
-  set_pairs(p, 1);
   p.idesc = idesc_bf16(BM, bn, false, false);
   p.C = P0; p.ldc = r; p.c_bs = m * r;
   p.Cs = P0s; p.cs_stride = (int64_t)count * m * r;
   p.flags = flags;
   p.max_spins = max_spins;
-  cudaError_t e = launch_gemm<false, false>(ma, mb, p, s);
+  cudaError_t e = launch_gemm<false, false, 1>(ma, mb, p, s);
   if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
   return e;
 }
@@ -423,12 +426,11 @@ cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, int count, int
   p.tiles_m = (int)((n + BM - 1) / BM);
   p.tiles_n = (int)((r + bn - 1) / bn);
   p.num_kb = (int)((m + BK - 1) / BK);
-  set_pairs(p, 1);
   p.idesc = idesc_bf16(BM, bn, true, true);
   p.C = R; p.ldc = r; p.c_bs = n * r;
   p.flags = flags;
   p.max_spins = max_spins;
-  cudaError_t e = launch_gemm<true, true>(ma, mb, p, s);
+  cudaError_t e = launch_gemm<true, true, 1>(ma, mb, p, s);
   if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
   return e;
 }
@@ -439,7 +441,8 @@ cudaError_t tc_gram(const bf16* Xs, float* W, int count, int64_t m, int64_t r, i
   using namespace tc;
   *nlaunch = 0;
   *done = false;
-  const int bn = pick_block_n(r, 64);
+  // 128 x 128 tiles of the symmetric result; only those on or below the diagonal
+  const int bn = r <= 64 ? 64 : 128;
   CUtensorMap ma, mb;
   if (!map3d(&ma, Xs, true, r, m, 3 * (uint64_t)count, 64, BK)) return cudaSuccess;
   if (!map3d(&mb, Xs, true, r, m, 3 * (uint64_t)count, 64, BK)) return cudaSuccess;
@@ -450,12 +453,12 @@ cudaError_t tc_gram(const bf16* Xs, float* W, int count, int64_t m, int64_t r, i
   p.tiles_m = (int)((r + BM - 1) / BM);
   p.tiles_n = (int)((r + bn - 1) / bn);
   p.num_kb = (int)((m + BK - 1) / BK);
-  set_pairs(p, 6);
   p.idesc = idesc_bf16(BM, bn, true, true);
   p.C = W; p.ldc = r; p.c_bs = r * r;
   p.flags = flags; p.need_mask = need; p.skip_mask = skip;
+  p.lower_only = bn == BM;
   p.max_spins = max_spins;
-  cudaError_t e = launch_gemm<true, true>(ma, mb, p, s);
+  cudaError_t e = launch_gemm<true, true, 3>(ma, mb, p, s);
   if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
   return e;
 }
@@ -466,7 +469,7 @@ cudaError_t tc_apply(const bf16* Xs, const bf16* Ls, float* Y, bf16* Ys, int cou
   using namespace tc;
   *nlaunch = 0;
   *done = false;
-  const int bn = pick_block_n(r, 16);
+  const int bn = r <= 128 ? (int)r : 128;   // three parts of A and B per stage
   CUtensorMap ma, mb;
   if (!map3d(&ma, Xs, true, r, m, 3 * (uint64_t)count, BK, BM)) return cudaSuccess;
   if (!map3d(&mb, Ls, true, r, r, 3 * (uint64_t)count, BK, bn)) return cudaSuccess;
@@ -477,13 +480,12 @@ cudaError_t tc_apply(const bf16* Xs, const bf16* Ls, float* Y, bf16* Ys, int cou
   p.tiles_m = (int)((m + BM - 1) / BM);
   p.tiles_n = (int)((r + bn - 1) / bn);
   p.num_kb = (int)((r + BK - 1) / BK);
-  set_pairs(p, 6);
   p.idesc = idesc_bf16(BM, bn, false, false);
   p.C = Y; p.ldc = r; p.c_bs = m * r;
   p.Cs = Ys; p.cs_stride = (int64_t)count * m * r;
   p.flags = flags; p.need_mask = need; p.skip_mask = skip;
   p.max_spins = max_spins;
-  cudaError_t e = launch_gemm<false, false>(ma, mb, p, s);
+  cudaError_t e = launch_gemm<false, false, 3>(ma, mb, p, s);
   if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
   return e;
 }
@@ -502,8 +504,10 @@ struct UpdP {
 constexpr uint32_t UPD_A_BYTES = BM * BK * 2;           // 16 KB
 constexpr uint32_t UPD_B_BYTES = 2 * UPD_BN * BK * 2;   // 32 KB (R rows then Q rows)
 constexpr uint32_t SLAB_BYTES = BM * SLAB * 4;          // 16 KB per tensor
+// + one 128 x 32 staging slab each for M' and X', so a load slab is released as soon
+// as it has been read, without waiting for the TMA store of the results
 constexpr size_t UPD_SMEM = 1024 + UPD_STAGES * (UPD_A_BYTES + UPD_B_BYTES) +
-                            SLAB_STAGES * 3 * SLAB_BYTES + 256;
+                            SLAB_STAGES * 3 * SLAB_BYTES + 2 * SLAB_BYTES + 256;
 
 __global__ void __launch_bounds__(NT, 1)
     k_tc_update(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmR,
@@ -516,7 +520,8 @@ __global__ void __launch_bounds__(NT, 1)
   uint8_t* sA = smem;
   uint8_t* sB = sA + UPD_STAGES * UPD_A_BYTES;
   uint8_t* sS = sB + UPD_STAGES * UPD_B_BYTES;  // [stage][M | G | X] slabs
-  uint64_t* full = reinterpret_cast<uint64_t*>(sS + SLAB_STAGES * 3 * SLAB_BYTES);
+  uint8_t* sO = sS + SLAB_STAGES * 3 * SLAB_BYTES;  // staging of M' | X'
+  uint64_t* full = reinterpret_cast<uint64_t*>(sO + 2 * SLAB_BYTES);
   uint64_t* empty = full + UPD_STAGES;
   uint64_t* sfull = empty + UPD_STAGES;
   uint64_t* sempty = sfull + SLAB_STAGES;
@@ -675,15 +680,20 @@ __global__ void __launch_bounds__(NT, 1)
         tmem_wait_ld();
         if (!wait_bounded(sfull + stage, phase, p.max_spins, abort)) { ok = false; break; }
         uint8_t* slab = sS + stage * 3 * SLAB_BYTES;
-        uint8_t* rm = slab + row * 128;
-        uint8_t* rg = slab + SLAB_BYTES + row * 128;
-        uint8_t* rx = slab + 2 * SLAB_BYTES + row * 128;
+        const uint8_t* rm = slab + row * 128;
+        const uint8_t* rg = slab + SLAB_BYTES + row * 128;
+        const uint8_t* rx = slab + 2 * SLAB_BYTES + row * 128;
+        uint8_t* om = sO + row * 128;
+        uint8_t* ox = sO + SLAB_BYTES + row * 128;
+        // this warp's previous store must have finished reading its staging rows
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const int off = ((c ^ (row & 7)) << 4);
-          float4 mv = *reinterpret_cast<float4*>(rm + off);
+          float4 mv = *reinterpret_cast<const float4*>(rm + off);
           const float4 gv = *reinterpret_cast<const float4*>(rg + off);
-          float4 xv = *reinterpret_cast<float4*>(rx + off);
+          float4 xv = *reinterpret_cast<const float4*>(rx + off);
           mv.x = (mv.x + gv.x) - p.omm * ar[4 * c + 0];
           mv.y = (mv.y + gv.y) - p.omm * ar[4 * c + 1];
           mv.z = (mv.z + gv.z) - p.omm * ar[4 * c + 2];
@@ -692,17 +702,17 @@ __global__ void __launch_bounds__(NT, 1)
           xv.y = xv.y - p.lrs * aq[4 * c + 1];
           xv.z = xv.z - p.lrs * aq[4 * c + 2];
           xv.w = xv.w - p.lrs * aq[4 * c + 3];
-          *reinterpret_cast<float4*>(rm + off) = mv;
-          *reinterpret_cast<float4*>(rx + off) = xv;
+          *reinterpret_cast<float4*>(om + off) = mv;
+          *reinterpret_cast<float4*>(ox + off) = xv;
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sempty + stage);  // the load slab is free again
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&tmMs, slab + ew * 32 * 128, n0 + sl * SLAB, m0 + ew * 32, b);
-          tma_store_3d(&tmXs, slab + 2 * SLAB_BYTES + ew * 32 * 128, n0 + sl * SLAB, m0 + ew * 32, b);
+          tma_store_3d(&tmMs, sO + ew * 32 * 128, n0 + sl * SLAB, m0 + ew * 32, b);
+          tma_store_3d(&tmXs, sO + SLAB_BYTES + ew * 32 * 128, n0 + sl * SLAB, m0 + ew * 32, b);
           bulk_commit();
-          bulk_wait_read0();
-          mbar_arrive(sempty + stage);
         }
         __syncwarp();
         if (++stage == SLAB_STAGES) { stage = 0; phase ^= 1; }

@@ -78,6 +78,7 @@ def test_defaults():
     ((1, 256, 16, 32), dion.ERR_UNSUPPORTED_SHAPE),      # r > n
     ((1, 256, 128, 0), dion.ERR_UNSUPPORTED_SHAPE),
     ((1, 1 << 31, 128, 32), dion.ERR_UNSUPPORTED_SHAPE),  # too large
+    ((65536, 32, 16, 16), dion.ERR_UNSUPPORTED_SHAPE),     # too many matrices in one bucket
 ])
 def test_init_shape_checks(bucket, code):
     c, h, ws = _init([bucket])
