@@ -71,7 +71,10 @@ enum {
 
 /* Arithmetic of the four rank-r contractions (B Q, B^T P, P R^T, P Q^T). */
 typedef enum dion_precision {
-  DION_PREC_FP32 = 0,  /* fp32 operands, fp32 accumulation                           */
+  DION_PREC_FP32 = 0,  /* fp32-accurate: on CUDA cores fp32 FMA; on the tensor path the
+                          operands are split into three bf16 parts (x = x0 + x1 + x2)
+                          and B Q, B^T P sum six part products (about 2^-24 relative),
+                          the update three (about 2^-17); fp32 accumulation          */
   DION_PREC_BF16 = 1   /* B, Q, P, R rounded to bf16 (round to nearest even), fp32
                           accumulation; Gram, Cholesky and the triangular apply stay
                           fp32                                                       */

@@ -46,7 +46,7 @@ struct Plan {
   int64_t mat0;
   int nsplit;
   size_t off_Bg, off_Qg, off_P0, off_P, off_P2, off_Pg, off_W, off_Linv, off_dinv, off_R, off_Rg,
-      off_Qng, off_part, off_flags, off_stats, off_P0s, off_Ps, off_Linvs;
+      off_Qng, off_part, off_flags, off_stats, off_P0s, off_Ps, off_Linvs, off_sched;
 };
 
 struct EventPair {
@@ -140,23 +140,23 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
   const dion_options& o = c.h->opt;
   const bool bf = o.precision == DION_PREC_BF16;
   const bool tensor = o.kernel_path == DION_PATH_TENSOR;
-  const int ge = bf ? 2 : 4;
-  (void)ge;
+  const bool split = tensor && !bf;  // fp32 contractions from three-way bf16 splits
   void* Bg = ws + p.off_Bg;
   void* Qg = ws + p.off_Qg;
   float* P0 = reinterpret_cast<float*>(ws + p.off_P0);
   float* P = reinterpret_cast<float*>(ws + p.off_P);
   float* P2 = reinterpret_cast<float*>(ws + p.off_P2);
-  void* Pg = bf ? (void*)(ws + p.off_Pg) : (void*)P;
+  void* Pg = (bf || split) ? (void*)(ws + p.off_Pg) : (void*)P;
   float* W = reinterpret_cast<float*>(ws + p.off_W);
   float* Linv = reinterpret_cast<float*>(ws + p.off_Linv);
   float* dinv = reinterpret_cast<float*>(ws + p.off_dinv);
   float* R = reinterpret_cast<float*>(ws + p.off_R);
-  void* Rg = bf ? (void*)(ws + p.off_Rg) : (void*)R;
-  void* Qng = bf ? (void*)(ws + p.off_Qng) : (void*)bp.Q;
+  void* Rg = (bf || split) ? (void*)(ws + p.off_Rg) : (void*)R;
+  void* Qng = (bf || split) ? (void*)(ws + p.off_Qng) : (void*)bp.Q;
   float* part = reinterpret_cast<float*>(ws + p.off_part);
   int32_t* flags = reinterpret_cast<int32_t*>(ws + p.off_flags);
   float* stats = reinterpret_cast<float*>(ws + p.off_stats);
+  int* sched = reinterpret_cast<int*>(ws + p.off_sched);
   __nv_bfloat16* P0s = reinterpret_cast<__nv_bfloat16*>(ws + p.off_P0s);
   __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ps);
   __nv_bfloat16* Linvs = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Linvs);
@@ -165,22 +165,52 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
   const int cnt = p.count;
   cudaStream_t s = c.s;
 
-  DION_LAUNCH(c, 1, dion::launch_init_flags(flags, stats, cnt,
+  DION_LAUNCH(c, 1, dion::launch_init_flags(flags, stats, sched, cnt,
                                             o.orth_mode == DION_ORTH_HOUSEHOLDER ? DION_MAT_FALLBACK : 0,
                                             s));
 
-  // step 1: B = M + G in the precision of the contractions
-  begin_cls(c, DION_KCLASS_FORM_B);
-  DION_LAUNCH(c, 1, dion::launch_form_b(bp.M, bp.G, Bg, bf, (int64_t)cnt * m * n, s));
-  end_cls(c);
+  // steps 1 and 2 fused on the tensor path when one N tile covers r: B = M + G is
+  // formed in shared memory, fed to the MMA and stored once as bf16
+  const bool fused_bq = tensor && bf && r <= 256;
 
   begin_cls(c, DION_KCLASS_PREP_Q);
-  DION_LAUNCH(c, 1, dion::launch_prep_q(bp.Q, Qg, bf, cnt, n, r, s));
+  if (split)
+    DION_LAUNCH(c, 1, dion::launch_prep_q_split(bp.Q, Qg, cnt, n, r, s));
+  else
+    DION_LAUNCH(c, 1, dion::launch_prep_q(bp.Q, Qg, bf, cnt, n, r, s));
   end_cls(c);
+
+  // step 1: B = M + G in the precision of the contractions
+  if (!fused_bq) {
+    begin_cls(c, DION_KCLASS_FORM_B);
+    if (split)
+      DION_LAUNCH(c, 1, dion::launch_form_b_split(bp.M, bp.G, Bg, (int64_t)cnt * m * n, s));
+    else
+      DION_LAUNCH(c, 1, dion::launch_form_b(bp.M, bp.G, Bg, bf, (int64_t)cnt * m * n, s));
+    end_cls(c);
+  }
 
   // step 2: P0 = B Q
   begin_cls(c, DION_KCLASS_GEMM_BQ);
-  {
+  if (fused_bq) {
+    int nl = 0;
+    bool done = false;
+    cudaError_t e = dion::tc_formb_bq(bp.M, bp.G, Qg, Bg, P0s, cnt, m, n, r, o.max_wait_spins,
+                                      flags, s, &nl, &done);
+    c.launches += nl;
+    if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_formb_bq: %s", cudaGetErrorString(e));
+    if (!done) return fail(DION_ERR_CUDA, "tc_formb_bq: %s", dion::tc_map_error());
+    p0s_ready = true;
+  } else if (split) {
+    int nl = 0;
+    bool done = false;
+    cudaError_t e = dion::tc_gemm_bq_split((const __nv_bfloat16*)Bg, (const __nv_bfloat16*)Qg, P0s,
+                                           cnt, m, n, r, o.max_wait_spins, flags, s, &nl, &done);
+    c.launches += nl;
+    if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_gemm_bq_split: %s", cudaGetErrorString(e));
+    if (!done) return fail(DION_ERR_CUDA, "tc_gemm_bq_split: %s", dion::tc_map_error());
+    p0s_ready = true;
+  } else {
     bool done = false;
     if (tensor && bf) {
       int nl = 0;
@@ -280,7 +310,8 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
     }
     DION_LAUNCH(c, 1, dion::launch_householder(P0, p0s_ready ? P0s : nullptr, P2, P0, P, flags,
                                                cnt, m, r, s));
-    DION_LAUNCH(c, 1, dion::launch_finalize_p(P, P2, Pg, bf, flags, cnt, m, r, P, s));
+    DION_LAUNCH(c, 1, dion::launch_finalize_p(P2, Pg, bf ? 1 : (split ? 2 : 0), flags, cnt, m, r,
+                                              P, s));
   }
   end_cls(c);
 
@@ -288,7 +319,15 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
   begin_cls(c, DION_KCLASS_GEMM_BTP);
   {
     bool done = false;
-    if (tensor && bf) {
+    if (split) {
+      int nl = 0;
+      cudaError_t e = dion::tc_gemm_btp_split((const __nv_bfloat16*)Bg, (const __nv_bfloat16*)Pg, R,
+                                              cnt, m, n, r, o.max_wait_spins, flags, s, &nl, &done);
+      c.launches += nl;
+      if (e != cudaSuccess)
+        return fail(DION_ERR_CUDA, "tc_gemm_btp_split: %s", cudaGetErrorString(e));
+      if (!done) return fail(DION_ERR_CUDA, "tc_gemm_btp_split: %s", dion::tc_map_error());
+    } else if (tensor && bf) {
       int nl = 0;
       cudaError_t e = dion::tc_gemm_btp(Bg, Pg, R, cnt, m, n, r, o.max_wait_spins, flags, s, &nl, &done);
       c.launches += nl;
@@ -308,7 +347,8 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
 
   // step 6: Q = colnorm(R), plus the GEMM copies of R and Q for the update
   begin_cls(c, DION_KCLASS_COLNORM);
-  DION_LAUNCH(c, 2, dion::launch_colnorm(R, bp.Q, Rg, Qng, bf, part, p.nsplit, flags, cnt, n, r, s));
+  DION_LAUNCH(c, 2, dion::launch_colnorm(R, bp.Q, Rg, Qng, bf ? 1 : (split ? 2 : 0), part,
+                                         p.nsplit, flags, cnt, n, r, s));
   end_cls(c);
 
   // steps 5 and 7: M <- B - (1 - mu) P R^T and X <- X - lr s P Q^T in one pass
@@ -316,10 +356,10 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
   {
     bool done = false;
     const float lrs = lr * p.scale;
-    if (tensor && bf) {
+    if (tensor) {
       int nl = 0;
-      cudaError_t e = dion::tc_update(Pg, Rg, Qng, bp.G, bp.M, bp.X, cnt, m, n, r, o.mu, lrs,
-                                      o.max_wait_spins, flags, s, &nl, &done);
+      cudaError_t e = dion::tc_update(Pg, Rg, Qng, split, bp.G, bp.M, bp.X, cnt, m, n, r, o.mu,
+                                      lrs, o.max_wait_spins, flags, sched, s, &nl, &done);
       c.launches += nl;
       if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_update: %s", cudaGetErrorString(e));
       if (!done) return fail(DION_ERR_CUDA, "tc_update: %s", dion::tc_map_error());
@@ -421,7 +461,9 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
   dion_status st = check_options(o);
   if (st != DION_OK) return st;
   const bool bf = o.precision == DION_PREC_BF16;
-  const size_t ge = bf ? 2 : 4;
+  // fp32 precision on the tensor path keeps B, Q, P, R as three bf16 parts
+  const bool split = !bf && o.kernel_path == DION_PATH_TENSOR;
+  const size_t ge = bf ? 2 : (split ? 6 : 4);
   std::vector<Plan> plans;
   size_t off = 0;
   int64_t mats = 0;
@@ -462,13 +504,13 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
     p.off_P0 = take(c * d.m * d.r * 4);
     p.off_P = take(c * d.m * d.r * 4);
     p.off_P2 = take(c * d.m * d.r * 4);
-    p.off_Pg = bf ? take(c * d.m * d.r * 2) : 0;
+    p.off_Pg = (bf || split) ? take(c * d.m * d.r * ge) : 0;
     p.off_W = take(c * d.r * d.r * 4);
     p.off_Linv = take(c * d.r * d.r * 4);
     p.off_dinv = take(dion::chol_dinv_floats(d.count, d.r) * 4);
     p.off_R = take(c * d.n * d.r * 4);
-    p.off_Rg = bf ? take(c * d.n * d.r * 2) : 0;
-    p.off_Qng = bf ? take(c * d.n * d.r * 2) : 0;
+    p.off_Rg = (bf || split) ? take(c * d.n * d.r * ge) : 0;
+    p.off_Qng = (bf || split) ? take(c * d.n * d.r * ge) : 0;
     p.off_part = take(c * p.nsplit * d.r * 4);
     p.off_flags = take(c * 4);
     p.off_stats = take(c * 8);
@@ -476,6 +518,7 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
     p.off_P0s = take(c * d.m * d.r * 6);
     p.off_Ps = take(c * d.m * d.r * 6);
     p.off_Linvs = take(c * d.r * d.r * 6);
+    p.off_sched = take(64);  // tile counters of the dynamically scheduled kernels
     plans.push_back(p);
   }
   dion_ctx* h = new (std::nothrow) dion_ctx();

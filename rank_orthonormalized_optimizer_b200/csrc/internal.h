@@ -39,13 +39,21 @@ cudaError_t launch_form_b(const float* M, const float* G, void* Bg, bool use_bf1
                           cudaStream_t s);
 cudaError_t launch_prep_q(const float* Q, void* Qg, bool use_bf16, int count, int64_t n, int64_t r,
                           cudaStream_t s);
-cudaError_t launch_init_flags(int32_t* flags, float* stats, int count, int32_t init_bits,
-                              cudaStream_t s);
-cudaError_t launch_finalize_p(const float* P, const float* P2, void* Pg, bool use_bf16,
-                              const int32_t* flags, int count, int64_t m, int64_t r,
-                              float* P_out, cudaStream_t s);
+// three-way bf16 splits ([3][...] planes) for fp32 contractions on the tensor cores
+cudaError_t launch_form_b_split(const float* M, const float* G, void* Bs, int64_t elems,
+                                cudaStream_t s);
+cudaError_t launch_prep_q_split(const float* Q, void* Qs, int count, int64_t n, int64_t r,
+                                cudaStream_t s);
+// Zero the per-matrix flags (or set init_bits), the Cholesky statistics and the 16
+// tile counters of the bucket's dynamically scheduled kernels.
+cudaError_t launch_init_flags(int32_t* flags, float* stats, int* sched, int count,
+                              int32_t init_bits, cudaStream_t s);
+// mode 0: fp32 P only; 1: + bf16 copy Pg; 2: + three-way bf16 split Pg
+cudaError_t launch_finalize_p(const float* P2, void* Pg, int mode, const int32_t* flags,
+                              int count, int64_t m, int64_t r, float* P, cudaStream_t s);
 int colnorm_splits(int count, int64_t n);
-cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, bool use_bf16,
+// mode 0: Q only; 1: + bf16 R, Q; 2: + three-way bf16 splits of R, Q
+cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, int mode,
                            float* part, int nsplit, int32_t* flags, int count, int64_t n,
                            int64_t r, cudaStream_t s);
 cudaError_t launch_split3(const float* src, void* dst, int64_t n, int64_t dst_stride,

@@ -58,6 +58,36 @@ __global__ void __launch_bounds__(256) k_form_b(const float4* __restrict__ M,
   }
 }
 
+// B = M + G kept to fp32 accuracy as three bf16 parts [3][elems] (for the fp32
+// contractions on bf16 tensor cores): 8 bytes read, 6 written per element.
+__global__ void __launch_bounds__(256) k_form_b_split(const float4* __restrict__ M,
+                                                       const float4* __restrict__ G,
+                                                       bf16* __restrict__ Bs, int64_t n4,
+                                                       int64_t stride) {
+  const int64_t step = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += step) {
+    const float4 a = __ldcs(M + i), g = __ldcs(G + i);
+    const float v[4] = {a.x + g.x, a.y + g.y, a.z + g.z, a.w + g.w};
+    __align__(8) bf16 h[4], m[4], l[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) split3_bf16(v[q], h[q], m[q], l[q]);
+    reinterpret_cast<uint2*>(Bs)[i] = *reinterpret_cast<const uint2*>(h);
+    reinterpret_cast<uint2*>(Bs + stride)[i] = *reinterpret_cast<const uint2*>(m);
+    reinterpret_cast<uint2*>(Bs + 2 * stride)[i] = *reinterpret_cast<const uint2*>(l);
+  }
+}
+
+cudaError_t launch_form_b_split(const float* M, const float* G, void* Bs, int64_t elems,
+                                cudaStream_t s) {
+  const int64_t n4 = elems / 4;
+  int64_t grid = (n4 + 255) / 256;
+  if (grid > (int64_t)sm_count() * 8) grid = (int64_t)sm_count() * 8;
+  if (grid < 1) grid = 1;
+  k_form_b_split<<<(unsigned)grid, 256, 0, s>>>((const float4*)M, (const float4*)G, (bf16*)Bs, n4,
+                                                elems);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_form_b(const float* M, const float* G, void* Bg, bool use_bf16, int64_t elems,
                           cudaStream_t s) {
   const int64_t n4 = elems / 4;
@@ -75,9 +105,9 @@ cudaError_t launch_form_b(const float* M, const float* G, void* Bg, bool use_bf1
 // Qg[b][j][i] = Q[b][i][j]: the n x r factor transposed to r x n so that the
 // contraction B Q reads both operands along n (the reduction axis).  64 x 64 tiles:
 // float4 loads along r, 4-element stores along n.
-template <typename T>
+template <typename T, bool SPLIT>
 __global__ void __launch_bounds__(256) k_prep_q(const float* __restrict__ Q, T* __restrict__ Qg,
-                                                 int64_t n, int64_t r) {
+                                                 int64_t n, int64_t r, int64_t split_stride) {
   __shared__ float tile[64][65];
   const int64_t b = blockIdx.z;
   const float* q = Q + b * n * r;
@@ -100,7 +130,15 @@ __global__ void __launch_bounds__(256) k_prep_q(const float* __restrict__ Q, T* 
     const int64_t j = j0 + y, i = i0 + 4 * x4;
     if (j >= r || i >= n) continue;
     T* dst = qg + j * n + i;
-    if (i + 3 < n) {
+    if (SPLIT) {  // three bf16 parts, each plane [count][r][n]
+      for (int q2 = 0; q2 < 4 && i + q2 < n; ++q2) {
+        bf16 h, m, l;
+        split3_bf16(tile[y][4 * x4 + q2], h, m, l);
+        reinterpret_cast<bf16*>(dst)[q2] = h;
+        reinterpret_cast<bf16*>(dst)[q2 + split_stride] = m;
+        reinterpret_cast<bf16*>(dst)[q2 + 2 * split_stride] = l;
+      }
+    } else if (i + 3 < n) {
       if (sizeof(T) == 2) {
         __nv_bfloat162 lo = __floats2bfloat162_rn(tile[y][4 * x4], tile[y][4 * x4 + 1]);
         __nv_bfloat162 hi = __floats2bfloat162_rn(tile[y][4 * x4 + 2], tile[y][4 * x4 + 3]);
@@ -122,9 +160,16 @@ cudaError_t launch_prep_q(const float* Q, void* Qg, bool use_bf16, int count, in
                           cudaStream_t s) {
   dim3 grid((unsigned)((r + 63) / 64), (unsigned)((n + 63) / 64), (unsigned)count);
   if (use_bf16)
-    k_prep_q<bf16><<<grid, 256, 0, s>>>(Q, (bf16*)Qg, n, r);
+    k_prep_q<bf16, false><<<grid, 256, 0, s>>>(Q, (bf16*)Qg, n, r, 0);
   else
-    k_prep_q<float><<<grid, 256, 0, s>>>(Q, (float*)Qg, n, r);
+    k_prep_q<float, false><<<grid, 256, 0, s>>>(Q, (float*)Qg, n, r, 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep_q_split(const float* Q, void* Qs, int count, int64_t n, int64_t r,
+                                cudaStream_t s) {
+  dim3 grid((unsigned)((r + 63) / 64), (unsigned)((n + 63) / 64), (unsigned)count);
+  k_prep_q<bf16, true><<<grid, 256, 0, s>>>(Q, (bf16*)Qs, n, r, (int64_t)count * n * r);
   return cudaGetLastError();
 }
 
@@ -154,8 +199,10 @@ cudaError_t launch_split3(const float* src, void* dst, int64_t n, int64_t dst_st
 }
 
 // ---------------------------------------------------------- flags and status
-__global__ void k_init_flags(int32_t* flags, float* stats, int count, int32_t init_bits) {
+__global__ void k_init_flags(int32_t* flags, float* stats, int* sched, int count,
+                             int32_t init_bits) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < 16) sched[b] = 0;
   if (b < count) {
     flags[b] = init_bits;
     stats[2 * b] = 3.0e38f;  // running min of diag(L)
@@ -163,9 +210,10 @@ __global__ void k_init_flags(int32_t* flags, float* stats, int count, int32_t in
   }
 }
 
-cudaError_t launch_init_flags(int32_t* flags, float* stats, int count, int32_t init_bits,
-                              cudaStream_t s) {
-  k_init_flags<<<(count + 255) / 256, 256, 0, s>>>(flags, stats, count, init_bits);
+cudaError_t launch_init_flags(int32_t* flags, float* stats, int* sched, int count,
+                              int32_t init_bits, cudaStream_t s) {
+  const int n = count > 16 ? count : 16;
+  k_init_flags<<<(n + 255) / 256, 256, 0, s>>>(flags, stats, sched, count, init_bits);
   return cudaGetLastError();
 }
 
@@ -183,21 +231,31 @@ cudaError_t launch_write_status(const int32_t* flags, int32_t* d_status, int cou
 // ------------------------------------------------------------- final P
 // P holds the first Cholesky-QR pass or the Householder result; P2 the
 // second pass.  Picks per matrix, then writes the GEMM copy Pg (bf16 mode).
-template <bool BF16>
+// MODE 0: fp32 only; 1: + bf16 copy; 2: + three-way bf16 split (planes of count*m*r)
+template <int MODE>
 __global__ void k_finalize_p(float* __restrict__ P, const float* __restrict__ P2,
                              void* __restrict__ Pg, const int32_t* __restrict__ flags,
-                             int64_t mr4) {
+                             int64_t mr4, int64_t plane) {
   const int64_t b = blockIdx.y;
   const int32_t f = flags[b];
   const bool take2 = (f & F_CHOLQR2) && !(f & F_FALLBACK);
-  if (!take2 && !BF16) return;
+  if (!take2 && MODE == 0) return;
   float4* p = reinterpret_cast<float4*>(P) + b * mr4;
   const float4* p2 = reinterpret_cast<const float4*>(P2) + b * mr4;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < mr4;
        i += (int64_t)gridDim.x * blockDim.x) {
     float4 v = take2 ? p2[i] : p[i];
     if (take2) p[i] = v;
-    if (BF16) {
+    if (MODE == 2) {
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+      __align__(8) bf16 h[4], m[4], l[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) split3_bf16(vv[q], h[q], m[q], l[q]);
+      bf16* o = reinterpret_cast<bf16*>(Pg);
+      reinterpret_cast<uint2*>(o)[b * mr4 + i] = *reinterpret_cast<const uint2*>(h);
+      reinterpret_cast<uint2*>(o + plane)[b * mr4 + i] = *reinterpret_cast<const uint2*>(m);
+      reinterpret_cast<uint2*>(o + 2 * plane)[b * mr4 + i] = *reinterpret_cast<const uint2*>(l);
+    } else if (MODE == 1) {
       __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
       __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
       uint2 pk;
@@ -208,18 +266,19 @@ __global__ void k_finalize_p(float* __restrict__ P, const float* __restrict__ P2
   }
 }
 
-cudaError_t launch_finalize_p(const float* P, const float* P2, void* Pg, bool use_bf16,
-                              const int32_t* flags, int count, int64_t m, int64_t r,
-                              float* P_out, cudaStream_t s) {
-  (void)P;
+cudaError_t launch_finalize_p(const float* P2, void* Pg, int mode, const int32_t* flags,
+                              int count, int64_t m, int64_t r, float* P, cudaStream_t s) {
   const int64_t mr4 = m * r / 4;
   int64_t gx = (mr4 + 255) / 256;
   if (gx > 64) gx = 64;
   dim3 grid((unsigned)gx, (unsigned)count);
-  if (use_bf16)
-    k_finalize_p<true><<<grid, 256, 0, s>>>(P_out, P2, Pg, flags, mr4);
+  const int64_t plane = (int64_t)count * m * r;
+  if (mode == 2)
+    k_finalize_p<2><<<grid, 256, 0, s>>>(P, P2, Pg, flags, mr4, plane);
+  else if (mode == 1)
+    k_finalize_p<1><<<grid, 256, 0, s>>>(P, P2, Pg, flags, mr4, plane);
   else
-    k_finalize_p<false><<<grid, 256, 0, s>>>(P_out, P2, Pg, flags, mr4);
+    k_finalize_p<0><<<grid, 256, 0, s>>>(P, P2, Pg, flags, mr4, plane);
   return cudaGetLastError();
 }
 
@@ -269,7 +328,8 @@ __global__ void __launch_bounds__(256) k_colnorm_partial(const float* __restrict
   }
 }
 
-template <bool BF16>
+// MODE 0: Q only; 1: + bf16 R and Q; 2: + three-way bf16 splits of R and Q
+template <int MODE>
 __global__ void __launch_bounds__(256) k_colnorm_apply(const float* __restrict__ R,
                                                         float* __restrict__ Q,
                                                         void* __restrict__ Rg,
@@ -306,7 +366,24 @@ __global__ void __launch_bounds__(256) k_colnorm_apply(const float* __restrict__
     qv.z = n2 > 0.f ? rv.z / n2 : 0.f;
     qv.w = n3 > 0.f ? rv.w / n3 : 0.f;
     Q4[e] = qv;
-    if (BF16) {
+    if (MODE == 2) {
+      const int64_t plane = (int64_t)gridDim.y * n * vc;  // in float4 units
+      const float rr[4] = {rv.x, rv.y, rv.z, rv.w}, qq[4] = {qv.x, qv.y, qv.z, qv.w};
+      __align__(8) bf16 rh[4], rm[4], rl[4], qh[4], qm[4], ql[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        split3_bf16(rr[q], rh[q], rm[q], rl[q]);
+        split3_bf16(qq[q], qh[q], qm[q], ql[q]);
+      }
+      uint2* R2 = reinterpret_cast<uint2*>(Rg);
+      uint2* Q2 = reinterpret_cast<uint2*>(Qg);
+      R2[e] = *reinterpret_cast<const uint2*>(rh);
+      R2[e + plane] = *reinterpret_cast<const uint2*>(rm);
+      R2[e + 2 * plane] = *reinterpret_cast<const uint2*>(rl);
+      Q2[e] = *reinterpret_cast<const uint2*>(qh);
+      Q2[e + plane] = *reinterpret_cast<const uint2*>(qm);
+      Q2[e + 2 * plane] = *reinterpret_cast<const uint2*>(ql);
+    } else if (MODE == 1) {
       __nv_bfloat162 r01 = __floats2bfloat162_rn(rv.x, rv.y), r23 = __floats2bfloat162_rn(rv.z, rv.w);
       __nv_bfloat162 q01 = __floats2bfloat162_rn(qv.x, qv.y), q23 = __floats2bfloat162_rn(qv.z, qv.w);
       uint2 rp, qp;
@@ -327,7 +404,7 @@ int colnorm_splits(int count, int64_t n) {
   return (int)ns;
 }
 
-cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, bool use_bf16, float* part,
+cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, int mode, float* part,
                            int nsplit, int32_t* flags, int count, int64_t n, int64_t r,
                            cudaStream_t s) {
   const int64_t vc = r / 4;
@@ -343,19 +420,17 @@ cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, bool us
   const int64_t gx = (n + rows - 1) / rows;
   const size_t smem = (size_t)r * sizeof(float);
   if (smem > 48 * 1024) {
-    if (use_bf16)
-      cudaFuncSetAttribute(k_colnorm_apply<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
-    else
-      cudaFuncSetAttribute(k_colnorm_apply<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
+    cudaFuncSetAttribute(k_colnorm_apply<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(k_colnorm_apply<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(k_colnorm_apply<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   }
-  if (use_bf16)
-    k_colnorm_apply<true><<<dim3((unsigned)gx, (unsigned)count), 256, smem, s>>>(
-        R, Q, Rg, Qg, part, flags, n, r, nsplit, rows);
+  const dim3 grid((unsigned)gx, (unsigned)count);
+  if (mode == 2)
+    k_colnorm_apply<2><<<grid, 256, smem, s>>>(R, Q, Rg, Qg, part, flags, n, r, nsplit, rows);
+  else if (mode == 1)
+    k_colnorm_apply<1><<<grid, 256, smem, s>>>(R, Q, Rg, Qg, part, flags, n, r, nsplit, rows);
   else
-    k_colnorm_apply<false><<<dim3((unsigned)gx, (unsigned)count), 256, smem, s>>>(
-        R, Q, Rg, Qg, part, flags, n, r, nsplit, rows);
+    k_colnorm_apply<0><<<grid, 256, smem, s>>>(R, Q, Rg, Qg, part, flags, n, r, nsplit, rows);
   return cudaGetLastError();
 }
 

@@ -190,35 +190,46 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
     float* Lkk = blk_at(blk, k, k);
     float* Dk = dinv + k * CBLK;
     if (warp == 0) {
-      // Cholesky of the diagonal block, lane = row
+      // Cholesky of the diagonal block in registers: lane u holds row u; entries of
+      // other rows come by warp shuffle (fully unrolled, so the row stays in registers)
       const int u = lane;
+      float row[CB];
+#pragma unroll
+      for (int c = 0; c < CB; ++c) row[c] = Lkk[u * CBS + c];
       bool fail = false;
+#pragma unroll
       for (int j = 0; j < CB; ++j) {
-        const float d = Lkk[j * CBS + j];
-        if (!(d > 0.f) || !isfinite(d)) { fail = true; break; }
-        const float ljj = sqrtf(d);
+        const float d = __shfl_sync(0xffffffffu, row[j], j);
+        fail |= !(d > 0.f) || !isfinite(d);
+        const float ljj = sqrtf(fmaxf(d, 1e-30f));
         if (k * CB + j < r) { dmin = fminf(dmin, ljj); dmax = fmaxf(dmax, ljj); }
-        __syncwarp();
-        if (u > j) Lkk[u * CBS + j] /= ljj;
-        __syncwarp();
-        if (u == j) Lkk[j * CBS + j] = ljj;
-        if (u > j) {
-          const float luj = Lkk[u * CBS + j];
-          for (int c = j + 1; c <= u; ++c) Lkk[u * CBS + c] -= luj * Lkk[c * CBS + j];
+        if (u == j) row[j] = ljj;
+        if (u > j) row[j] = row[j] / ljj;
+#pragma unroll
+        for (int c = j + 1; c < CB; ++c) {
+          const float lcj = __shfl_sync(0xffffffffu, row[j], c);  // L[c][j]
+          if (u >= c) row[c] = fmaf(-row[j], lcj, row[c]);
         }
-        __syncwarp();
       }
+#pragma unroll
+      for (int c = 0; c < CB; ++c) Lkk[u * CBS + c] = (c <= u) ? row[c] : 0.f;
       if (fail) {
         if (lane == 0) s_fail = 1;
       } else {
-        // D_k = L_kk^-1 by forward substitution, lane = column
+        // D_k = L_kk^-1, lane v computes column v by forward substitution; row i of L
+        // is broadcast from lane i
         const int v = lane;
+        float x[CB];
+#pragma unroll
         for (int i = 0; i < CB; ++i) {
-          if (i < v) { Dk[i * CBS + v] = 0.f; continue; }
           float sacc = (i == v) ? 1.f : 0.f;
-          for (int t = v; t < i; ++t) sacc -= Lkk[i * CBS + t] * Dk[t * CBS + v];
-          Dk[i * CBS + v] = sacc / Lkk[i * CBS + i];
+#pragma unroll
+          for (int t = 0; t < i; ++t) sacc = fmaf(-__shfl_sync(0xffffffffu, row[t], i), x[t], sacc);
+          const float lii = __shfl_sync(0xffffffffu, row[i], i);
+          x[i] = (i < v) ? 0.f : sacc / lii;
         }
+#pragma unroll
+        for (int i = 0; i < CB; ++i) Dk[i * CBS + v] = x[i];
       }
     }
     __syncthreads();

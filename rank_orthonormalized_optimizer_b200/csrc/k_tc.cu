@@ -104,10 +104,11 @@ static int sm_count() {
 }
 
 // ------------------------------------------------------------------ device: timeouts
-// Mark DION_MAT_TIMEOUT on every matrix owning a tile from `t` on (this CTA's share).
-__device__ void mark_unfinished(int32_t* flags, int t, int ntiles, int tiles_per_mat) {
+// Mark DION_MAT_TIMEOUT on every matrix owning a tile t, t + stride, ... < t_end
+// (the tiles of this CTA it did not finish).
+__device__ void mark_unfinished(int32_t* flags, int t, int t_end, int tiles_per_mat, int stride) {
   int last = -1;
-  for (; t < ntiles; t += gridDim.x) {
+  for (; t < t_end; t += stride) {
     const int b = t / tiles_per_mat;
     if (b != last) {
       atomicOr(flags + b, F_TIMEOUT);
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (lane == 0) mbar_arrive(tempty + acc);
       ++lt;
     }
-    if (t < ntiles && lane == 0) mark_unfinished(p.flags, t, ntiles, tiles_per_mat);
+    if (t < ntiles && lane == 0) mark_unfinished(p.flags, t, ntiles, tiles_per_mat, gridDim.x);
   }
   __syncthreads();
   if (warp == 2) {
@@ -435,6 +436,60 @@ cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, int count, int
   return e;
 }
 
+// fp32 contractions on bf16 tensor cores: operands as three bf16 parts.
+cudaError_t tc_gemm_bq_split(const bf16* Bs, const bf16* Qs, bf16* P0s, int count, int64_t m,
+                             int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
+                             cudaStream_t s, int* nlaunch, bool* done) {
+  using namespace tc;
+  *nlaunch = 0;
+  *done = false;
+  const int bn = r <= 128 ? (int)r : 128;   // three parts of A and B per stage
+  CUtensorMap ma, mb;
+  if (!map3d(&ma, Bs, true, n, m, 3 * (uint64_t)count, BK, BM)) return cudaSuccess;
+  if (!map3d(&mb, Qs, true, n, r, 3 * (uint64_t)count, BK, bn)) return cudaSuccess;
+  GemmP p{};
+  p.M = m; p.N = r; p.K = n;
+  p.batch = count;
+  p.block_n = bn;
+  p.tiles_m = (int)((m + BM - 1) / BM);
+  p.tiles_n = (int)((r + bn - 1) / bn);
+  p.num_kb = (int)((n + BK - 1) / BK);
+  p.idesc = idesc_bf16(BM, bn, false, false);
+  p.C = nullptr; p.ldc = r; p.c_bs = m * r;
+  p.Cs = P0s; p.cs_stride = (int64_t)count * m * r;
+  p.flags = flags;
+  p.max_spins = max_spins;
+  cudaError_t e = launch_gemm<false, false, 3>(ma, mb, p, s);
+  if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
+  return e;
+}
+
+cudaError_t tc_gemm_btp_split(const bf16* Bs, const bf16* Ps, float* R, int count, int64_t m,
+                              int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
+                              cudaStream_t s, int* nlaunch, bool* done) {
+  using namespace tc;
+  *nlaunch = 0;
+  *done = false;
+  const int bn = r <= 64 ? 64 : 128;        // MN-major B: whole 64-wide atoms
+  CUtensorMap ma, mb;
+  if (!map3d(&ma, Bs, true, n, m, 3 * (uint64_t)count, 64, BK)) return cudaSuccess;
+  if (!map3d(&mb, Ps, true, r, m, 3 * (uint64_t)count, 64, BK)) return cudaSuccess;
+  GemmP p{};
+  p.M = n; p.N = r; p.K = m;
+  p.batch = count;
+  p.block_n = bn;
+  p.tiles_m = (int)((n + BM - 1) / BM);
+  p.tiles_n = (int)((r + bn - 1) / bn);
+  p.num_kb = (int)((m + BK - 1) / BK);
+  p.idesc = idesc_bf16(BM, bn, true, true);
+  p.C = R; p.ldc = r; p.c_bs = n * r;
+  p.flags = flags;
+  p.max_spins = max_spins;
+  cudaError_t e = launch_gemm<true, true, 3>(ma, mb, p, s);
+  if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
+  return e;
+}
+
 cudaError_t tc_gram(const bf16* Xs, float* W, int count, int64_t m, int64_t r, int32_t* flags,
                     int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s, int* nlaunch,
                     bool* done) {
@@ -492,14 +547,312 @@ cudaError_t tc_apply(const bf16* Xs, const bf16* Ls, float* Y, bf16* Ys, int cou
 
 namespace tc {
 
+// ------------------------------------------------------------------ fused B = M + G, P0 = B Q
+// Steps 1 and 2 in one pass over M and G: TMA stages fp32 tiles of M and G, four
+// converter warps (a row each) add them, round to bf16 and write the K-major,
+// 128-byte-swizzled A operand of the MMA; the same shared-memory bytes are stored by
+// TMA as bf16 B for the later B^T P.  B is read from HBM once (8 bytes per element)
+// and written once (2 bytes); nothing re-reads it for B Q.
+//   warp 0       TMA: M, G (fp32, 2 boxes of 32 columns each) and the Q^T tile
+//   warp 1       MMA issuer
+//   warp 2       TMEM allocator
+//   warps 4..7   epilogue: P0's three-way bf16 split
+//   warps 8..11  converters
+constexpr int FB_STAGES = 2;
+constexpr int FB_NT = 384;
+constexpr uint32_t FB_F32_BYTES = 2 * 2 * BM * 32 * 4;  // M and G, two 32-column boxes: 64 KB
+constexpr uint32_t FB_A_BYTES = BM * BK * 2;             // 16 KB
+
+struct FusedP {
+  int64_t m, n, r;
+  int batch, tiles_m, tiles_n, num_kb, block_n;
+  uint32_t idesc, b_bytes, tmem_cols;
+  bf16* P0s;
+  int64_t cs_stride;
+  int32_t* flags;
+  int64_t max_spins;
+};
+
+__global__ void __launch_bounds__(FB_NT, 1)
+    k_tc_formb_bq(const __grid_constant__ CUtensorMap tmM, const __grid_constant__ CUtensorMap tmG,
+                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmBs,
+                  const FusedP p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sF = smem;                                  // [stage][M box0 | M box1 | G box0 | G box1]
+  uint8_t* sA = sF + FB_STAGES * FB_F32_BYTES;         // [stage] bf16 A tile
+  uint8_t* sB = sA + FB_STAGES * FB_A_BYTES;           // [stage] Q^T tile
+  uint64_t* f_full = reinterpret_cast<uint64_t*>(sB + FB_STAGES * p.b_bytes);
+  uint64_t* f_empty = f_full + FB_STAGES;
+  uint64_t* b_full = f_empty + FB_STAGES;
+  uint64_t* b_empty = b_full + FB_STAGES;
+  uint64_t* a_full = b_empty + FB_STAGES;
+  uint64_t* a_empty = a_full + FB_STAGES;
+  uint64_t* tfull = a_empty + FB_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_per_mat = p.tiles_m * p.tiles_n;
+  const int ntiles = p.batch * tiles_per_mat;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < FB_STAGES; ++s) {
+      mbar_init(f_full + s, 1);
+      mbar_init(f_empty + s, 4);
+      mbar_init(b_full + s, 1);
+      mbar_init(b_empty + s, 1);
+      mbar_init(a_full + s, 4);
+      mbar_init(a_empty + s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull + a, 1);
+      mbar_init(tempty + a, 4);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    prefetch_map(&tmM);
+    prefetch_map(&tmG);
+    prefetch_map(&tmQ);
+    int stage = 0, used = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const int b = t / tiles_per_mat;
+      const int rem = t % tiles_per_mat;
+      const int m0 = (rem / p.tiles_n) * BM;
+      const int n0 = (rem % p.tiles_n) * p.block_n;
+      bool ok = true;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!wait_bounded(f_empty + stage, phase ^ 1, p.max_spins, abort) ||
+            !wait_bounded(b_empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
+        const int k0 = kb * BK;
+        uint8_t* f = sF + stage * FB_F32_BYTES;
+        mbar_expect_tx(f_full + stage, FB_F32_BYTES);
+        tma_load_3d(f, &tmM, f_full + stage, k0, m0, b);
+        tma_load_3d(f + 16384, &tmM, f_full + stage, k0 + 32, m0, b);
+        tma_load_3d(f + 32768, &tmG, f_full + stage, k0, m0, b);
+        tma_load_3d(f + 49152, &tmG, f_full + stage, k0 + 32, m0, b);
+        mbar_expect_tx(b_full + stage, p.b_bytes);
+        tma_load_3d(sB + stage * p.b_bytes, &tmQ, b_full + stage, k0, n0, b);
+        if (used < FB_STAGES) ++used;
+        if (++stage == FB_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+    if (*abort)
+      for (int i = 0; i < used; ++i) {
+        stage = (stage + FB_STAGES - 1) % FB_STAGES;
+        if (stage == FB_STAGES - 1) phase ^= 1;
+        wait_drain(f_full + stage, phase);
+        wait_drain(b_full + stage, phase);
+      }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    int stage = 0, lt = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      if (!wait_bounded(tempty + acc, ((lt >> 1) & 1) ^ 1, p.max_spins, abort)) break;
+      tc_fence_after();
+      const uint32_t d = tmem + acc * p.block_n;
+      bool ok = true;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!wait_bounded(b_full + stage, phase, p.max_spins, abort) ||
+            !wait_bounded(a_full + stage, phase, p.max_spins, abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + stage * FB_A_BYTES);
+        const uint32_t b_base = smem_u32(sB + stage * p.b_bytes);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          mma_bf16(d, sw128_desc(a_base + k * 32, 16, 1024), sw128_desc(b_base + k * 32, 16, 1024),
+                   p.idesc, (kb | k) != 0);
+        mma_commit(b_empty + stage);
+        mma_commit(a_empty + stage);
+        if (++stage == FB_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      mma_commit(tfull + acc);
+    }
+    mma_commit(drain);
+    wait_drain(drain, 0);
+  } else if (warp >= 8) {
+    // ---------------- converters: row = lane of this warp's 32-row quarter
+    const int cw = warp - 8;
+    const int row = cw * 32 + lane;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const int b = t / tiles_per_mat;
+      const int rem = t % tiles_per_mat;
+      const int m0 = (rem / p.tiles_n) * BM;
+      bool ok = true;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!wait_bounded(f_full + stage, phase, p.max_spins, abort) ||
+            !wait_bounded(a_empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
+        // the store issued from this A stage two k-blocks ago must have read it
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        __syncwarp();
+        const uint8_t* f = sF + stage * FB_F32_BYTES + row * 128;
+        uint8_t* a = sA + stage * FB_A_BYTES + row * 128;
+        const int sw = row & 7;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {  // 8 output chunks of 8 bf16 = columns 8c .. 8c+7
+          const int box = c >> 2;        // columns 0..31 in box 0, 32..63 in box 1
+          const int c0 = (2 * c) & 7, c1 = (2 * c + 1) & 7;  // fp32 chunks inside the box
+          const uint8_t* fm = f + box * 16384;
+          const uint8_t* fg = f + 32768 + box * 16384;
+          const float4 m0v = *reinterpret_cast<const float4*>(fm + ((c0 ^ sw) << 4));
+          const float4 m1v = *reinterpret_cast<const float4*>(fm + ((c1 ^ sw) << 4));
+          const float4 g0v = *reinterpret_cast<const float4*>(fg + ((c0 ^ sw) << 4));
+          const float4 g1v = *reinterpret_cast<const float4*>(fg + ((c1 ^ sw) << 4));
+          __nv_bfloat162 q0 = __floats2bfloat162_rn(m0v.x + g0v.x, m0v.y + g0v.y);
+          __nv_bfloat162 q1 = __floats2bfloat162_rn(m0v.z + g0v.z, m0v.w + g0v.w);
+          __nv_bfloat162 q2 = __floats2bfloat162_rn(m1v.x + g1v.x, m1v.y + g1v.y);
+          __nv_bfloat162 q3 = __floats2bfloat162_rn(m1v.z + g1v.z, m1v.w + g1v.w);
+          uint4 pk;
+          pk.x = *reinterpret_cast<uint32_t*>(&q0);
+          pk.y = *reinterpret_cast<uint32_t*>(&q1);
+          pk.z = *reinterpret_cast<uint32_t*>(&q2);
+          pk.w = *reinterpret_cast<uint32_t*>(&q3);
+          *reinterpret_cast<uint4*>(a + ((c ^ sw) << 4)) = pk;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(f_empty + stage);  // fp32 staging free again
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(a_full + stage);
+          tma_store_3d(&tmBs, sA + stage * FB_A_BYTES + cw * 32 * 128, kb * BK, m0 + cw * 32, b);
+          bulk_commit();
+        }
+        __syncwarp();
+        if (++stage == FB_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+    if (lane == 0) bulk_wait0();
+  } else if (warp >= 4) {
+    // ---------------- epilogue: P0's three-way bf16 split
+    const int ew = warp - 4;
+    int lt = 0;
+    int t = blockIdx.x;
+    for (; t < ntiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      if (!wait_bounded(tfull + acc, (lt >> 1) & 1, p.max_spins, abort)) break;
+      tc_fence_after();
+      const int b = t / tiles_per_mat;
+      const int rem = t % tiles_per_mat;
+      const int64_t row = (int64_t)(rem / p.tiles_n) * BM + ew * 32 + lane;
+      const int64_t n0 = (int64_t)(rem % p.tiles_n) * p.block_n;
+      const int64_t off = (int64_t)b * p.m * p.r + row * p.r;
+      const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * p.block_n;
+      for (int c = 0; c < p.block_n; c += 16) {
+        float v[16];
+        tmem_ld16(tbase + c, v);
+        tmem_wait_ld();
+        if (row < p.m && n0 + c < p.r) {
+          __align__(16) bf16 h[16], mi[16], lo[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) split3_bf16(v[q], h[q], mi[q], lo[q]);
+          bf16* base = p.P0s + off + n0 + c;
+          const uint4* sh = reinterpret_cast<const uint4*>(h);
+          const uint4* sm = reinterpret_cast<const uint4*>(mi);
+          const uint4* sl = reinterpret_cast<const uint4*>(lo);
+          reinterpret_cast<uint4*>(base)[0] = sh[0];
+          reinterpret_cast<uint4*>(base)[1] = sh[1];
+          reinterpret_cast<uint4*>(base + p.cs_stride)[0] = sm[0];
+          reinterpret_cast<uint4*>(base + p.cs_stride)[1] = sm[1];
+          reinterpret_cast<uint4*>(base + 2 * p.cs_stride)[0] = sl[0];
+          reinterpret_cast<uint4*>(base + 2 * p.cs_stride)[1] = sl[1];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty + acc);
+    }
+    if (t < ntiles && lane == 0) mark_unfinished(p.flags, t, ntiles, tiles_per_mat, gridDim.x);
+  }
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+}  // namespace tc
+
+cudaError_t tc_formb_bq(const float* M, const float* G, const void* Qg, void* Bg, bf16* P0s,
+                        int count, int64_t m, int64_t n, int64_t r, int64_t max_spins,
+                        int32_t* flags, cudaStream_t s, int* nlaunch, bool* done) {
+  using namespace tc;
+  *nlaunch = 0;
+  *done = false;
+  const int bn = pick_block_n(r, 16);
+  CUtensorMap mM, mG, mQ, mBs;
+  if (!map3d(&mM, M, false, n, m, count, 32, BM)) return cudaSuccess;
+  if (!map3d(&mG, G, false, n, m, count, 32, BM)) return cudaSuccess;
+  if (!map3d(&mQ, Qg, true, n, r, count, BK, bn)) return cudaSuccess;
+  if (!map3d(&mBs, Bg, true, n, m, count, BK, 32)) return cudaSuccess;
+  FusedP p{};
+  p.m = m; p.n = n; p.r = r;
+  p.batch = count;
+  p.block_n = bn;
+  p.tiles_m = (int)((m + BM - 1) / BM);
+  p.tiles_n = (int)((r + bn - 1) / bn);
+  p.num_kb = (int)((n + BK - 1) / BK);
+  p.idesc = idesc_bf16(BM, bn, false, false);
+  p.b_bytes = (uint32_t)bn * BK * 2;
+  p.tmem_cols = pow2_cols(2 * bn);
+  p.P0s = P0s;
+  p.cs_stride = (int64_t)count * m * r;
+  p.flags = flags;
+  p.max_spins = max_spins;
+  const size_t smem = 1024 + FB_STAGES * (FB_F32_BYTES + FB_A_BYTES + p.b_bytes) +
+                      (6 * FB_STAGES + 5) * 8 + 16;
+  cudaError_t e = cudaFuncSetAttribute(k_tc_formb_bq, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const int ntiles = count * p.tiles_m * p.tiles_n;
+  const int grid = ntiles < sm_count() ? ntiles : sm_count();
+  k_tc_formb_bq<<<grid, FB_NT, smem, s>>>(mM, mG, mQ, mBs, p);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
+  return e;
+}
+
+namespace tc {
+
 // ------------------------------------------------------------------ fused update
 struct UpdP {
   int64_t m, n;
   int batch, tiles_m, tiles_n, num_kb;
   float omm, lrs;  // 1 - mu, lr * s
   int32_t* flags;
+  int* tile_counter;  // zero before the launch; tiles are taken from it in order
+  int npairs;         // 1: bf16 operands; 3: split operands, products (1,0) (0,1) (0,0)
+  int pa[3], pb[3];   // part of P and of R, Q in each product
   int64_t max_spins;
 };
+
+// Tiles are handed out in order from a global counter rather than dealt round-robin:
+// CTAs then always work on neighbouring tiles (the same rows of M, G, X, so the same
+// DRAM pages) however their speeds drift over a long launch.
+constexpr int TILE_RING = 4;
 
 constexpr uint32_t UPD_A_BYTES = BM * BK * 2;           // 16 KB
 constexpr uint32_t UPD_B_BYTES = 2 * UPD_BN * BK * 2;   // 32 KB (R rows then Q rows)
@@ -507,7 +860,7 @@ constexpr uint32_t SLAB_BYTES = BM * SLAB * 4;          // 16 KB per tensor
 // + one 128 x 32 staging slab each for M' and X', so a load slab is released as soon
 // as it has been read, without waiting for the TMA store of the results
 constexpr size_t UPD_SMEM = 1024 + UPD_STAGES * (UPD_A_BYTES + UPD_B_BYTES) +
-                            SLAB_STAGES * 3 * SLAB_BYTES + 2 * SLAB_BYTES + 256;
+                            SLAB_STAGES * 3 * SLAB_BYTES + 2 * SLAB_BYTES + 384;
 
 __global__ void __launch_bounds__(NT, 1)
     k_tc_update(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmR,
@@ -528,13 +881,19 @@ __global__ void __launch_bounds__(NT, 1)
   uint64_t* tfull = sempty + SLAB_STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ring_full = drain + 1;
+  uint64_t* ring_empty = ring_full + TILE_RING;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring_empty + TILE_RING);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);  // TILE_RING tile ids
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_per_mat = p.tiles_m * p.tiles_n;
   const int ntiles = p.batch * tiles_per_mat;
   constexpr int NSLAB = UPD_BN / SLAB;
+  // consumers of the tile ring: slab producer, MMA issuer, four epilogue warps
+  constexpr int RING_CONSUMERS = 6;
+
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < UPD_STAGES; ++s) {
@@ -550,6 +909,10 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_init(tempty + a, 4);
     }
     mbar_init(drain, 1);
+    for (int s = 0; s < TILE_RING; ++s) {
+      mbar_init(ring_full + s, 1);
+      mbar_init(ring_empty + s, RING_CONSUMERS);
+    }
     *abort = 0;
     fence_mbar_init();
   }
@@ -563,26 +926,35 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // ---------------- operand producer: P tile and the R, Q rows of the tile
+    // ---------------- scheduler + operand producer: P tile and the R, Q rows of the tile
     prefetch_map(&tmP);
     prefetch_map(&tmR);
     prefetch_map(&tmQ);
-    int stage = 0, used = 0;
-    uint32_t phase = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    int stage = 0, used = 0, slot = 0;
+    uint32_t phase = 0, rphase = 0;
+    while (true) {
+      if (!wait_bounded(ring_empty + slot, rphase ^ 1, p.max_spins, abort)) break;
+      int t = atomicAdd(p.tile_counter, 1);
+      if (t >= ntiles) t = -1;
+      ring[slot] = t;
+      mbar_arrive(ring_full + slot);  // publishes the tile id to the consumers
+      if (++slot == TILE_RING) { slot = 0; rphase ^= 1; }
+      if (t < 0) break;
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
       const int m0 = (rem / p.tiles_n) * BM;
       const int n0 = (rem % p.tiles_n) * UPD_BN;
       bool ok = true;
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+      for (int it = 0; it < p.num_kb * p.npairs; ++it) {
+        const int kb = it / p.npairs, pi = it % p.npairs;
+        const int za = p.pa[pi] * p.batch + b, zb = p.pb[pi] * p.batch + b;
         if (!wait_bounded(empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
         mbar_expect_tx(full + stage, UPD_A_BYTES + UPD_B_BYTES);
         uint8_t* a_dst = sA + stage * UPD_A_BYTES;
         uint8_t* b_dst = sB + stage * UPD_B_BYTES;
-        tma_load_3d(a_dst, &tmP, full + stage, kb * BK, m0, b);
-        tma_load_3d(b_dst, &tmR, full + stage, kb * BK, n0, b);
-        tma_load_3d(b_dst + UPD_BN * BK * 2, &tmQ, full + stage, kb * BK, n0, b);
+        tma_load_3d(a_dst, &tmP, full + stage, kb * BK, m0, za);
+        tma_load_3d(b_dst, &tmR, full + stage, kb * BK, n0, zb);
+        tma_load_3d(b_dst + UPD_BN * BK * 2, &tmQ, full + stage, kb * BK, n0, zb);
         if (used < UPD_STAGES) ++used;
         if (++stage == UPD_STAGES) { stage = 0; phase ^= 1; }
       }
@@ -599,9 +971,14 @@ __global__ void __launch_bounds__(NT, 1)
     prefetch_map(&tmM);
     prefetch_map(&tmG);
     prefetch_map(&tmX);
-    int stage = 0, used = 0;
-    uint32_t phase = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    int stage = 0, used = 0, slot = 0;
+    uint32_t phase = 0, rphase = 0;
+    while (true) {
+      if (!wait_bounded(ring_full + slot, rphase, p.max_spins, abort)) break;
+      const int t = ring[slot];
+      mbar_arrive(ring_empty + slot);
+      if (++slot == TILE_RING) { slot = 0; rphase ^= 1; }
+      if (t < 0) break;
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
       const int m0 = (rem / p.tiles_n) * BM;
@@ -629,16 +1006,21 @@ __global__ void __launch_bounds__(NT, 1)
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer: acc = P [R | Q]^T, M = 128, N = 256
     constexpr uint32_t idesc = idesc_bf16(BM, 2 * UPD_BN, false, false);
-    int stage = 0;
-    uint32_t phase = 0;
+    int stage = 0, slot = 0;
+    uint32_t phase = 0, rphase = 0;
     int lt = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+    for (;; ++lt) {
+      if (!wait_bounded(ring_full + slot, rphase, p.max_spins, abort)) break;
+      const int t = ring[slot];
+      mbar_arrive(ring_empty + slot);
+      if (++slot == TILE_RING) { slot = 0; rphase ^= 1; }
+      if (t < 0) break;
       const int acc = lt & 1;
       if (!wait_bounded(tempty + acc, ((lt >> 1) & 1) ^ 1, p.max_spins, abort)) break;
       tc_fence_after();
       const uint32_t d = tmem + acc * 256;
       bool ok = true;
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+      for (int it = 0; it < p.num_kb * p.npairs; ++it) {
         if (!wait_bounded(full + stage, phase, p.max_spins, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_base = smem_u32(sA + stage * UPD_A_BYTES);
@@ -646,7 +1028,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)
           mma_bf16(d, sw128_desc(a_base + k * 32, 16, 1024), sw128_desc(b_base + k * 32, 16, 1024),
-                   idesc, (kb | k) != 0);
+                   idesc, (it | k) != 0);
         mma_commit(empty + stage);
         if (++stage == UPD_STAGES) { stage = 0; phase ^= 1; }
       }
@@ -659,14 +1041,19 @@ __global__ void __launch_bounds__(NT, 1)
     // ---------------- epilogue: one TMEM lane (tile row) per thread
     const int ew = warp - 4;
     const int row = ew * 32 + lane;  // row inside the tile
-    int stage = 0;
-    uint32_t phase = 0;
+    int stage = 0, slot = 0;
+    uint32_t phase = 0, rphase = 0;
     int lt = 0;
-    int t = blockIdx.x;
     bool ok = true;
-    for (; t < ntiles; t += gridDim.x, ++lt) {
+    for (;; ++lt) {
+      if (!wait_bounded(ring_full + slot, rphase, p.max_spins, abort)) { ok = false; break; }
+      const int t = ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ring_empty + slot);
+      if (++slot == TILE_RING) { slot = 0; rphase ^= 1; }
+      if (t < 0) break;
       const int acc = lt & 1;
-      if (!wait_bounded(tfull + acc, (lt >> 1) & 1, p.max_spins, abort)) break;
+      if (!wait_bounded(tfull + acc, (lt >> 1) & 1, p.max_spins, abort)) { ok = false; break; }
       tc_fence_after();
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
@@ -723,7 +1110,9 @@ __global__ void __launch_bounds__(NT, 1)
       if (lane == 0) mbar_arrive(tempty + acc);
     }
     if (lane == 0) bulk_wait0();
-    if (t < ntiles && lane == 0) mark_unfinished(p.flags, t, ntiles, tiles_per_mat);
+    // tiles are handed out dynamically, so after a give-up every matrix is suspect
+    if ((!ok || *abort) && lane == 0)
+      for (int b = 0; b < p.batch; ++b) atomicOr(p.flags + b, F_TIMEOUT);
   }
   __syncthreads();
   if (warp == 3) {
@@ -734,15 +1123,17 @@ __global__ void __launch_bounds__(NT, 1)
 
 }  // namespace tc
 
-cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, const float* G, float* M,
-                      float* X, int count, int64_t m, int64_t n, int64_t r, float mu, float lr_scale,
-                      int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch, bool* done) {
+cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, bool split, const float* G,
+                      float* M, float* X, int count, int64_t m, int64_t n, int64_t r, float mu,
+                      float lr_scale, int64_t max_spins, int32_t* flags, int* tile_counter,
+                      cudaStream_t s, int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
   CUtensorMap mP, mR, mQ, mM, mG, mX, mMs, mXs;
-  bool ok = map3d(&mP, Pg, true, r, m, count, BK, BM) && map3d(&mR, Rg, true, r, n, count, BK, UPD_BN) &&
-            map3d(&mQ, Qg, true, r, n, count, BK, UPD_BN) &&
+  const uint64_t zc = (split ? 3 : 1) * (uint64_t)count;
+  bool ok = map3d(&mP, Pg, true, r, m, zc, BK, BM) && map3d(&mR, Rg, true, r, n, zc, BK, UPD_BN) &&
+            map3d(&mQ, Qg, true, r, n, zc, BK, UPD_BN) &&
             map3d(&mM, M, false, n, m, count, SLAB, BM) && map3d(&mG, G, false, n, m, count, SLAB, BM) &&
             map3d(&mX, X, false, n, m, count, SLAB, BM) &&
             map3d(&mMs, M, false, n, m, count, SLAB, 32) && map3d(&mXs, X, false, n, m, count, SLAB, 32);
@@ -756,6 +1147,12 @@ cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, const floa
   p.omm = 1.f - mu;
   p.lrs = lr_scale;
   p.flags = flags;
+  p.tile_counter = tile_counter;
+  // split parts hi and mid carry about 17 bits: three products reach ~2^-17 relative
+  p.npairs = split ? 3 : 1;
+  p.pa[0] = split ? 1 : 0; p.pb[0] = 0;
+  p.pa[1] = 0; p.pb[1] = split ? 1 : 0;
+  p.pa[2] = 0; p.pb[2] = 0;
   p.max_spins = max_spins;
   cudaError_t e = cudaFuncSetAttribute(k_tc_update, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)UPD_SMEM);

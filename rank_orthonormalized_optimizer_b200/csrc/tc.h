@@ -18,15 +18,31 @@ const char* tc_map_error();
 cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, __nv_bfloat16* P0s, int count,
                        int64_t m, int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
                        cudaStream_t s, int* nlaunch, bool* done);
+// Steps 1 and 2 fused: Bg[b] = bf16(M[b] + G[b]) (written for B^T P) and the
+// three-way bf16 split of P0[b] = Bg[b] Qg[b]^T into P0s ([3][count][m][r]).
+cudaError_t tc_formb_bq(const float* M, const float* G, const void* Qg, void* Bg,
+                        __nv_bfloat16* P0s, int count, int64_t m, int64_t n, int64_t r,
+                        int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
+                        bool* done);
 // R[b] (n x r, fp32) = Bg[b]^T (n x m) * Pg[b] (m x r, bf16).
 cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, int count, int64_t m,
                         int64_t n, int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s,
                         int* nlaunch, bool* done);
 // M <- (M + G) - (1 - mu) Pg Rg^T and X <- X - lr_scale Pg Qg^T (Pg: m x r, Rg, Qg: n x r, bf16).
-cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, const float* G, float* M,
-                      float* X, int count, int64_t m, int64_t n, int64_t r, float mu,
-                      float lr_scale, int64_t max_spins, int32_t* flags, cudaStream_t s,
-                      int* nlaunch, bool* done);
+// tile_counter: one int in device memory, zero before the call (tiles are taken from it).
+// split: Pg, Rg, Qg are three-way bf16 splits ([3][count][...]) of fp32 operands.
+cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, bool split, const float* G,
+                      float* M, float* X, int count, int64_t m, int64_t n, int64_t r, float mu,
+                      float lr_scale, int64_t max_spins, int32_t* flags, int* tile_counter,
+                      cudaStream_t s, int* nlaunch, bool* done);
+// fp32 contractions from three-way bf16 splits: P0s = split(Bs Qs^T), R = Bs^T Ps.
+cudaError_t tc_gemm_bq_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Qs,
+                             __nv_bfloat16* P0s, int count, int64_t m, int64_t n, int64_t r,
+                             int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
+                             bool* done);
+cudaError_t tc_gemm_btp_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Ps, float* R,
+                              int count, int64_t m, int64_t n, int64_t r, int64_t max_spins,
+                              int32_t* flags, cudaStream_t s, int* nlaunch, bool* done);
 
 // W[b] (r x r, fp32) = X[b]^T X[b] from the three-way split Xs ([3][count][m][r] bf16),
 // six split products; matrices failing (flags & need) == need && !(flags & skip) skipped.
