@@ -70,6 +70,11 @@ struct dion_ctx {
   size_t events_used;
   double prof_ms[DION_KCLASS_COUNT];
   int64_t prof_launches[DION_KCLASS_COUNT];
+  // streams on which the buckets' orthonormalisations run side by side
+  int side_device;
+  std::vector<cudaStream_t> side;
+  std::vector<cudaEvent_t> side_done;
+  cudaEvent_t fork_ev;
 };
 
 namespace {
@@ -95,11 +100,12 @@ dion_status check_options(const dion_options& o) {
 // Per-step record of kernel launches (host counter) and optional events.
 struct StepCtx {
   dion_handle h;
-  cudaStream_t s;
+  cudaStream_t s;      // the stream the current phase runs on
   int launches;
   int cur_cls;
   EventPair* open;
   int open_at;
+  std::vector<int> p0s_ready;  // per bucket: P0's split was written by B Q
 };
 
 void begin_cls(StepCtx& c, int cls) {
@@ -135,8 +141,12 @@ void end_cls(StepCtx& c) {
     if (e_ != cudaSuccess) return fail(DION_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
   } while (0)
 
-dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, float lr,
-                       char* ws, int32_t* d_status) {
+// Phases of one step; each runs over every bucket before the next starts.
+enum Phase { PH_INIT, PH_PREPQ, PH_FORMB, PH_BQ, PH_ORTH, PH_BTP, PH_COLNORM, PH_UPDATE,
+             PH_STATUS, PH_COUNT };
+
+dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_bucket_ptrs& bp,
+                       float lr, char* ws, int32_t* d_status) {
   const dion_options& o = c.h->opt;
   const bool bf = o.precision == DION_PREC_BF16;
   const bool tensor = o.kernel_path == DION_PATH_TENSOR;
@@ -160,28 +170,35 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
   __nv_bfloat16* P0s = reinterpret_cast<__nv_bfloat16*>(ws + p.off_P0s);
   __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ps);
   __nv_bfloat16* Linvs = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Linvs);
-  bool p0s_ready = false;
+  int& p0s_ready = c.p0s_ready[bi];
   const int64_t m = p.m, n = p.n, r = p.r;
   const int cnt = p.count;
   cudaStream_t s = c.s;
 
-  DION_LAUNCH(c, 1, dion::launch_init_flags(flags, stats, sched, cnt,
-                                            o.orth_mode == DION_ORTH_HOUSEHOLDER ? DION_MAT_FALLBACK : 0,
-                                            s));
+  if (phase == PH_INIT) {
+    p0s_ready = 0;
+    DION_LAUNCH(c, 1, dion::launch_init_flags(flags, stats, sched, cnt,
+                                              o.orth_mode == DION_ORTH_HOUSEHOLDER ? DION_MAT_FALLBACK : 0,
+                                              s));
+    return DION_OK;
+  }
 
   // steps 1 and 2 fused on the tensor path when one N tile covers r: B = M + G is
   // formed in shared memory, fed to the MMA and stored once as bf16
   const bool fused_bq = tensor && bf && r <= 256;
 
+  if (phase == PH_PREPQ) {
   begin_cls(c, DION_KCLASS_PREP_Q);
   if (split)
     DION_LAUNCH(c, 1, dion::launch_prep_q_split(bp.Q, Qg, cnt, n, r, s));
   else
     DION_LAUNCH(c, 1, dion::launch_prep_q(bp.Q, Qg, bf, cnt, n, r, s));
   end_cls(c);
+  return DION_OK;
+  }
 
   // step 1: B = M + G in the precision of the contractions
-  if (!fused_bq) {
+  if (phase == PH_FORMB && !fused_bq) {
     begin_cls(c, DION_KCLASS_FORM_B);
     if (split)
       DION_LAUNCH(c, 1, dion::launch_form_b_split(bp.M, bp.G, Bg, (int64_t)cnt * m * n, s));
@@ -191,6 +208,7 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
   }
 
   // step 2: P0 = B Q
+  if (phase == PH_BQ) {
   begin_cls(c, DION_KCLASS_GEMM_BQ);
   if (fused_bq) {
     int nl = 0;
@@ -232,8 +250,11 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
     }
   }
   end_cls(c);
+  return DION_OK;
+  }
 
   // step 3: P = orth(P0) -- Cholesky-QR, optional second pass, Householder fallback
+  if (phase == PH_ORTH) {
   begin_cls(c, DION_KCLASS_ORTH);
   {
     auto gram = [&](const float* src) {
@@ -314,8 +335,11 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
                                               P, s));
   }
   end_cls(c);
+  return DION_OK;
+  }
 
   // step 4: R = B^T P
+  if (phase == PH_BTP) {
   begin_cls(c, DION_KCLASS_GEMM_BTP);
   {
     bool done = false;
@@ -344,14 +368,20 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
     }
   }
   end_cls(c);
+  return DION_OK;
+  }
 
   // step 6: Q = colnorm(R), plus the GEMM copies of R and Q for the update
+  if (phase == PH_COLNORM) {
   begin_cls(c, DION_KCLASS_COLNORM);
   DION_LAUNCH(c, 2, dion::launch_colnorm(R, bp.Q, Rg, Qng, bf ? 1 : (split ? 2 : 0), part,
                                          p.nsplit, flags, cnt, n, r, s));
   end_cls(c);
+  return DION_OK;
+  }
 
   // steps 5 and 7: M <- B - (1 - mu) P R^T and X <- X - lr s P Q^T in one pass
+  if (phase == PH_UPDATE) {
   begin_cls(c, DION_KCLASS_UPDATE);
   {
     bool done = false;
@@ -370,9 +400,40 @@ dion_status run_bucket(StepCtx& c, const Plan& p, const dion_bucket_ptrs& bp, fl
                                            lrs, s));
   }
   end_cls(c);
-
-  if (d_status) DION_LAUNCH(c, 1, dion::launch_write_status(flags, d_status + p.mat0, cnt, s));
   return DION_OK;
+  }
+
+  if (phase == PH_STATUS && d_status)
+    DION_LAUNCH(c, 1, dion::launch_write_status(flags, d_status + p.mat0, cnt, s));
+  return DION_OK;
+}
+
+// Side streams for the orthonormalisation phase, made on first use on a device.
+bool ensure_side_streams(dion_handle h, size_t want) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (h->side_device != dev) {
+    for (auto st : h->side) cudaStreamDestroy(st);
+    for (auto ev : h->side_done) cudaEventDestroy(ev);
+    if (h->fork_ev) cudaEventDestroy(h->fork_ev);
+    h->side.clear();
+    h->side_done.clear();
+    h->fork_ev = nullptr;
+    if (cudaEventCreateWithFlags(&h->fork_ev, cudaEventDisableTiming) != cudaSuccess) return false;
+    h->side_device = dev;
+  }
+  while (h->side.size() < want) {
+    cudaStream_t st;
+    cudaEvent_t ev;
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) {
+      cudaStreamDestroy(st);
+      return false;
+    }
+    h->side.push_back(st);
+    h->side_done.push_back(ev);
+  }
+  return true;
 }
 
 dion_status check_device(dion_handle h) {
@@ -533,6 +594,8 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
   h->profiling = false;
   h->events_used = 0;
   for (int i = 0; i < DION_KCLASS_COUNT; ++i) { h->prof_ms[i] = 0; h->prof_launches[i] = 0; }
+  h->side_device = -1;
+  h->fork_ev = nullptr;
   *out = h;
   *workspace_bytes = off;
   return DION_OK;
@@ -544,13 +607,33 @@ dion_status dion_step_batched(dion_handle h, const dion_bucket_ptrs* ptrs, int32
   dion_status st = check_step_args(h, ptrs, nbuckets, d_workspace, workspace_bytes, d_status);
   if (st != DION_OK) return st;
   if (!std::isfinite(lr)) return fail(DION_ERR_INVALID_ARG, "lr is not finite");
-  StepCtx c{h, reinterpret_cast<cudaStream_t>(stream), 0, -1, nullptr, 0};
-  for (int32_t b = 0; b < nbuckets; ++b) {
-    st = run_bucket(c, h->plans[b], ptrs[b], lr, static_cast<char*>(d_workspace), d_status);
-    if (st != DION_OK) {
-      end_cls(c);
-      h->last_launches = c.launches;
-      return st;
+  cudaStream_t main = reinterpret_cast<cudaStream_t>(stream);
+  StepCtx c{h, main, 0, -1, nullptr, 0, std::vector<int>(nbuckets, 0)};
+  char* ws = static_cast<char*>(d_workspace);
+  // the buckets' orthonormalisations are chains of short, latency-bound kernels:
+  // run them side by side on their own streams, forked from and joined to `main`
+  const bool fork = nbuckets > 1 && ensure_side_streams(h, (size_t)nbuckets);
+  for (int phase = 0; phase < PH_COUNT; ++phase) {
+    const bool side = fork && phase == PH_ORTH;
+    if (side) {
+      cudaEventRecord(h->fork_ev, main);
+      for (int32_t b = 0; b < nbuckets; ++b) cudaStreamWaitEvent(h->side[b], h->fork_ev, 0);
+    }
+    for (int32_t b = 0; b < nbuckets; ++b) {
+      c.s = side ? h->side[b] : main;
+      st = run_bucket(c, b, phase, h->plans[b], ptrs[b], lr, ws, d_status);
+      if (st != DION_OK) {
+        end_cls(c);
+        h->last_launches = c.launches;
+        return st;
+      }
+    }
+    if (side) {
+      for (int32_t b = 0; b < nbuckets; ++b) {
+        cudaEventRecord(h->side_done[b], h->side[b]);
+        cudaStreamWaitEvent(main, h->side_done[b], 0);
+      }
+      c.s = main;
     }
   }
   h->last_launches = c.launches;
@@ -591,6 +674,9 @@ dion_status dion_free(dion_handle h) {
     cudaEventDestroy(ep.a);
     cudaEventDestroy(ep.b);
   }
+  for (auto st : h->side) cudaStreamDestroy(st);
+  for (auto ev : h->side_done) cudaEventDestroy(ev);
+  if (h->fork_ev) cudaEventDestroy(h->fork_ev);
   h->magic = 0;
   delete h;
   return DION_OK;
