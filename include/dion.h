@@ -61,7 +61,9 @@ typedef enum dion_status {
 /* Per-matrix status bits written to d_status[] by every step (OR-ed). */
 enum {
   DION_MAT_OK = 0,
-  DION_MAT_FALLBACK = 1,      /* Cholesky-QR rejected; Householder QR produced P        */
+  DION_MAT_FALLBACK = 1,      /* Cholesky-QR rejected; P came from the fallback (shifted
+                                 Cholesky-QR iteration for r > 256 on the tensor path,
+                                 else Householder QR): the same Q factor                 */
   DION_MAT_CHOLQR2 = 2,       /* a second Cholesky-QR pass was applied                   */
   DION_MAT_NONFINITE = 4,     /* a Gram matrix held Inf/NaN (inputs were not finite)     */
   DION_MAT_TIMEOUT = 8,       /* a bounded device wait ran out; this matrix's outputs
@@ -83,10 +85,15 @@ typedef enum dion_precision {
 /* How P = orth(B Q) is formed. */
 typedef enum dion_orth_mode {
   DION_ORTH_AUTO = 0,        /* Cholesky-QR; a second pass when max|P^T P - I| > orth_tol;
-                                Householder when a pivot fails or the Cholesky diagonal
-                                ratio exceeds fallback_cond                              */
-  DION_ORTH_CHOLQR = 1,      /* one Cholesky-QR pass (+ Householder fallback)            */
-  DION_ORTH_CHOLQR2 = 2,     /* always two passes (+ Householder fallback)               */
+                                the fallback when a pivot fails or the Cholesky diagonal
+                                ratio exceeds fallback_cond: for r > 256 on the tensor
+                                path, shifted Cholesky-QR iterated until
+                                max|P^T P - I| <= orth_tol (at most 16 iterations, run
+                                as a CUDA graph with a conditional node; not when the
+                                caller's stream is being captured), then Householder QR
+                                for whatever is left; otherwise Householder QR            */
+  DION_ORTH_CHOLQR = 1,      /* one Cholesky-QR pass (+ the fallback)                    */
+  DION_ORTH_CHOLQR2 = 2,     /* always two passes (+ the fallback)                       */
   DION_ORTH_HOUSEHOLDER = 3  /* Householder QR for every matrix                          */
 } dion_orth_mode;
 
@@ -155,7 +162,10 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets,
  *   d_status    device int32 array, one word per matrix (bucket by bucket,
  *               slot by slot), overwritten with DION_MAT_* bits; may be NULL
  * Within a bucket the matrices are independent.  X, M and Q are written only
- * by the last kernels of the step.
+ * by the last kernels of the step.  Work runs on `stream` and on streams owned by
+ * the handle, forked from and joined back to `stream` with events; the first
+ * step with a fallback-capable plan (r > 256 on the tensor path) for a given
+ * workspace builds a CUDA graph (host memory owned by the handle).
  */
 dion_status dion_step_batched(dion_handle h, const dion_bucket_ptrs* ptrs,
                               int32_t nbuckets, float lr, void* d_workspace,

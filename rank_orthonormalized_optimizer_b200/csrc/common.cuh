@@ -16,6 +16,17 @@ constexpr int32_t F_CHOLQR2 = DION_MAT_CHOLQR2;
 constexpr int32_t F_NONFINITE = DION_MAT_NONFINITE;
 constexpr int32_t F_TIMEOUT = DION_MAT_TIMEOUT;
 constexpr int32_t F_ZERO_COL = DION_MAT_ZERO_COLUMN;
+constexpr int32_t F_PUBLIC = 0xFFFF;  // bits reported to the caller
+// Internal bits of the shifted Cholesky-QR iteration that replaces Householder QR for
+// flagged matrices when r > 256 (never reported):
+constexpr int32_t F_SMORE = 1 << 16;    // this iterate is not orthonormal yet
+constexpr int32_t F_SDONE = 1 << 17;    // the iterate in P is the final P
+constexpr int32_t F_SFAIL = 1 << 18;    // a factorisation failed: Householder QR takes over
+constexpr int32_t F_SITER = 1 << 19;    // P holds an iterate (P0 R^-1, R upper triangular)
+constexpr int32_t F_SNOSHIFT = 1 << 20; // well conditioned now: no shift from here on
+// Per-matrix statistics of the factorisation, ST floats each: min and max of diag(L),
+// the largest diagonal entry of the Gram (shifted iteration), the shift last added.
+constexpr int ST = 4;
 
 typedef __nv_bfloat16 bf16;
 

@@ -17,6 +17,7 @@
 #include <vector>
 
 #include "../../include/dion.h"
+#include "common.cuh"
 #include "internal.h"
 #include "tc.h"
 
@@ -46,7 +47,7 @@ struct Plan {
   int64_t mat0;
   int nsplit;
   size_t off_Bg, off_Qg, off_P0, off_P, off_P2, off_Pg, off_W, off_Linv, off_dinv, off_R, off_Rg,
-      off_Qng, off_part, off_flags, off_stats, off_P0s, off_Ps, off_Linvs, off_sched;
+      off_Qng, off_part, off_flags, off_stats, off_P0s, off_Ps, off_Linvs, off_sched, off_Ws, off_Ts;
 };
 
 struct EventPair {
@@ -75,6 +76,17 @@ struct dion_ctx {
   std::vector<cudaStream_t> side;
   std::vector<cudaEvent_t> side_done;
   cudaEvent_t fork_ev;
+  // per bucket: the shifted Cholesky-QR loop of the fallback (r > 256 on the tensor
+  // path) as a CUDA graph with a conditional while node, built on first use for a
+  // workspace and device and launched every step
+  struct FbGraph {
+    const void* ws;
+    int device;
+    cudaGraphExec_t exec;
+  };
+  std::vector<FbGraph> fb;
+  cudaStream_t cap;  // stream the loop body is captured on
+  int cap_device;
 };
 
 namespace {
@@ -141,6 +153,143 @@ void end_cls(StepCtx& c) {
     if (e_ != cudaSuccess) return fail(DION_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
   } while (0)
 
+constexpr int kFbMaxRounds = 8;   // two iterations per round
+constexpr int kFbRoundsSlot = 8;  // int of the bucket's scheduler area counting rounds
+
+struct FbBufs {
+  float *W, *Linv, *stats, *P;
+  int32_t* flags;
+  int* rounds;
+  __nv_bfloat16 *P0s, *Ps, *Ws, *Ts, *Linvs;
+};
+
+// One step of the shifted Cholesky-QR iteration on `s`: A_{k+1} = A_k R^-1 from the
+// split src into P (fp32) and the split dst.
+dion_status fb_iteration(const Plan& p, const dion_options& o, const FbBufs& f,
+                         const __nv_bfloat16* src, __nv_bfloat16* dst, cudaStream_t s) {
+  const int32_t need = DION_MAT_FALLBACK;
+  const int32_t skip = dion::F_SDONE | dion::F_SFAIL | DION_MAT_NONFINITE;
+  int nl = 0;
+  bool done = false;
+  cudaError_t e = dion::tc_gram(src, f.W, f.Ws, p.count, p.m, p.r, f.flags, need, skip,
+                                o.max_wait_spins, s, &nl, &done);
+  if (e != cudaSuccess || !done)
+    return fail(DION_ERR_CUDA, "shifted iteration, Gram: %s",
+                e != cudaSuccess ? cudaGetErrorString(e) : dion::tc_map_error());
+  dion::CholArgs ca{};
+  ca.W = f.W; ca.Linv = f.Linv; ca.Linvs = f.Linvs; ca.flags = f.flags; ca.stats = f.stats;
+  ca.count = p.count; ca.r = p.r; ca.m = p.m; ca.pass = 3;
+  ca.fallback_cond = o.fallback_cond; ca.orth_tol = o.orth_tol;
+  const char* what = "";
+  e = dion::launch_chol_inv_rec(ca, f.Ws, f.Ts, o.max_wait_spins, s, &nl, &done, &what);
+  if (e != cudaSuccess || !done)
+    return fail(DION_ERR_CUDA, "shifted iteration, factorisation (%s): %s", what,
+                e != cudaSuccess ? cudaGetErrorString(e) : dion::tc_map_error());
+  e = dion::tc_apply(src, f.Linvs, f.P, dst, p.count, p.m, p.r, f.flags, need, skip,
+                     o.max_wait_spins, s, &nl, &done);
+  if (e != cudaSuccess || !done)
+    return fail(DION_ERR_CUDA, "shifted iteration, apply: %s",
+                e != cudaSuccess ? cudaGetErrorString(e) : dion::tc_map_error());
+  e = dion::launch_fb_mark(f.flags, p.count, s);
+  if (e != cudaSuccess) return fail(DION_ERR_CUDA, "shifted iteration: %s", cudaGetErrorString(e));
+  return DION_OK;
+}
+
+// Graph: [start: reset the loop state, condition = some matrix needs the loop]
+//        while (condition) { iteration P0s -> Ps; iteration Ps -> P0s; condition update }
+// With no flagged matrix only the start kernel runs.
+dion_status fb_build(dion_handle h, const Plan& p, const FbBufs& f, cudaGraphExec_t* out) {
+  const dion_options& o = h->opt;
+  cudaStream_t cs = h->cap;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  dion_status st = DION_OK;
+  cudaError_t e = cudaGraphCreate(&graph, 0);
+  if (e != cudaSuccess) return fail(DION_ERR_CUDA, "cudaGraphCreate: %s", cudaGetErrorString(e));
+  auto bail = [&](const char* what, cudaError_t err) {
+    cudaGraph_t junk = nullptr;
+    cudaStreamCaptureStatus cst;
+    if (cudaStreamIsCapturing(cs, &cst) == cudaSuccess && cst != cudaStreamCaptureStatusNone)
+      cudaStreamEndCapture(cs, &junk);
+    cudaGraphDestroy(graph);
+    return st != DION_OK ? st : fail(DION_ERR_CUDA, "fallback graph, %s: %s", what, cudaGetErrorString(err));
+  };
+  cudaGraphConditionalHandle cond;
+  e = cudaGraphConditionalHandleCreate(&cond, graph, 0, cudaGraphCondAssignDefault);
+  if (e != cudaSuccess) return bail("conditional handle", e);
+  e = cudaStreamBeginCaptureToGraph(cs, graph, nullptr, nullptr, 0, cudaStreamCaptureModeRelaxed);
+  if (e != cudaSuccess) return bail("capture", e);
+  e = dion::launch_fb_cond(f.flags, f.stats, p.count, cond, f.rounds, kFbMaxRounds, true, cs);
+  if (e != cudaSuccess) return bail("start kernel", e);
+  e = cudaStreamEndCapture(cs, &graph);
+  if (e != cudaSuccess) return bail("end capture", e);
+  cudaGraphNode_t first = nullptr;
+  size_t nnodes = 1;
+  e = cudaGraphGetNodes(graph, &first, &nnodes);
+  if (e != cudaSuccess || nnodes != 1) return bail("start node", e);
+  cudaGraphNodeParams cp{};
+  cp.type = cudaGraphNodeTypeConditional;
+  cp.conditional.handle = cond;
+  cp.conditional.type = cudaGraphCondTypeWhile;
+  cp.conditional.size = 1;
+  cudaGraphNode_t loop = nullptr;
+  e = cudaGraphAddNode(&loop, graph, &first, 1, &cp);
+  if (e != cudaSuccess) return bail("while node", e);
+  cudaGraph_t body = cp.conditional.phGraph_out[0];
+  e = cudaStreamBeginCaptureToGraph(cs, body, nullptr, nullptr, 0, cudaStreamCaptureModeRelaxed);
+  if (e != cudaSuccess) return bail("body capture", e);
+  if ((st = fb_iteration(p, o, f, f.P0s, f.Ps, cs)) != DION_OK) return bail("body", cudaSuccess);
+  if ((st = fb_iteration(p, o, f, f.Ps, f.P0s, cs)) != DION_OK) return bail("body", cudaSuccess);
+  e = dion::launch_fb_cond(f.flags, f.stats, p.count, cond, f.rounds, kFbMaxRounds, false, cs);
+  if (e != cudaSuccess) return bail("condition kernel", e);
+  e = cudaStreamEndCapture(cs, &body);
+  if (e != cudaSuccess) return bail("end body capture", e);
+  e = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (e != cudaSuccess) return fail(DION_ERR_CUDA, "fallback graph instantiate: %s", cudaGetErrorString(e));
+  *out = exec;
+  return DION_OK;
+}
+
+// Launch bucket bi's loop on s, building its graph first if needed.  *launched is false
+// when s is being captured by the caller (a graph with a conditional node is not
+// nested then): the flagged matrices then go to Householder QR directly.
+dion_status fb_launch(dion_handle h, int bi, const Plan& p, const void* ws, const FbBufs& f,
+                      cudaStream_t s, bool* launched) {
+  *launched = false;
+  cudaStreamCaptureStatus cst;
+  if (cudaStreamIsCapturing(s, &cst) != cudaSuccess || cst != cudaStreamCaptureStatusNone)
+    return DION_OK;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(DION_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (h->cap && h->cap_device != dev) {
+    cudaStreamDestroy(h->cap);
+    h->cap = nullptr;
+  }
+  if (!h->cap) {
+    e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return fail(DION_ERR_CUDA, "capture stream: %s", cudaGetErrorString(e));
+    h->cap_device = dev;
+  }
+  if (h->fb.size() < h->plans.size()) h->fb.resize(h->plans.size(), dion_ctx::FbGraph{nullptr, -1, nullptr});
+  dion_ctx::FbGraph& g = h->fb[bi];
+  if (g.exec && (g.ws != ws || g.device != dev)) {
+    cudaGraphExecDestroy(g.exec);
+    g.exec = nullptr;
+  }
+  if (!g.exec) {
+    dion_status st = fb_build(h, p, f, &g.exec);
+    if (st != DION_OK) return st;
+    g.ws = ws;
+    g.device = dev;
+  }
+  e = cudaGraphLaunch(g.exec, s);
+  if (e != cudaSuccess) return fail(DION_ERR_CUDA, "fallback graph launch: %s", cudaGetErrorString(e));
+  *launched = true;
+  return DION_OK;
+}
+
 // Phases of one step; each runs over every bucket before the next starts.
 enum Phase { PH_INIT, PH_PREPQ, PH_FORMB, PH_BQ, PH_ORTH, PH_BTP, PH_COLNORM, PH_UPDATE,
              PH_STATUS, PH_COUNT };
@@ -170,6 +319,8 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
   __nv_bfloat16* P0s = reinterpret_cast<__nv_bfloat16*>(ws + p.off_P0s);
   __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ps);
   __nv_bfloat16* Linvs = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Linvs);
+  __nv_bfloat16* Ws = p.off_Ws ? reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ws) : nullptr;
+  __nv_bfloat16* Ts = p.off_Ts ? reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ts) : nullptr;
   int& p0s_ready = c.p0s_ready[bi];
   const int64_t m = p.m, n = p.n, r = p.r;
   const int cnt = p.count;
@@ -279,8 +430,8 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     dion::CholArgs ca{};
     ca.W = W; ca.Linv = Linv; ca.dinv = dinv; ca.flags = flags; ca.stats = stats;
     ca.count = cnt; ca.r = r; ca.fallback_cond = o.fallback_cond;
-    const int chol_launches = r <= 256 ? 1 : (int)(2 + 3 * ((r + 31) / 32) + (r + 31) / 32);
-    const int64_t mr = (int64_t)cnt * m * r, rr = (int64_t)cnt * r * r;
+    const int chol_launches = dion::chol_inv_launches(r);
+    const int64_t mr = (int64_t)cnt * m * r;
     // tensor cores: Gram and triangular apply from three-way bf16 splits (fp32-accurate)
     int nl = 0;
     bool done = false;
@@ -294,24 +445,39 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     if (o.orth_mode != DION_ORTH_HOUSEHOLDER && tensor) {
       dion_status st;
       cudaError_t e;
+      // L^-1 and its split (the factorisation writes both): one kernel for r <= 256,
+      // the recursion on the tensor cores above
+      ca.Linvs = Linvs;
+      auto chol = [&]() -> dion_status {
+        if (r <= 256) {
+          DION_LAUNCH(c, 1, dion::launch_chol_inv(ca, s));
+          return DION_OK;
+        }
+        const char* what = "";
+        e = dion::launch_chol_inv_rec(ca, Ws, Ts, o.max_wait_spins, s, &nl, &done, &what);
+        c.launches += nl;
+        if (e != cudaSuccess)
+          return fail(DION_ERR_CUDA, "recursive factorisation (%s): %s", what, cudaGetErrorString(e));
+        if (!done) return fail(DION_ERR_CUDA, "recursive factorisation (%s): %s", what,
+                               dion::tc_map_error());
+        return DION_OK;
+      };
       if (!p0s_ready) DION_LAUNCH(c, 1, dion::launch_split3(P0, P0s, mr, mr, s));
-      e = dion::tc_gram(P0s, W, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s, &nl,
-                        &done);
+      e = dion::tc_gram(P0s, W, Ws, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s,
+                        &nl, &done);
       if ((st = tc_check(e, "tc_gram")) != DION_OK) return st;
       ca.pass = 1; ca.orth_tol = o.orth_tol;
-      DION_LAUNCH(c, chol_launches, dion::launch_chol_inv(ca, s));
-      DION_LAUNCH(c, 1, dion::launch_split3(Linv, Linvs, rr, rr, s));
+      if ((st = chol()) != DION_OK) return st;
       e = dion::tc_apply(P0s, Linvs, P, Ps, cnt, m, r, flags, 0, DION_MAT_FALLBACK,
                          o.max_wait_spins, s, &nl, &done);
       if ((st = tc_check(e, "tc_apply")) != DION_OK) return st;
       if (o.orth_mode != DION_ORTH_CHOLQR) {
-        e = dion::tc_gram(Ps, W, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s, &nl,
-                          &done);
+        e = dion::tc_gram(Ps, W, Ws, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s,
+                          &nl, &done);
         if ((st = tc_check(e, "tc_gram")) != DION_OK) return st;
         ca.pass = 2;
         ca.orth_tol = o.orth_mode == DION_ORTH_CHOLQR2 ? -1.f : o.orth_tol;
-        DION_LAUNCH(c, chol_launches, dion::launch_chol_inv(ca, s));
-        DION_LAUNCH(c, 1, dion::launch_split3(Linv, Linvs, rr, rr, s));
+        if ((st = chol()) != DION_OK) return st;
         e = dion::tc_apply(Ps, Linvs, P2, nullptr, cnt, m, r, flags, DION_MAT_CHOLQR2,
                            DION_MAT_FALLBACK, o.max_wait_spins, s, &nl, &done);
         if ((st = tc_check(e, "tc_apply")) != DION_OK) return st;
@@ -328,6 +494,15 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
         DION_LAUNCH(c, chol_launches, dion::launch_chol_inv(ca, s));
         DION_LAUNCH(c, gl, dion::launch_gemm_simt(apply(P, P2, DION_MAT_CHOLQR2), false, s));
       }
+    }
+    // matrices Cholesky-QR gave up on: r > 256 on the tensor path iterate shifted
+    // Cholesky-QR (on the tensor cores); Householder QR takes the rest, one CTA each
+    if (tensor && r > 256 && o.orth_mode != DION_ORTH_HOUSEHOLDER) {
+      FbBufs fbb{W, Linv, stats, P, flags, sched + kFbRoundsSlot, P0s, Ps, Ws, Ts, Linvs};
+      bool launched = false;
+      dion_status fst = fb_launch(c.h, bi, p, ws, fbb, s, &launched);
+      if (fst != DION_OK) return fst;
+      c.launches += launched ? 1 : 0;
     }
     DION_LAUNCH(c, 1, dion::launch_householder(P0, p0s_ready ? P0s : nullptr, P2, P0, P, flags,
                                                cnt, m, r, s));
@@ -574,12 +749,17 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
     p.off_Qng = (bf || split) ? take(c * d.n * d.r * ge) : 0;
     p.off_part = take(c * p.nsplit * d.r * 4);
     p.off_flags = take(c * 4);
-    p.off_stats = take(c * 8);
+    p.off_stats = take(c * 4 * 4);
     // three-way bf16 splits for the tensor-core orthonormalisation
     p.off_P0s = take(c * d.m * d.r * 6);
     p.off_Ps = take(c * d.m * d.r * 6);
     p.off_Linvs = take(c * d.r * d.r * 6);
     p.off_sched = take(64);  // tile counters of the dynamically scheduled kernels
+    if (o.kernel_path == DION_PATH_TENSOR && d.r > 256) {
+      // splits of the Gram / its updates and of L21 for the recursive factorisation
+      p.off_Ws = take(c * d.r * d.r * 6);
+      p.off_Ts = take(c * d.r * d.r * 6);
+    }
     plans.push_back(p);
   }
   dion_ctx* h = new (std::nothrow) dion_ctx();
@@ -596,6 +776,8 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
   for (int i = 0; i < DION_KCLASS_COUNT; ++i) { h->prof_ms[i] = 0; h->prof_launches[i] = 0; }
   h->side_device = -1;
   h->fork_ev = nullptr;
+  h->cap = nullptr;
+  h->cap_device = -1;
   *out = h;
   *workspace_bytes = off;
   return DION_OK;
@@ -610,34 +792,51 @@ dion_status dion_step_batched(dion_handle h, const dion_bucket_ptrs* ptrs, int32
   cudaStream_t main = reinterpret_cast<cudaStream_t>(stream);
   StepCtx c{h, main, 0, -1, nullptr, 0, std::vector<int>(nbuckets, 0)};
   char* ws = static_cast<char*>(d_workspace);
-  // the buckets' orthonormalisations are chains of short, latency-bound kernels:
-  // run them side by side on their own streams, forked from and joined to `main`
+  // Each bucket's orthonormalisation is a chain of short, latency-bound kernels that
+  // needs only that bucket's P0.  It is forked onto the bucket's own stream as soon
+  // as B Q has written P0, so it runs beside the B Q of the later buckets and the
+  // B^T P, column norms and update of the earlier ones; the main stream joins it
+  // just before that bucket's B^T P.
   const bool fork = nbuckets > 1 && ensure_side_streams(h, (size_t)nbuckets);
-  for (int phase = 0; phase < PH_COUNT; ++phase) {
-    const bool side = fork && phase == PH_ORTH;
-    if (side) {
+  int32_t forked = 0, joined = 0;  // side streams [joined, forked) still to be joined
+  auto run = [&](int phase, int32_t b, cudaStream_t s) -> dion_status {
+    c.s = s;
+    return run_bucket(c, b, phase, h->plans[b], ptrs[b], lr, ws, d_status);
+  };
+  auto finish = [&](dion_status result) -> dion_status {
+    end_cls(c);
+    // a failed step still leaves `main` ordered after every forked chain
+    for (; joined < forked; ++joined) cudaStreamWaitEvent(main, h->side_done[joined], 0);
+    h->last_launches = c.launches;
+    return result;
+  };
+  for (int phase : {PH_INIT, PH_PREPQ})
+    for (int32_t b = 0; b < nbuckets; ++b)
+      if ((st = run(phase, b, main)) != DION_OK) return finish(st);
+  for (int32_t b = 0; b < nbuckets; ++b) {
+    for (int phase : {PH_FORMB, PH_BQ})
+      if ((st = run(phase, b, main)) != DION_OK) return finish(st);
+    if (fork) {
       cudaEventRecord(h->fork_ev, main);
-      for (int32_t b = 0; b < nbuckets; ++b) cudaStreamWaitEvent(h->side[b], h->fork_ev, 0);
+      cudaStreamWaitEvent(h->side[b], h->fork_ev, 0);
+      st = run(PH_ORTH, b, h->side[b]);
+      end_cls(c);
+      cudaEventRecord(h->side_done[b], h->side[b]);
+      forked = b + 1;
+    } else {
+      st = run(PH_ORTH, b, main);
     }
-    for (int32_t b = 0; b < nbuckets; ++b) {
-      c.s = side ? h->side[b] : main;
-      st = run_bucket(c, b, phase, h->plans[b], ptrs[b], lr, ws, d_status);
-      if (st != DION_OK) {
-        end_cls(c);
-        h->last_launches = c.launches;
-        return st;
-      }
-    }
-    if (side) {
-      for (int32_t b = 0; b < nbuckets; ++b) {
-        cudaEventRecord(h->side_done[b], h->side[b]);
-        cudaStreamWaitEvent(main, h->side_done[b], 0);
-      }
-      c.s = main;
-    }
+    if (st != DION_OK) return finish(st);
   }
-  h->last_launches = c.launches;
-  return DION_OK;
+  for (int32_t b = 0; b < nbuckets; ++b) {
+    if (fork) {
+      cudaStreamWaitEvent(main, h->side_done[b], 0);
+      joined = b + 1;
+    }
+    for (int phase : {PH_BTP, PH_COLNORM, PH_UPDATE, PH_STATUS})
+      if ((st = run(phase, b, main)) != DION_OK) return finish(st);
+  }
+  return finish(DION_OK);
 }
 
 dion_status dion_step_batched_from_host(dion_handle h, const dion_bucket_ptrs* ptrs,
@@ -677,6 +876,9 @@ dion_status dion_free(dion_handle h) {
   for (auto st : h->side) cudaStreamDestroy(st);
   for (auto ev : h->side_done) cudaEventDestroy(ev);
   if (h->fork_ev) cudaEventDestroy(h->fork_ev);
+  for (auto& g : h->fb)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  if (h->cap) cudaStreamDestroy(h->cap);
   h->magic = 0;
   delete h;
   return DION_OK;

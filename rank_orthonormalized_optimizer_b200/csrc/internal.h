@@ -1,6 +1,7 @@
 // Internal interface between the host planner (dion_api.cu) and the kernels.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -72,6 +73,7 @@ cudaError_t launch_update_simt(const void* Pg, const void* Rg, const void* Qg, b
 struct CholArgs {
   float* W;            // [count, r, r] Gram on entry (lower part overwritten by L)
   float* Linv;         // [count, r, r] receives L^-1 (upper part zero)
+  __nv_bfloat16* Linvs;  // [3][count, r, r] three-way split of L^-1 (may be null)
   float* dinv;         // [count, r, 32] scratch: inverses of 32x32 diagonal blocks
   int32_t* flags;      // [count]
   float* stats;        // [count, 2] min and max of diag(L) (positive floats)
@@ -80,9 +82,32 @@ struct CholArgs {
   int pass;            // 1 or 2
   float fallback_cond; // pass 1: diag ratio limit
   float orth_tol;      // pass 2: skip the second pass when max|W - I| <= orth_tol
+  int64_t o, nl;       // leaf of the recursive factorisation: block (o, o) of size nl
+  int64_t m;           // rows of P0 (pass 3: scales the shift)
 };
+// pass 3 = one step of the shifted Cholesky-QR iteration (launch_chol_inv_rec only)
+// r <= 256: one kernel; larger r: the blocked CUDA-core factorisation (many launches).
 cudaError_t launch_chol_inv(const CholArgs& a, cudaStream_t s);
+int chol_inv_launches(int64_t r);
+// Recursive factorisation with the triangular inverse on the tensor cores, for r > 256:
+//   [W11 .; W21 W22] -> L11, L11^-1 (recursion); L21 = W21 L11^-T; W22 -= L21 L21^T;
+//   L22, L22^-1 (recursion); (L^-1)21 = -L22^-1 L21 L11^-1,
+// leaves of at most 256 by the one-kernel factorisation.  Products are fp32-accurate
+// (three-way bf16 splits).  W's split Ws ([3][count][r][r]) must hold the split of
+// W's lower 128 x 128 tiles on entry (the Gram writes it); Ts is scratch of the same
+// size.  a.Linvs is required.  *nlaunch receives the number of kernels launched;
+// *what names the failing step when the return is not cudaSuccess or *done is false.
+cudaError_t launch_chol_inv_rec(const CholArgs& a, __nv_bfloat16* Ws, __nv_bfloat16* Ts,
+                                int64_t max_spins, cudaStream_t s, int* nlaunch, bool* done,
+                                const char** what);
+// Shifted Cholesky-QR iteration for the flagged matrices (r > 256): the loop's
+// condition kernel (begin: reset the iteration state) and the per-iteration marker.
+cudaError_t launch_fb_cond(int32_t* flags, float* stats, int count, cudaGraphConditionalHandle h,
+                           int* rounds, int max_rounds, bool begin, cudaStream_t s);
+cudaError_t launch_fb_mark(int32_t* flags, int count, cudaStream_t s);
 // P0 fp32, or (when P0s is not null) its three-way bf16 split [3][count][m][r].
+// Matrices flagged F_FALLBACK and not finished by the shifted iteration; those the
+// iteration had started restart from their iterate in P.
 cudaError_t launch_householder(const float* P0, const void* P0s, float* work_cm, float* q_cm,
                                float* P, int32_t* flags, int count, int64_t m, int64_t r,
                                cudaStream_t s);

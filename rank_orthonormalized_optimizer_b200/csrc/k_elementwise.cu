@@ -205,8 +205,10 @@ __global__ void k_init_flags(int32_t* flags, float* stats, int* sched, int count
   if (b < 16) sched[b] = 0;
   if (b < count) {
     flags[b] = init_bits;
-    stats[2 * b] = 3.0e38f;  // running min of diag(L)
-    stats[2 * b + 1] = 0.f;  // running max of diag(L)
+    stats[ST * b] = 3.0e38f;     // running min of diag(L)
+    stats[ST * b + 1] = 0.f;     // running max of diag(L)
+    stats[ST * b + 2] = 0.f;
+    stats[ST * b + 3] = 0.f;
   }
 }
 
@@ -219,7 +221,7 @@ cudaError_t launch_init_flags(int32_t* flags, float* stats, int* sched, int coun
 
 __global__ void k_write_status(const int32_t* flags, int32_t* st, int count) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < count) st[b] = flags[b];
+  if (b < count) st[b] = flags[b] & F_PUBLIC;
 }
 
 cudaError_t launch_write_status(const int32_t* flags, int32_t* d_status, int count,

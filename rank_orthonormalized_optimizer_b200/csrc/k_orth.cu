@@ -16,6 +16,7 @@
 //     factor Cholesky-QR reaches in exact arithmetic.
 #include "common.cuh"
 #include "internal.h"
+#include "tc.h"
 
 namespace dion {
 
@@ -23,97 +24,18 @@ namespace {
 constexpr int CHOL_SMALL_MAX = 256;
 constexpr int NB = 32;  // panel width of the blocked factorisation
 
-__device__ __forceinline__ int64_t tri(int64_t i, int64_t j) { return i * (i + 1) / 2 + j; }
-
+// pass 1: Cholesky-QR; pass 2: its second pass (matrices with F_CHOLQR2); pass 3: the
+// shifted iteration (matrices with F_FALLBACK still iterating)
 __device__ __forceinline__ bool skip_matrix(int32_t f, int pass) {
+  if (pass == 3) return !(f & F_FALLBACK) || (f & (F_SDONE | F_SFAIL | F_NONFINITE));
   return (f & F_FALLBACK) || (pass == 2 && !(f & F_CHOLQR2));
 }
-}  // namespace
-
-// ------------------------------------------------ r <= 256: one CTA, shared memory
-template <int NT>
-__global__ void __launch_bounds__(NT) k_chol_small(CholArgs a) {
-  extern __shared__ float sm[];
-  const int64_t r = a.r;
-  float* L = sm;                  // packed lower triangle, r(r+1)/2
-  float* col = L + tri(r, 0);     // r
-  float* red = col + r;           // 32
-  const int b = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NW = NT / 32;
-  const int32_t f0 = a.flags[b];
-  if (f0 & F_FALLBACK) return;
-  const float* W = a.W + (int64_t)b * r * r;
-
-  float dev = 0.f;
-  bool nonfin = false;
-  for (int64_t i = warp; i < r; i += NW)
-    for (int64_t j = lane; j <= i; j += 32) {
-      const float v = W[i * r + j];
-      L[tri(i, j)] = v;
-      nonfin |= !isfinite(v);
-      dev = fmaxf(dev, fabsf(v - (i == j ? 1.f : 0.f)));
-    }
-  nonfin = __syncthreads_or(nonfin);
-  if (nonfin) {
-    if (tid == 0) atomicOr(a.flags + b, F_NONFINITE | F_FALLBACK);
-    return;
-  }
-  if (a.pass == 2) {
-    dev = block_max<NT>(dev, red);
-    if (dev <= a.orth_tol) return;  // the first pass is orthonormal enough
-  }
-
-  // right-looking Cholesky, column by column
-  float dmin = 3.0e38f, dmax = 0.f;
-  bool fail = false;
-  for (int64_t j = 0; j < r; ++j) {
-    const float d = L[tri(j, j)];
-    if (!(d > 0.f) || !isfinite(d)) { fail = true; break; }
-    const float ljj = sqrtf(d);
-    dmin = fminf(dmin, ljj);
-    dmax = fmaxf(dmax, ljj);
-    for (int64_t i = j + 1 + tid; i < r; i += NT) {
-      const float v = L[tri(i, j)] / ljj;
-      L[tri(i, j)] = v;
-      col[i] = v;
-    }
-    __syncthreads();
-    if (tid == 0) L[tri(j, j)] = ljj;
-    for (int64_t i = j + 1 + warp; i < r; i += NW) {
-      const float ci = col[i];
-      for (int64_t k = j + 1 + lane; k <= i; k += 32) L[tri(i, k)] -= ci * col[k];
-    }
-    __syncthreads();
-  }
-  if (fail || (a.pass == 1 && dmax > a.fallback_cond * dmin)) {
-    if (tid == 0) atomicOr(a.flags + b, F_FALLBACK);
-    return;
-  }
-  if (tid == 0) {
-    a.stats[2 * b] = dmin;
-    a.stats[2 * b + 1] = dmax;
-  }
-
-  // L^-1 in place, row by row: row i of the inverse needs rows < i of it
-  for (int64_t i = 0; i < r; ++i) {
-    for (int64_t k = tid; k <= i; k += NT) col[k] = L[tri(i, k)];
-    __syncthreads();
-    const float inv_ii = 1.f / col[i];
-    for (int64_t j = warp; j < i; j += NW) {
-      float s = 0.f;
-      for (int64_t k = j + lane; k < i; k += 32) s = fmaf(col[k], L[tri(k, j)], s);
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) L[tri(i, j)] = -s * inv_ii;
-    }
-    if (tid == 0) L[tri(i, i)] = inv_ii;
-    __syncthreads();
-  }
-  float* Li = a.Linv + (int64_t)b * r * r;
-  for (int64_t i = warp; i < r; i += NW)
-    for (int64_t j = lane; j < r; j += 32) Li[i * r + j] = (j <= i) ? L[tri(i, j)] : 0.f;
-  if (a.pass == 2 && tid == 0) atomicOr(a.flags + b, F_CHOLQR2);
+// the bits a failed factorisation sets
+__device__ __forceinline__ int32_t fail_bits(int pass, bool nonfinite) {
+  if (pass == 3) return F_SFAIL;
+  return nonfinite ? (F_NONFINITE | F_FALLBACK) : F_FALLBACK;
 }
+}  // namespace
 
 // ------------------------------------ r <= 256: one CTA, 32 x 32 blocks in shared memory
 // Right-looking blocked Cholesky with the triangular inverse, all on chip:
@@ -123,6 +45,10 @@ __global__ void __launch_bounds__(NT) k_chol_small(CholArgs a) {
 //   then L^-1 block row by block row: X_ij = -D_i sum_{k=j}^{i-1} L_ik X_kj, X_ii = D_i.
 // Rows and columns past r are padded with the identity, which factors and inverts
 // to itself.  Padded stride 33 keeps row-per-lane accesses free of bank conflicts.
+// With a.nl > 0 the kernel factors the diagonal block of size nl at (a.o, a.o) of each
+// matrix as a leaf of the recursive factorisation: the pass-2 test against I was made
+// for the whole matrix before, the diagonal statistics are merged by atomics, and the
+// diagonal-ratio test is left to the end of the recursion.
 namespace {
 constexpr int CB = 32, CBS = 33, CBLK = CB * CBS;
 __device__ __forceinline__ float* blk_at(float* base, int i, int j) {
@@ -138,7 +64,10 @@ size_t chol_blocked_smem_bytes(int64_t r) {
 template <int NT>
 __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
   extern __shared__ float sm[];
-  const int r = (int)a.r;
+  const bool leaf = a.nl > 0;
+  const int r = (int)(leaf ? a.nl : a.r);  // size of the factored block
+  const int64_t ld = a.r;                  // row stride of W and L^-1
+  const int64_t org = a.o * ld + a.o;      // block origin inside each matrix
   const int T = (r + CB - 1) / CB;
   float* blk = sm;                                  // T(T+1)/2 lower blocks
   float* dinv = blk + (T * (T + 1) / 2) * CBLK;     // T inverses of the diagonal blocks
@@ -149,8 +78,8 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = NT / 32;
   const int32_t f0 = a.flags[b];
-  if (f0 & F_FALLBACK) return;
-  const float* W = a.W + (int64_t)b * r * r;
+  if ((leaf || a.pass == 3) ? skip_matrix(f0, a.pass) : (f0 & F_FALLBACK) != 0) return;
+  const float* W = a.W + (int64_t)b * ld * ld + org;
 
   // load the lower blocks, padding with the identity; check finiteness and |W - I|
   float dev = 0.f;
@@ -164,7 +93,7 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
     const int gi = bi * CB + u, gj = bj * CB + v;
     float val;
     if (gi < r && gj < r) {
-      val = W[(int64_t)gi * r + gj];
+      val = W[(int64_t)gi * ld + gj];
       if (gj <= gi) {
         nonfin |= !isfinite(val);
         dev = fmaxf(dev, fabsf(val - (gi == gj ? 1.f : 0.f)));
@@ -177,10 +106,10 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
   if (tid == 0) s_fail = 0;
   nonfin = __syncthreads_or(nonfin);
   if (nonfin) {
-    if (tid == 0) atomicOr(a.flags + b, F_NONFINITE | F_FALLBACK);
+    if (tid == 0) atomicOr(a.flags + b, fail_bits(a.pass, true));
     return;
   }
-  if (a.pass == 2) {
+  if (a.pass == 2 && !leaf) {
     dev = block_max<NT>(dev, red);
     if (dev <= a.orth_tol) return;  // the first pass is orthonormal enough
   }
@@ -234,7 +163,7 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
     }
     __syncthreads();
     if (s_fail) {
-      if (tid == 0) atomicOr(a.flags + b, F_FALLBACK);
+      if (tid == 0) atomicOr(a.flags + b, fail_bits(a.pass, false));
       return;
     }
     // panel: L_ik = W_ik D_k^T, one thread per row of the panel
@@ -276,15 +205,20 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
     __syncthreads();
   }
 
-  if (a.pass == 1 && dmax > a.fallback_cond * dmin) s_fail = 1;  // warp 0 only
+  if (!leaf && a.pass == 1 && dmax > a.fallback_cond * dmin) s_fail = 1;  // warp 0 only
   __syncthreads();
   if (s_fail) {
     if (tid == 0) atomicOr(a.flags + b, F_FALLBACK);
     return;
   }
   if (tid == 0) {
-    a.stats[2 * b] = dmin;
-    a.stats[2 * b + 1] = dmax;
+    if (leaf) {
+      atomic_min_pos(a.stats + ST * b, dmin);
+      atomic_max_pos(a.stats + ST * b + 1, dmax);
+    } else {
+      a.stats[ST * b] = dmin;
+      a.stats[ST * b + 1] = dmax;
+    }
   }
 
   // L^-1 block row by block row; X_ij overwrites L_ij once row i is done
@@ -324,8 +258,10 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
     __syncthreads();
   }
 
-  // write L^-1 (zeros above the diagonal)
-  float* Li = a.Linv + (int64_t)b * r * r;
+  // write L^-1 (zeros above the diagonal) and, when asked, its three-way bf16 split
+  const int64_t mo = (int64_t)b * ld * ld + org;
+  float* Li = a.Linv + mo;
+  const int64_t part = (int64_t)a.count * ld * ld;
   for (int64_t e = tid; e < (int64_t)r * r; e += NT) {
     const int gi = (int)(e / r), gj = (int)(e % r);
     float val = 0.f;
@@ -333,35 +269,61 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
       const int bi = gi / CB, bj = gj / CB, u = gi % CB, v = gj % CB;
       val = (bi == bj) ? dinv[bi * CBLK + u * CBS + v] : blk_at(blk, bi, bj)[u * CBS + v];
     }
-    Li[e] = val;
+    const int64_t at = (int64_t)gi * ld + gj;
+    Li[at] = val;
+    if (a.Linvs) {
+      bf16 h, mi, lo;
+      split3_bf16(val, h, mi, lo);
+      bf16* d = a.Linvs + mo + at;
+      d[0] = h;
+      d[part] = mi;
+      d[2 * part] = lo;
+    }
   }
-  if (a.pass == 2 && tid == 0) atomicOr(a.flags + b, F_CHOLQR2);
+  if (!leaf && a.pass == 2 && tid == 0) atomicOr(a.flags + b, F_CHOLQR2);
 }
 
 // ---------------------------------------------- r > 256: blocked, multi-launch
-// Pass 2 entry: compare W with I; set F_CHOLQR2 when the second pass is needed.
+// Entry of the blocked and recursive factorisations: non-finite entries of W send
+// the matrix to the fallback; in pass 2, W is compared with I and F_CHOLQR2 is set
+// when the second pass is needed.  Grid (count, chunks): any CTA that sees a
+// deviation sets the bit.  Chunk 0 resets the diagonal statistics.
+// Pass 3 (shifted iteration): a deviation sets F_SMORE, a non-finite entry F_SFAIL, and
+// the largest diagonal entry of W goes to the statistics (it scales the shift).
 __global__ void __launch_bounds__(256) k_gram_check(CholArgs a) {
   __shared__ float red[32];
   const int b = blockIdx.x;
+  if (a.pass != 3 && blockIdx.y == 0 && threadIdx.x == 0) {
+    a.stats[ST * b] = 3.0e38f;
+    a.stats[ST * b + 1] = 0.f;
+  }
   const int32_t f = a.flags[b];
-  if (f & F_FALLBACK) return;
+  if (a.pass == 3 ? skip_matrix(f, 3) : (f & F_FALLBACK) != 0) return;
   const int64_t r = a.r;
   const float* W = a.W + (int64_t)b * r * r;
-  float dev = 0.f;
+  float dev = 0.f, dmax = 0.f;
   bool nonfin = false;
-  for (int64_t i = threadIdx.x >> 5; i < r; i += 8)
+  const int64_t rows_per = (r + gridDim.y - 1) / gridDim.y;
+  const int64_t i0 = blockIdx.y * rows_per, i1 = i0 + rows_per < r ? i0 + rows_per : r;
+  for (int64_t i = i0 + (threadIdx.x >> 5); i < i1; i += 8)
     for (int64_t j = threadIdx.x & 31; j <= i; j += 32) {
       const float v = W[i * r + j];
       nonfin |= !isfinite(v);
       dev = fmaxf(dev, fabsf(v - (i == j ? 1.f : 0.f)));
+      if (i == j) dmax = fmaxf(dmax, v);
     }
   nonfin = __syncthreads_or(nonfin);
   dev = block_max<256>(dev, red);
+  if (a.pass == 3) dmax = block_max<256>(dmax, red);
   if (threadIdx.x == 0) {
     if (nonfin)
-      atomicOr(a.flags + b, F_NONFINITE | F_FALLBACK);
+      atomicOr(a.flags + b, a.pass == 3 ? F_SFAIL : (F_NONFINITE | F_FALLBACK));
     else if (a.pass == 2 && dev > a.orth_tol)
       atomicOr(a.flags + b, F_CHOLQR2);
+    else if (a.pass == 3) {
+      if (dev > a.orth_tol) atomicOr(a.flags + b, F_SMORE);
+      atomic_max_pos(a.stats + ST * b + 2, dmax);
+    }
   }
 }
 
@@ -432,8 +394,8 @@ __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int64_t k0) {
     if (i < nb) a.dinv[((int64_t)b * r + k0 + i) * NB + j] = Dinv[i][j];
   }
   if (tid == 0 && a.pass == 1) {
-    atomic_min_pos(a.stats + 2 * b, dmin);
-    atomic_max_pos(a.stats + 2 * b + 1, dmax);
+    atomic_min_pos(a.stats + ST * b, dmin);
+    atomic_max_pos(a.stats + ST * b + 1, dmax);
   }
 }
 
@@ -506,7 +468,7 @@ __global__ void k_chol_cond(CholArgs a) {
   if (b >= a.count) return;
   const int32_t f = a.flags[b];
   if (skip_matrix(f, a.pass)) return;
-  if (a.pass == 1 && a.stats[2 * b + 1] > a.fallback_cond * a.stats[2 * b])
+  if (a.pass == 1 && a.stats[ST * b + 1] > a.fallback_cond * a.stats[ST * b])
     atomicOr(a.flags + b, F_FALLBACK);
 }
 
@@ -569,17 +531,35 @@ __global__ void __launch_bounds__(256) k_trinv_row(CholArgs a, int64_t I) {
 
 size_t chol_dinv_floats(int count, int64_t r) { return (size_t)count * r * NB; }
 
+namespace {
+// CTAs per matrix of the entry check: about 128 rows each, at most 64
+unsigned gram_check_chunks(int64_t r) {
+  const int64_t c = (r + 127) / 128;
+  return (unsigned)(c < 1 ? 1 : (c > 64 ? 64 : c));
+}
+
+cudaError_t launch_chol_blocked(const CholArgs& a, cudaStream_t s) {
+  constexpr int NT = 512;
+  const size_t smem = chol_blocked_smem_bytes(a.nl > 0 ? a.nl : a.r);
+  // the size of the largest block, not of this one: leaves of several sizes are
+  // captured into one graph, whose launches are checked against the attribute later
+  cudaError_t e = cudaFuncSetAttribute(k_chol_blocked<NT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)chol_blocked_smem_bytes(CHOL_SMALL_MAX));
+  if (e != cudaSuccess) return e;
+  k_chol_blocked<NT><<<a.count, NT, smem, s>>>(a);
+  return cudaGetLastError();
+}
+}  // namespace
+
+int chol_inv_launches(int64_t r) {
+  const int64_t T = (r + NB - 1) / NB;
+  return r <= CHOL_SMALL_MAX ? 1 : (int)(2 + 3 * T + T);
+}
+
 cudaError_t launch_chol_inv(const CholArgs& a, cudaStream_t s) {
-  if (a.r <= CHOL_SMALL_MAX) {
-    constexpr int NT = 512;
-    const size_t smem = chol_blocked_smem_bytes(a.r);
-    cudaError_t e = cudaFuncSetAttribute(k_chol_blocked<NT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k_chol_blocked<NT><<<a.count, NT, smem, s>>>(a);
-    return cudaGetLastError();
-  }
-  k_gram_check<<<a.count, 256, 0, s>>>(a);
+  if (a.r <= CHOL_SMALL_MAX) return launch_chol_blocked(a, s);
+  k_gram_check<<<dim3((unsigned)a.count, gram_check_chunks(a.r)), 256, 0, s>>>(a);
   const int64_t T = (a.r + NB - 1) / NB;
   for (int64_t kb = 0; kb < T; ++kb) {
     const int64_t k0 = kb * NB;
@@ -597,14 +577,205 @@ cudaError_t launch_chol_inv(const CholArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// -------------------------------------------- r > 256: recursive, on the tensor cores
+__global__ void k_fb_shift(float* W, int32_t* flags, float* stats, int64_t m, int64_t r);
+
+namespace {
+struct RecCtx {
+  const CholArgs* a;
+  bf16 *Ws, *Ts;
+  int64_t max_spins;
+  cudaStream_t s;
+  int32_t need, skip;
+  int launches;
+  const char* what;
+};
+
+// element offset of entry (i, j) of matrix 0, part 0
+inline int64_t at(const RecCtx& c, int64_t i, int64_t j) { return i * c.a->r + j; }
+
+cudaError_t rec_gemm(RecCtx& c, const TcBlockGemm& g, const char* what, bool* done) {
+  int nl = 0;
+  cudaError_t e = tc_block_gemm(g, c.a->count, c.a->r, c.a->flags, c.need, c.skip, c.max_spins,
+                                c.s, &nl, done);
+  c.launches += nl;
+  if (e != cudaSuccess || !*done) c.what = what;
+  return e;
+}
+
+// Factor the diagonal block (o, o) of size n: L^-1 of the block into Linv / Linvs.
+cudaError_t rec_chol(RecCtx& c, int64_t o, int64_t n, bool* done) {
+  const CholArgs& a = *c.a;
+  if (n <= CHOL_SMALL_MAX) {
+    CholArgs leaf = a;
+    leaf.o = o;
+    leaf.nl = n;
+    ++c.launches;
+    cudaError_t e = launch_chol_blocked(leaf, c.s);
+    if (e != cudaSuccess) c.what = "leaf factorisation";
+    *done = true;
+    return e;
+  }
+  // the first block a multiple of 128 so that every leaf starts on a 128 boundary:
+  // a 128-aligned tile window then never straddles two leaves, which is what lets the
+  // products skip the zero triangles of L^-1 without reading outside the leaves
+  const int64_t n1 = (n / 2 + 127) / 128 * 128, n2 = n - n1, i = o + n1;
+  cudaError_t e = rec_chol(c, o, n1, done);
+  if (e != cudaSuccess || !*done) return e;
+  TcBlockGemm g{};
+  // L21 = W21 (L11^-1)^T, split only, into Ts
+  g.A = c.Ws + at(c, i, o); g.B = a.Linvs + at(c, o, o);
+  g.M = n2; g.N = n1; g.K = n1;
+  g.Cs = c.Ts + at(c, i, o); g.alpha = 1.f; g.kr = TC_KR_B_LOWER_NK;
+  if ((e = rec_gemm(c, g, "L21 = W21 L11^-T", done)) != cudaSuccess || !*done) return e;
+  // W22 -= L21 L21^T (lower tiles), keeping W's split current
+  g = TcBlockGemm{};
+  g.A = c.Ts + at(c, i, o); g.B = c.Ts + at(c, i, o);
+  g.M = n2; g.N = n2; g.K = n1;
+  g.C = a.W + at(c, i, i); g.Cs = c.Ws + at(c, i, i);
+  g.alpha = -1.f; g.accumulate = true; g.lower_only = true;
+  if ((e = rec_gemm(c, g, "W22 -= L21 L21^T", done)) != cudaSuccess || !*done) return e;
+  if ((e = rec_chol(c, i, n2, done)) != cudaSuccess || !*done) return e;
+  // T = L21 L11^-1 (split only, over W21's split, which is no longer needed)
+  g = TcBlockGemm{};
+  g.A = c.Ts + at(c, i, o); g.B = a.Linvs + at(c, o, o); g.b_mn = true;
+  g.M = n2; g.N = n1; g.K = n1;
+  g.Cs = c.Ws + at(c, i, o); g.alpha = 1.f; g.kr = TC_KR_B_LOWER_KN;
+  if ((e = rec_gemm(c, g, "T = L21 L11^-1", done)) != cudaSuccess || !*done) return e;
+  // (L^-1)21 = -L22^-1 T
+  g = TcBlockGemm{};
+  g.A = a.Linvs + at(c, i, i); g.B = c.Ws + at(c, i, o); g.b_mn = true;
+  g.M = n2; g.N = n1; g.K = n2;
+  g.C = a.Linv + at(c, i, o); g.Cs = a.Linvs + at(c, i, o);
+  g.alpha = -1.f; g.kr = TC_KR_A_LOWER_MK;
+  return rec_gemm(c, g, "(L^-1)21 = -L22^-1 T", done);
+}
+}  // namespace
+
+cudaError_t launch_chol_inv_rec(const CholArgs& a, bf16* Ws, bf16* Ts, int64_t max_spins,
+                                cudaStream_t s, int* nlaunch, bool* done, const char** what) {
+  *nlaunch = 0;
+  *done = false;
+  *what = "";
+  if (a.r <= CHOL_SMALL_MAX || !a.Linvs || !Ws || !Ts || a.nl != 0) return cudaErrorInvalidValue;
+  const int32_t need = a.pass == 2 ? F_CHOLQR2 : (a.pass == 3 ? F_FALLBACK : 0);
+  const int32_t skip = a.pass == 3 ? (F_SDONE | F_SFAIL | F_NONFINITE) : F_FALLBACK;
+  RecCtx c{&a, Ws, Ts, max_spins, s, need, skip, 0, ""};
+  k_gram_check<<<dim3((unsigned)a.count, gram_check_chunks(a.r)), 256, 0, s>>>(a);
+  ++c.launches;
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess && a.pass == 3) {
+    k_fb_shift<<<a.count, 256, 0, s>>>(a.W, a.flags, a.stats, a.m, a.r);
+    ++c.launches;
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = rec_chol(c, 0, a.r, done);
+  else c.what = "entry check";
+  if (e == cudaSuccess && *done) {
+    k_chol_cond<<<(a.count + 255) / 256, 256, 0, s>>>(a);
+    ++c.launches;
+    e = cudaGetLastError();
+    if (e != cudaSuccess) c.what = "diagonal-ratio test";
+  }
+  *nlaunch = c.launches;
+  *what = c.what;
+  return e;
+}
+
+// ------------------------------------- shifted Cholesky-QR iteration (fallback, r > 256)
+// For the matrices whose Cholesky-QR failed (F_FALLBACK, finite): A_0 = P0,
+// A_{k+1} = A_k R_k^-1 with R_k^T R_k = A_k^T A_k + s_k I.  Every iterate is P0 times an
+// upper-triangular matrix with a positive diagonal, so the orthonormal limit is P0's
+// Q factor with diag(R) > 0, the same P as Householder QR (shifted Cholesky-QR:
+// Fukaya, Kannan, Nakatsukasa, Yamamoto and Yanagisawa, SIAM J. Sci. Comput. 2020).
+// The shift s_k = 2 u (sqrt(m r) + r) max_i (A_k^T A_k)_ii (u = 2^-24) exceeds the
+// rounding of the computed Gram, so the factorisation exists; singular values below
+// sqrt(s_k) grow by about 1/sqrt(s_k) per step.  Once every pivot of a shifted
+// factorisation is above 10 sqrt(s_k) the iterate is well conditioned and later steps
+// are plain Cholesky-QR.  A matrix is done when max |A_k^T A_k - I| <= orth_tol.
+
+// Start (begin != 0) or continue the loop: the conditional is set while some matrix
+// is still iterating and fewer than max_rounds rounds have run.  One CTA.
+__global__ void __launch_bounds__(256) k_fb_cond(int32_t* flags, float* stats, int count,
+                                                 cudaGraphConditionalHandle h, int* rounds,
+                                                 int max_rounds, int begin) {
+  bool any = false;
+  for (int b = threadIdx.x; b < count; b += blockDim.x) {
+    const int32_t f = flags[b];
+    if (begin) {
+      if ((f & F_FALLBACK) && !(f & F_NONFINITE)) {
+        atomicAnd(flags + b, ~(F_SMORE | F_SDONE | F_SFAIL | F_SITER | F_SNOSHIFT));
+        stats[ST * b] = 3.0e38f;
+        stats[ST * b + 2] = 0.f;
+        stats[ST * b + 3] = 0.f;
+        any = true;
+      }
+    } else {
+      any |= !skip_matrix(f, 3);
+    }
+  }
+  any = __syncthreads_or(any);
+  if (threadIdx.x == 0) {
+    const int k = begin ? 0 : *rounds + 1;
+    *rounds = k;
+    cudaGraphSetConditional(h, (any && k < max_rounds) ? 1u : 0u);
+  }
+}
+
+// After the entry check of an iteration: finish converged matrices; otherwise add the
+// shift to the diagonal of W.  One CTA per matrix.
+__global__ void __launch_bounds__(256) k_fb_shift(float* W, int32_t* flags, float* stats,
+                                                  int64_t m, int64_t r) {
+  const int b = blockIdx.x;
+  const int32_t f = flags[b];
+  if (skip_matrix(f, 3)) return;
+  const float dmin = stats[ST * b], dmax_w = stats[ST * b + 2], s_prev = stats[ST * b + 3];
+  __syncthreads();
+  if ((f & F_SITER) && !(f & F_SMORE)) {
+    if (threadIdx.x == 0) atomicOr(flags + b, F_SDONE);
+    return;
+  }
+  const bool noshift = (f & F_SNOSHIFT) || (s_prev > 0.f && dmin * dmin > 100.f * s_prev);
+  const float s = noshift ? 0.f
+                          : 2.f * 5.9604645e-8f * (sqrtf((float)m * (float)r) + (float)r) * dmax_w;
+  if (s > 0.f) {
+    float* w = W + (int64_t)b * r * r;
+    for (int64_t i = threadIdx.x; i < r; i += blockDim.x) w[i * r + i] += s;
+  }
+  if (threadIdx.x == 0) {
+    atomicAnd(flags + b, ~F_SMORE);
+    if (noshift) atomicOr(flags + b, F_SNOSHIFT);
+    stats[ST * b] = 3.0e38f;
+    stats[ST * b + 2] = 0.f;
+    stats[ST * b + 3] = s;
+  }
+}
+
+// After the apply of an iteration: the matrices still iterating now hold A_{k+1} in P.
+__global__ void k_fb_mark(int32_t* flags, int count) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < count && !skip_matrix(flags[b], 3)) atomicOr(flags + b, F_SITER);
+}
+
+cudaError_t launch_fb_cond(int32_t* flags, float* stats, int count, cudaGraphConditionalHandle h,
+                           int* rounds, int max_rounds, bool begin, cudaStream_t s) {
+  k_fb_cond<<<1, 256, 0, s>>>(flags, stats, count, h, rounds, max_rounds, begin ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fb_mark(int32_t* flags, int count, cudaStream_t s) {
+  k_fb_mark<<<(count + 255) / 256, 256, 0, s>>>(flags, count);
+  return cudaGetLastError();
+}
+
 // -------------------------------------------------------------- Householder
 // Thin QR of P0 (m x r) for the matrices flagged F_FALLBACK.  work_cm and
 // q_cm are m x r column-major scratch (q_cm may alias P0: P0 is read first).
 // P receives the orthonormal factor with column signs fixed so that the
 // triangular factor has a non-negative diagonal.
 __global__ void __launch_bounds__(1024) k_householder(const float* P0, const bf16* P0s,
-                                                      int64_t split_stride, float* work_cm,
-                                                      float* q_cm, float* P,
+                                                      const float* Pit, int64_t split_stride,
+                                                      float* work_cm, float* q_cm, float* P,
                                                       const int32_t* flags, int64_t m,
                                                       int64_t r) {
   extern __shared__ float hs[];
@@ -613,10 +784,14 @@ __global__ void __launch_bounds__(1024) k_householder(const float* P0, const bf1
   float* red = hs + 2 * r;  // 32
   __shared__ float tile[32][33];
   const int b = blockIdx.x;
-  if (!(flags[b] & F_FALLBACK)) return;
+  const int32_t f = flags[b];
+  if (!(f & F_FALLBACK) || (f & F_SDONE)) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = 32;
-  const float* p0 = P0 + (int64_t)b * m * r;
+  // an iterate P0 R^-1 of the shifted iteration has the same Q factor as P0
+  const bool iter = (f & F_SITER) != 0;
+  if (iter) P0s = nullptr;
+  const float* p0 = (iter ? Pit : P0) + (int64_t)b * m * r;
   float* A = work_cm + (int64_t)b * m * r;
   float* Qc = q_cm + (int64_t)b * m * r;
   float* Pout = P + (int64_t)b * m * r;
@@ -710,14 +885,15 @@ __global__ void __launch_bounds__(1024) k_householder(const float* P0, const bf1
 cudaError_t launch_householder(const float* P0, const void* P0s, float* work_cm, float* q_cm,
                                float* P, int32_t* flags, int count, int64_t m, int64_t r,
                                cudaStream_t s) {
+  // matrices the shifted iteration left unfinished restart from their iterate, held in P
   const size_t smem = (size_t)(2 * r + 32) * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k_householder,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  k_householder<<<count, 1024, smem, s>>>(P0, (const bf16*)P0s, (int64_t)count * m * r, work_cm,
-                                          q_cm, P, flags, m, r);
+  k_householder<<<count, 1024, smem, s>>>(P0, (const bf16*)P0s, P, (int64_t)count * m * r,
+                                          work_cm, q_cm, P, flags, m, r);
   return cudaGetLastError();
 }
 

@@ -86,11 +86,49 @@ static bool map3d(CUtensorMap* m, const void* base, bool bf16, uint64_t d0, uint
   return true;
 }
 
+// 3-D map over a block (d1 rows x d0 columns) of each matrix of a stack whose rows are
+// ld elements apart and whose matrices are ms elements apart.
+static bool map3d_block(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                        uint64_t ld, uint64_t ms, uint32_t b0, uint32_t b1) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) {
+    snprintf(tl_map_error, sizeof(tl_map_error), "cuTensorMapEncodeTiled unavailable");
+    return false;
+  }
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {ld * 2, ms * 2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(tl_map_error, sizeof(tl_map_error),
+             "cuTensorMapEncodeTiled -> %d (block base %p, %llu x %llu x %llu, ld %llu, box %u x %u)",
+             (int)r, base, (unsigned long long)d0, (unsigned long long)d1, (unsigned long long)d2,
+             (unsigned long long)ld, b0, b1);
+    return false;
+  }
+  return true;
+}
+
 }  // namespace tc
 
 const char* tc_map_error() { return tc::tl_map_error; }
 
 namespace tc {
+
+static int smem_optin() {
+  static int bytes = 0;
+  if (!bytes) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&bytes, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (bytes <= 0) bytes = 227 * 1024;
+  }
+  return bytes;
+}
 
 static int sm_count() {
   static int sms = 0;
@@ -138,8 +176,22 @@ struct GemmP {
   int32_t* flags;
   int32_t need_mask, skip_mask;      // matrices whose flags fail this are skipped
   int lower_only;                    // skip tiles above the diagonal (symmetric results)
+  int epi;                           // 0: C = acc;  1: C = alpha acc;  2: C += alpha acc
+  float alpha;
+  int kr;                            // triangular-operand K ranges (TC_KR_* bits)
   int64_t max_spins;
 };
+
+// K blocks [kb0, kb1) that can hold non-zero products for the tile at (m0, n0) when an
+// operand is lower triangular (entries past the diagonal are zero and are not read).
+__device__ __forceinline__ void k_range(const GemmP& p, int m0, int n0, int& kb0, int& kb1) {
+  kb0 = 0;
+  kb1 = p.num_kb;
+  if (p.kr & TC_KR_B_LOWER_NK) kb1 = min(kb1, (n0 + p.block_n + BK - 1) / BK);
+  if (p.kr & TC_KR_B_LOWER_KN) kb0 = n0 / BK;
+  if (p.kr & TC_KR_A_LOWER_MK) kb1 = min(kb1, (m0 + BM + BK - 1) / BK);
+  if (kb1 <= kb0) kb1 = kb0 + 1;  // never empty: a block past K loads as zeros
+}
 
 __device__ __forceinline__ bool tile_active(const GemmP& p, int t, int tiles_per_mat) {
   if (p.lower_only) {
@@ -207,8 +259,10 @@ __global__ void __launch_bounds__(NT, 1)
       const int rem = t % tiles_per_mat;
       const int m0 = (rem / p.tiles_n) * BM;
       const int n0 = (rem % p.tiles_n) * p.block_n;
+      int kb0, kb1;
+      k_range(p, m0, n0, kb0, kb1);
       bool ok = true;
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!wait_bounded(empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
         mbar_expect_tx(full + stage, stage_a + stage_b);
         const int k0 = kb * BK;
@@ -259,8 +313,11 @@ __global__ void __launch_bounds__(NT, 1)
       if (!wait_bounded(tempty + acc, acc_phase ^ 1, p.max_spins, abort)) break;
       tc_fence_after();
       const uint32_t d = tmem + acc * p.acc_stride;
+      const int rem = t % tiles_per_mat;
+      int kb0, kb1;
+      k_range(p, (rem / p.tiles_n) * BM, (rem % p.tiles_n) * p.block_n, kb0, kb1);
       bool ok = true;
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!wait_bounded(full + stage, phase, p.max_spins, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_base = smem_u32(sA + (size_t)stage * stage_a);
@@ -275,7 +332,7 @@ __global__ void __launch_bounds__(NT, 1)
                                      : sw128_desc(ab + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? sw128_desc(bb + k * 2048, 8192, 1024)
                                      : sw128_desc(bb + k * 32, 16, 1024);
-            mma_bf16(d, ad, bd, p.idesc, (kb | k | q) != 0);
+            mma_bf16(d, ad, bd, p.idesc, ((kb - kb0) | k | q) != 0);
           }
         }
         mma_commit(empty + stage);
@@ -309,6 +366,19 @@ __global__ void __launch_bounds__(NT, 1)
         tmem_ld16(tbase + c, v);
         tmem_wait_ld();
         if (row < p.M && n0 + c < p.N) {
+          if (p.epi != 0) {
+            float old[16];
+            if (p.epi == 2) {
+              const float4* src = reinterpret_cast<const float4*>(p.C + off + n0 + c);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float4 o4 = src[q];
+                old[4 * q] = o4.x; old[4 * q + 1] = o4.y; old[4 * q + 2] = o4.z; old[4 * q + 3] = o4.w;
+              }
+            }
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[q] = p.epi == 2 ? fmaf(p.alpha, v[q], old[q]) : p.alpha * v[q];
+          }
           if (p.C) {
             float4* dst = reinterpret_cast<float4*>(p.C + off + n0 + c);
 #pragma unroll
@@ -366,8 +436,13 @@ static cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Gem
   p.tmem_cols = pow2_cols(2 * p.block_n);
   const size_t smem = 1024 + stages * stage_bytes + (2 * stages + 5) * 8 + 16;
   auto kern = k_tc_gemm<A_MN, B_MN, SPLIT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // the device's limit rather than this launch's need: a launch captured into a graph
+  // is checked against the attribute when the graph runs, after later launches of the
+  // same kernel with other shapes may have set it
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem_optin());
   if (e != cudaSuccess) return e;
+  if ((int)smem > smem_optin()) return cudaErrorInvalidValue;
   const int ntiles = p.batch * p.tiles_m * p.tiles_n;
   const int grid = ntiles < sm_count() ? ntiles : sm_count();
   kern<<<grid, NT, smem, s>>>(ma, mb, p);
@@ -490,9 +565,9 @@ cudaError_t tc_gemm_btp_split(const bf16* Bs, const bf16* Ps, float* R, int coun
   return e;
 }
 
-cudaError_t tc_gram(const bf16* Xs, float* W, int count, int64_t m, int64_t r, int32_t* flags,
-                    int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s, int* nlaunch,
-                    bool* done) {
+cudaError_t tc_gram(const bf16* Xs, float* W, bf16* Ws, int count, int64_t m, int64_t r,
+                    int32_t* flags, int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s,
+                    int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
@@ -510,6 +585,7 @@ cudaError_t tc_gram(const bf16* Xs, float* W, int count, int64_t m, int64_t r, i
   p.num_kb = (int)((m + BK - 1) / BK);
   p.idesc = idesc_bf16(BM, bn, true, true);
   p.C = W; p.ldc = r; p.c_bs = r * r;
+  p.Cs = Ws; p.cs_stride = (int64_t)count * r * r;
   p.flags = flags; p.need_mask = need; p.skip_mask = skip;
   p.lower_only = bn == BM;
   p.max_spins = max_spins;
@@ -539,8 +615,53 @@ cudaError_t tc_apply(const bf16* Xs, const bf16* Ls, float* Y, bf16* Ys, int cou
   p.C = Y; p.ldc = r; p.c_bs = m * r;
   p.Cs = Ys; p.cs_stride = (int64_t)count * m * r;
   p.flags = flags; p.need_mask = need; p.skip_mask = skip;
+  p.kr = TC_KR_B_LOWER_NK;  // L^-1 is lower triangular: column tile j needs k <= j only
   p.max_spins = max_spins;
   cudaError_t e = launch_gemm<false, false, 3>(ma, mb, p, s);
+  if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
+  return e;
+}
+
+cudaError_t tc_block_gemm(const TcBlockGemm& g, int count, int64_t r, int32_t* flags,
+                          int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s,
+                          int* nlaunch, bool* done) {
+  using namespace tc;
+  *nlaunch = 0;
+  *done = false;
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0 || (g.N % 16) != 0 || (g.accumulate && !g.C) ||
+      (!g.C && !g.Cs))
+    return cudaErrorInvalidValue;
+  // whole 64-wide atoms for an MN-major B; 16-column granules otherwise
+  const int bn = g.b_mn ? (g.N <= 64 ? 64 : 128) : (g.N <= 128 ? (int)g.N : 128);
+  const uint64_t z = 3 * (uint64_t)count, rr = (uint64_t)r * r;
+  CUtensorMap ma, mb;
+  const bool ok =
+      (g.a_mn ? map3d_block(&ma, g.A, g.M, g.K, z, r, rr, 64, BK)
+              : map3d_block(&ma, g.A, g.K, g.M, z, r, rr, BK, BM)) &&
+      (g.b_mn ? map3d_block(&mb, g.B, g.N, g.K, z, r, rr, 64, BK)
+              : map3d_block(&mb, g.B, g.K, g.N, z, r, rr, BK, bn));
+  if (!ok) return cudaSuccess;
+  GemmP p{};
+  p.M = g.M; p.N = g.N; p.K = g.K;
+  p.batch = count;
+  p.block_n = bn;
+  p.tiles_m = (int)((g.M + BM - 1) / BM);
+  p.tiles_n = (int)((g.N + bn - 1) / bn);
+  p.num_kb = (int)((g.K + BK - 1) / BK);
+  p.idesc = idesc_bf16(BM, bn, g.a_mn, g.b_mn);
+  p.C = g.C; p.ldc = r; p.c_bs = r * r;
+  p.Cs = g.Cs; p.cs_stride = (int64_t)count * r * r;
+  p.flags = flags; p.need_mask = need; p.skip_mask = skip;
+  p.lower_only = g.lower_only && bn == BM;
+  p.epi = g.accumulate ? 2 : 1;
+  p.alpha = g.alpha;
+  p.kr = g.kr;
+  p.max_spins = max_spins;
+  cudaError_t e;
+  if (g.a_mn && g.b_mn) e = launch_gemm<true, true, 3>(ma, mb, p, s);
+  else if (g.a_mn) e = launch_gemm<true, false, 3>(ma, mb, p, s);
+  else if (g.b_mn) e = launch_gemm<false, true, 3>(ma, mb, p, s);
+  else e = launch_gemm<false, false, 3>(ma, mb, p, s);
   if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
   return e;
 }

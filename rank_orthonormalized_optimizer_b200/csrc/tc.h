@@ -46,14 +46,48 @@ cudaError_t tc_gemm_btp_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Ps, 
 
 // W[b] (r x r, fp32) = X[b]^T X[b] from the three-way split Xs ([3][count][m][r] bf16),
 // six split products; matrices failing (flags & need) == need && !(flags & skip) skipped.
-cudaError_t tc_gram(const __nv_bfloat16* Xs, float* W, int count, int64_t m, int64_t r,
-                    int32_t* flags, int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s,
-                    int* nlaunch, bool* done);
+// Only the 128 x 128 tiles on and below the diagonal are written (r > 64), and, when Ws
+// is not null, their split ([3][count][r][r]) as well.
+cudaError_t tc_gram(const __nv_bfloat16* Xs, float* W, __nv_bfloat16* Ws, int count, int64_t m,
+                    int64_t r, int32_t* flags, int32_t need, int32_t skip, int64_t max_spins,
+                    cudaStream_t s, int* nlaunch, bool* done);
 // Y[b] (m x r, fp32) = X[b] L[b]^T from the splits Xs ([3][count][m][r]) and Ls
-// ([3][count][r][r], L lower triangular), optionally writing Y's split to Ys.
+// ([3][count][r][r], L lower triangular), optionally writing Y's split to Ys.  Column
+// tile j reads L[j][k] for k below the end of its 128-wide window only: the entries of
+// L above the diagonal inside that window must be zero, those further right are not read.
 cudaError_t tc_apply(const __nv_bfloat16* Xs, const __nv_bfloat16* Ls, float* Y,
                      __nv_bfloat16* Ys, int count, int64_t m, int64_t r, int32_t* flags,
                      int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s, int* nlaunch,
                      bool* done);
+
+// Triangular operands: K blocks that can only multiply zeros are skipped.
+enum {
+  TC_KR_B_LOWER_NK = 1,  // B stored [N][K], B[j][k] = 0 for k > j
+  TC_KR_B_LOWER_KN = 2,  // B stored [K][N], B[k][j] = 0 for k < j
+  TC_KR_A_LOWER_MK = 4,  // A stored [M][K], A[i][k] = 0 for k > i
+};
+
+// One product on blocks of a stack of r x r matrices (rows r elements apart, matrices
+// r * r apart; operands are three-way bf16 splits [3][count][r][r], pointers at the
+// block origin of part 0):  C = alpha op(A) op(B)  or  C += alpha op(A) op(B).
+// a_mn: A is stored transposed ([K][M]); b_mn: B is stored [K][N] (else [N][K]).
+// C (fp32, may be null unless accumulating) and Cs (its split, may be null) are block
+// origins in stacks of the same geometry.  N must be a multiple of 16.
+struct TcBlockGemm {
+  const __nv_bfloat16* A;
+  bool a_mn;
+  const __nv_bfloat16* B;
+  bool b_mn;
+  int64_t M, N, K;
+  float* C;
+  __nv_bfloat16* Cs;
+  float alpha;
+  bool accumulate;
+  int kr;           // TC_KR_* bits
+  bool lower_only;  // only 128 x 128 tiles on or below the block's diagonal
+};
+cudaError_t tc_block_gemm(const TcBlockGemm& g, int count, int64_t r, int32_t* flags,
+                          int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s,
+                          int* nlaunch, bool* done);
 
 }  // namespace dion

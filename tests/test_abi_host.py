@@ -113,6 +113,20 @@ def test_workspace_covers_the_layout():
     dion.dion_free(h)
 
 
+def test_workspace_recursive_factorisation_scratch():
+    # r > 256 on the tensor path: two more [3][count][r][r] bf16 splits (the Gram's and
+    # L21's) for the recursive Cholesky factorisation; none at r <= 256, none on the
+    # CUDA-core path (bf16 GEMM inputs: the two plans differ in nothing else)
+    def ws_of(r, path):
+        c, h, ws = _init([(8, 1024, 1024, r)], kernel_path=path)
+        assert c == dion.OK
+        dion.dion_free(h)
+        return ws
+
+    assert ws_of(512, 0) - ws_of(512, 1) == 2 * 8 * 512 * 512 * 6
+    assert ws_of(256, 0) == ws_of(256, 1)
+
+
 def test_step_argument_checks_without_device():
     c, h, ws = _init([(2, 256, 128, 32)])
     assert c == dion.OK

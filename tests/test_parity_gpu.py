@@ -121,6 +121,9 @@ EDGE = [
     ("full_rank_square", [(2, 64, 64, 64)]),
     ("wide", [(2, 48, 520, 32)]),
     ("many_small", [(300, 32, 16, 16)]),
+    # r > 256: the recursive factorisation, with a last block of 16 (272 = 256 + 16;
+    # 784 = 512 + 272) and row counts that are not multiples of the 128-row tiles
+    ("recursive_chol", [(2, 600, 560, 272), (2, 1100, 800, 784)]),
 ]
 
 
@@ -144,6 +147,71 @@ def test_orth_modes(mode, bit):
     st = run.status.cpu().numpy()
     if bit:
         assert np.all(st & bit), st
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_rank_deficient_large_r_falls_back(precision):
+    """r = 320 > 256 (recursive factorisation).  Slot 0 gets B of rank 64 < r: in fp32
+    its Gram is singular to working precision, the factorisation fails a pivot or the
+    diagonal-ratio test, and the matrix goes to Householder QR (bf16 rounding of B
+    makes it full rank with small singular values, so there the route is not fixed).
+    Its P is not unique (only col(B) is fixed), so the check is the invariants:
+    P^T P = I and B - P P^T B = 0 (to the rounding of B in bf16).  Slot 1 gets a
+    full-rank Gaussian B in the same bucket and must match the oracle's step."""
+    m, n, r, k = 512, 384, 320, 64
+    wl = W.custom("lowrank_r320", [(2, m, n, r)], precision=precision, steps=1)
+    run = GpuRun(wl)
+    X0, Q0 = run.X[0].clone(), run.Q[0].clone()
+    g = torch.Generator().manual_seed(5)
+    U = torch.linalg.qr(torch.randn(m, k, generator=g, dtype=torch.float64))[0]
+    V = torch.linalg.qr(torch.randn(n, k, generator=g, dtype=torch.float64))[0]
+    G = torch.stack([U @ V.T, torch.randn(m, n, generator=g, dtype=torch.float64)]).float()
+    run.step(1, G_override=[G.cuda()])
+    st = run.status.cpu().numpy()
+    assert not st[1] & 1, st
+    if precision == "fp32":
+        assert st[0] & 1, st
+    assert not np.any(st & (4 | 8)), st
+    assert run.orth_error() <= ORTH_TOL
+    P = run.P(0)[0].double().cpu()
+    B = G[0].double()
+    res = B - P @ (P.T @ B)
+    assert (res.norm() / B.norm()).item() <= (1e-5 if precision == "fp32" else 1e-2)
+    X, M, Q, _, _ = oracle.dion_step(X0[1].cpu().numpy(), np.zeros((m, n)), G[1].numpy(),
+                                     Q0[1].cpu().numpy(), wl.mu, wl.lr)
+    tol = TOL[precision]
+    assert oracle.rel_fro(run.X[0][1].double().cpu().numpy(), X) <= tol
+    assert oracle.rel_fro(run.M[0][1].double().cpu().numpy(), M) <= tol
+
+
+def test_shifted_iteration_recovers_qr_of_ill_conditioned_p0():
+    """r = 384 > 256 and cond(P0) ~ 1e5: Cholesky-QR fails its diagonal-ratio test and the
+    shifted Cholesky-QR iteration (not Householder) produces P.  Whatever route, P must
+    be P0's Q factor: P^T P = I, and R = P^T P0 upper triangular with a positive
+    diagonal, P0 = P R.  These hold to rounding whatever the conditioning (the entries of
+    P itself do not: they move by up to cond(P0) u)."""
+    m, n, r = 640, 512, 384
+    wl = W.custom("illcond_r384", [(2, m, n, r)], precision="fp32", steps=1)
+    run = GpuRun(wl)
+    Q0 = run.Q[0].double().cpu()
+    g = torch.Generator().manual_seed(11)
+    U = torch.linalg.qr(torch.randn(2, m, n, generator=g, dtype=torch.float64))[0]
+    V = torch.linalg.qr(torch.randn(2, n, n, generator=g, dtype=torch.float64))[0]
+    sig = torch.logspace(0, -5, n, dtype=torch.float64)
+    B = (U * sig) @ V.transpose(1, 2)
+    run.step(1, G_override=[B.float().cuda()])
+    st = run.status.cpu().numpy()
+    assert np.all(st & 1) and not np.any(st & (4 | 8)), st
+    assert run.orth_error() <= ORTH_TOL
+    P = run.P(0).double().cpu()
+    P0 = B.float().double() @ Q0
+    R = P.transpose(1, 2) @ P0
+    for i in range(2):
+        scale = torch.linalg.norm(P0[i])
+        # both at the level of P's own orthogonality error (<= orth_tol = 2e-5 at exit)
+        assert torch.linalg.norm(torch.tril(R[i], -1)) / scale <= 1e-4
+        assert torch.all(torch.diagonal(R[i]) > 0)
+        assert torch.linalg.norm(P0[i] - P[i] @ torch.triu(R[i])) / scale <= 1e-4
 
 
 def test_update_norm_is_lr_s_sqrt_r():
