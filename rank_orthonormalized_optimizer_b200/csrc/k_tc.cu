@@ -31,6 +31,7 @@ namespace dion {
 namespace tc {
 
 constexpr int BM = 128;       // tile rows = TMEM lanes
+constexpr int KCHUNK_SUMSQ = 8;  // K blocks per accumulation chunk of sums of squares
 constexpr int BK = 64;        // bf16 elements per 128-byte swizzle row
 constexpr int NT = 256;       // threads per CTA
 constexpr int UPD_BN = 128;   // update tile columns (acc uses 2 * UPD_BN TMEM columns)
@@ -179,8 +180,19 @@ struct GemmP {
   int epi;                           // 0: C = acc;  1: C = alpha acc;  2: C += alpha acc
   float alpha;
   int kr;                            // triangular-operand K ranges (TC_KR_* bits)
+  int kchunk;                        // K blocks per accumulation chunk (0: one chunk)
   int64_t max_spins;
 };
+
+// The tensor cores add each MMA's products into the fp32 accumulator with a rounding
+// that is biased (toward zero): over thousands of MMAs the bias grows with K and, for
+// sums of like-signed terms such as the diagonal of a Gram matrix, it does not average
+// out (about 2.5e-5 relative at K = 4096 with six split products per step).  Long K
+// ranges are therefore cut into chunks of kchunk blocks, each accumulated from zero in
+// TMEM, and the epilogue adds the chunks in fp32 registers (round to nearest) into C.
+__device__ __forceinline__ int n_chunks(const GemmP& p, int kb0, int kb1) {
+  return p.kchunk > 0 ? (kb1 - kb0 + p.kchunk - 1) / p.kchunk : 1;
+}
 
 // K blocks [kb0, kb1) that can hold non-zero products for the tile at (m0, n0) when an
 // operand is lower triangular (entries past the diagonal are zero and are not read).
@@ -306,18 +318,22 @@ __global__ void __launch_bounds__(NT, 1)
     int stage = 0;
     uint32_t phase = 0;
     int lt = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
       if (!tile_active(p, t, tiles_per_mat)) continue;
-      const int acc = lt & 1;
-      const uint32_t acc_phase = (lt >> 1) & 1;
-      if (!wait_bounded(tempty + acc, acc_phase ^ 1, p.max_spins, abort)) break;
-      tc_fence_after();
-      const uint32_t d = tmem + acc * p.acc_stride;
       const int rem = t % tiles_per_mat;
       int kb0, kb1;
       k_range(p, (rem / p.tiles_n) * BM, (rem % p.tiles_n) * p.block_n, kb0, kb1);
-      bool ok = true;
-      for (int kb = kb0; kb < kb1; ++kb) {
+      const int nch = n_chunks(p, kb0, kb1);
+      for (int ch = 0; ch < nch && ok; ++ch) {
+      const int acc = lt & 1;
+      const uint32_t acc_phase = (lt >> 1) & 1;
+      if (!wait_bounded(tempty + acc, acc_phase ^ 1, p.max_spins, abort)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d = tmem + acc * p.acc_stride;
+      const int c0 = p.kchunk > 0 ? kb0 + ch * p.kchunk : kb0;
+      const int c1 = p.kchunk > 0 ? min(kb1, c0 + p.kchunk) : kb1;
+      for (int kb = c0; kb < c1; ++kb) {
         if (!wait_bounded(full + stage, phase, p.max_spins, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_base = smem_u32(sA + (size_t)stage * stage_a);
@@ -332,7 +348,7 @@ __global__ void __launch_bounds__(NT, 1)
                                      : sw128_desc(ab + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? sw128_desc(bb + k * 2048, 8192, 1024)
                                      : sw128_desc(bb + k * 32, 16, 1024);
-            mma_bf16(d, ad, bd, p.idesc, ((kb - kb0) | k | q) != 0);
+            mma_bf16(d, ad, bd, p.idesc, ((kb - c0) | k | q) != 0);
           }
         }
         mma_commit(empty + stage);
@@ -341,71 +357,84 @@ __global__ void __launch_bounds__(NT, 1)
       if (!ok) break;
       mma_commit(tfull + acc);
       ++lt;
+      }
     }
     mma_commit(drain);
     wait_drain(drain, 0);
   } else if (warp >= 4) {
     // ---------------- epilogue: TMEM -> registers -> global (fp32 and/or bf16 split)
+    // chunk 0 stores (or accumulates when p.epi == 2); later chunks of the tile add into
+    // C; the split Cs is written from the final value, after the last chunk
     const int ew = warp - 4;
     int lt = 0;
     int t = blockIdx.x;
+    bool ok = true;
     for (; t < ntiles; t += gridDim.x) {
       if (!tile_active(p, t, tiles_per_mat)) continue;
       const int b = t / tiles_per_mat;
-      const int acc = lt & 1;
-      const uint32_t acc_phase = (lt >> 1) & 1;
-      if (!wait_bounded(tfull + acc, acc_phase, p.max_spins, abort)) break;
-      tc_fence_after();
       const int rem = t % tiles_per_mat;
       const int64_t row = (int64_t)(rem / p.tiles_n) * BM + ew * 32 + lane;
       const int64_t n0 = (int64_t)(rem % p.tiles_n) * p.block_n;
       const int64_t off = (int64_t)b * p.c_bs + row * p.ldc;
-      const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * p.acc_stride;
-      for (int c = 0; c < p.block_n; c += 16) {
-        float v[16];
-        tmem_ld16(tbase + c, v);
-        tmem_wait_ld();
-        if (row < p.M && n0 + c < p.N) {
-          if (p.epi != 0) {
-            float old[16];
-            if (p.epi == 2) {
-              const float4* src = reinterpret_cast<const float4*>(p.C + off + n0 + c);
+      int kb0, kb1;
+      k_range(p, (rem / p.tiles_n) * BM, (int)n0, kb0, kb1);
+      const int nch = n_chunks(p, kb0, kb1);
+      for (int ch = 0; ch < nch; ++ch) {
+        const int acc = lt & 1;
+        const uint32_t acc_phase = (lt >> 1) & 1;
+        if (!wait_bounded(tfull + acc, acc_phase, p.max_spins, abort)) { ok = false; break; }
+        tc_fence_after();
+        const int epi = ch == 0 ? p.epi : 2;
+        const float alpha = p.epi == 0 ? 1.f : p.alpha;
+        const bool last = ch == nch - 1;
+        const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * p.acc_stride;
+        for (int c = 0; c < p.block_n; c += 16) {
+          float v[16];
+          tmem_ld16(tbase + c, v);
+          tmem_wait_ld();
+          if (row < p.M && n0 + c < p.N) {
+            if (epi != 0) {
+              float old[16];
+              if (epi == 2) {
+                const float4* src = reinterpret_cast<const float4*>(p.C + off + n0 + c);
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const float4 o4 = src[q];
-                old[4 * q] = o4.x; old[4 * q + 1] = o4.y; old[4 * q + 2] = o4.z; old[4 * q + 3] = o4.w;
+                for (int q = 0; q < 4; ++q) {
+                  const float4 o4 = src[q];
+                  old[4 * q] = o4.x; old[4 * q + 1] = o4.y; old[4 * q + 2] = o4.z; old[4 * q + 3] = o4.w;
+                }
               }
+#pragma unroll
+              for (int q = 0; q < 16; ++q) v[q] = epi == 2 ? fmaf(alpha, v[q], old[q]) : alpha * v[q];
             }
+            if (p.C) {
+              float4* dst = reinterpret_cast<float4*>(p.C + off + n0 + c);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) v[q] = p.epi == 2 ? fmaf(p.alpha, v[q], old[q]) : p.alpha * v[q];
-          }
-          if (p.C) {
-            float4* dst = reinterpret_cast<float4*>(p.C + off + n0 + c);
+              for (int q = 0; q < 4; ++q)
+                dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            }
+            if (p.Cs && last) {
+              __align__(16) bf16 h[16], mi[16], lo[16];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          }
-          if (p.Cs) {
-            __align__(16) bf16 h[16], mi[16], lo[16];
-#pragma unroll
-            for (int q = 0; q < 16; ++q) split3_bf16(v[q], h[q], mi[q], lo[q]);
-            bf16* base = p.Cs + off + n0 + c;
-            uint4* d0 = reinterpret_cast<uint4*>(base);
-            uint4* d1 = reinterpret_cast<uint4*>(base + p.cs_stride);
-            uint4* d2 = reinterpret_cast<uint4*>(base + 2 * p.cs_stride);
-            const uint4* sh = reinterpret_cast<const uint4*>(h);
-            const uint4* sm = reinterpret_cast<const uint4*>(mi);
-            const uint4* sl = reinterpret_cast<const uint4*>(lo);
-            d0[0] = sh[0]; d0[1] = sh[1];
-            d1[0] = sm[0]; d1[1] = sm[1];
-            d2[0] = sl[0]; d2[1] = sl[1];
+              for (int q = 0; q < 16; ++q) split3_bf16(v[q], h[q], mi[q], lo[q]);
+              bf16* base = p.Cs + off + n0 + c;
+              uint4* d0 = reinterpret_cast<uint4*>(base);
+              uint4* d1 = reinterpret_cast<uint4*>(base + p.cs_stride);
+              uint4* d2 = reinterpret_cast<uint4*>(base + 2 * p.cs_stride);
+              const uint4* sh = reinterpret_cast<const uint4*>(h);
+              const uint4* sm = reinterpret_cast<const uint4*>(mi);
+              const uint4* sl = reinterpret_cast<const uint4*>(lo);
+              d0[0] = sh[0]; d0[1] = sh[1];
+              d1[0] = sm[0]; d1[1] = sm[1];
+              d2[0] = sl[0]; d2[1] = sl[1];
+            }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty + acc);
+        ++lt;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty + acc);
-      ++lt;
+      if (!ok) break;
     }
     if (t < ntiles && lane == 0) mark_unfinished(p.flags, t, ntiles, tiles_per_mat, gridDim.x);
   }
@@ -588,6 +617,7 @@ cudaError_t tc_gram(const bf16* Xs, float* W, bf16* Ws, int count, int64_t m, in
   p.Cs = Ws; p.cs_stride = (int64_t)count * r * r;
   p.flags = flags; p.need_mask = need; p.skip_mask = skip;
   p.lower_only = bn == BM;
+  p.kchunk = KCHUNK_SUMSQ;  // the diagonal sums squares: keep the accumulation unbiased
   p.max_spins = max_spins;
   cudaError_t e = launch_gemm<true, true, 3>(ma, mb, p, s);
   if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
@@ -656,6 +686,7 @@ cudaError_t tc_block_gemm(const TcBlockGemm& g, int count, int64_t r, int32_t* f
   p.epi = g.accumulate ? 2 : 1;
   p.alpha = g.alpha;
   p.kr = g.kr;
+  if (g.accumulate) p.kchunk = KCHUNK_SUMSQ;  // W22 -= L21 L21^T: squares on the diagonal
   p.max_spins = max_spins;
   cudaError_t e;
   if (g.a_mn && g.b_mn) e = launch_gemm<true, true, 3>(ma, mb, p, s);
