@@ -185,7 +185,7 @@ dion_status fb_iteration(const Plan& p, const dion_options& o, const FbBufs& f,
   if (e != cudaSuccess || !done)
     return fail(DION_ERR_CUDA, "shifted iteration, factorisation (%s): %s", what,
                 e != cudaSuccess ? cudaGetErrorString(e) : dion::tc_map_error());
-  e = dion::tc_apply(src, f.Linvs, f.P, dst, p.count, p.m, p.r, f.flags, need, skip,
+  e = dion::tc_apply(src, f.Linvs, f.P, dst, nullptr, p.count, p.m, p.r, f.flags, need, skip,
                      o.max_wait_spins, s, &nl, &done);
   if (e != cudaSuccess || !done)
     return fail(DION_ERR_CUDA, "shifted iteration, apply: %s",
@@ -408,6 +408,7 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
   if (phase == PH_ORTH) {
   begin_cls(c, DION_KCLASS_ORTH);
   {
+    bool pg_ready = false;  // Pg already holds the first pass's P
     auto gram = [&](const float* src) {
       dion::GemmDesc d{};
       d.A = {src, m * r, 1, r};
@@ -468,17 +469,22 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
       if ((st = tc_check(e, "tc_gram")) != DION_OK) return st;
       ca.pass = 1; ca.orth_tol = o.orth_tol;
       if ((st = chol()) != DION_OK) return st;
-      e = dion::tc_apply(P0s, Linvs, P, Ps, cnt, m, r, flags, 0, DION_MAT_FALLBACK,
-                         o.max_wait_spins, s, &nl, &done);
+      // the first pass writes P and its GEMM copy Pg at once (in split mode Pg is the
+      // split the second pass reads); the finalize then touches only the matrices that
+      // took the second pass or the fallback
+      __nv_bfloat16* P1s = split ? reinterpret_cast<__nv_bfloat16*>(Pg) : Ps;
+      e = dion::tc_apply(P0s, Linvs, P, P1s, bf ? reinterpret_cast<__nv_bfloat16*>(Pg) : nullptr,
+                         cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s, &nl, &done);
       if ((st = tc_check(e, "tc_apply")) != DION_OK) return st;
+      pg_ready = true;
       if (o.orth_mode != DION_ORTH_CHOLQR) {
-        e = dion::tc_gram(Ps, W, Ws, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s,
+        e = dion::tc_gram(P1s, W, Ws, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s,
                           &nl, &done);
         if ((st = tc_check(e, "tc_gram")) != DION_OK) return st;
         ca.pass = 2;
         ca.orth_tol = o.orth_mode == DION_ORTH_CHOLQR2 ? -1.f : o.orth_tol;
         if ((st = chol()) != DION_OK) return st;
-        e = dion::tc_apply(Ps, Linvs, P2, nullptr, cnt, m, r, flags, DION_MAT_CHOLQR2,
+        e = dion::tc_apply(P1s, Linvs, P2, nullptr, nullptr, cnt, m, r, flags, DION_MAT_CHOLQR2,
                            DION_MAT_FALLBACK, o.max_wait_spins, s, &nl, &done);
         if ((st = tc_check(e, "tc_apply")) != DION_OK) return st;
       }
@@ -507,7 +513,7 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     DION_LAUNCH(c, 1, dion::launch_householder(P0, p0s_ready ? P0s : nullptr, P2, P0, P, flags,
                                                cnt, m, r, s));
     DION_LAUNCH(c, 1, dion::launch_finalize_p(P2, Pg, bf ? 1 : (split ? 2 : 0), flags, cnt, m, r,
-                                              P, s));
+                                              P, pg_ready, s));
   }
   end_cls(c);
   return DION_OK;
@@ -521,14 +527,16 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     if (split) {
       int nl = 0;
       cudaError_t e = dion::tc_gemm_btp_split((const __nv_bfloat16*)Bg, (const __nv_bfloat16*)Pg, R,
-                                              cnt, m, n, r, o.max_wait_spins, flags, s, &nl, &done);
+                                              part, cnt, m, n, r, o.max_wait_spins, flags, s, &nl,
+                                              &done);
       c.launches += nl;
       if (e != cudaSuccess)
         return fail(DION_ERR_CUDA, "tc_gemm_btp_split: %s", cudaGetErrorString(e));
       if (!done) return fail(DION_ERR_CUDA, "tc_gemm_btp_split: %s", dion::tc_map_error());
     } else if (tensor && bf) {
       int nl = 0;
-      cudaError_t e = dion::tc_gemm_btp(Bg, Pg, R, cnt, m, n, r, o.max_wait_spins, flags, s, &nl, &done);
+      cudaError_t e = dion::tc_gemm_btp(Bg, Pg, R, part, cnt, m, n, r, o.max_wait_spins, flags, s,
+                                        &nl, &done);
       c.launches += nl;
       if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_gemm_btp: %s", cudaGetErrorString(e));
       if (!done) return fail(DION_ERR_CUDA, "tc_gemm_btp: %s", dion::tc_map_error());
@@ -549,8 +557,9 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
   // step 6: Q = colnorm(R), plus the GEMM copies of R and Q for the update
   if (phase == PH_COLNORM) {
   begin_cls(c, DION_KCLASS_COLNORM);
-  DION_LAUNCH(c, 2, dion::launch_colnorm(R, bp.Q, Rg, Qng, bf ? 1 : (split ? 2 : 0), part,
-                                         p.nsplit, flags, cnt, n, r, s));
+  DION_LAUNCH(c, 2,
+              dion::launch_colnorm(R, bp.Q, Rg, Qng, bf ? 1 : (split ? 2 : 0), part, p.nsplit,
+                                   tensor, flags, cnt, n, r, s));
   end_cls(c);
   return DION_OK;
   }
@@ -733,7 +742,9 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
     p.scale = d.scale > 0.f ? d.scale : (float)std::sqrt((double)d.m / (double)d.n);
     p.mat0 = mats;
     mats += d.count;
-    p.nsplit = dion::colnorm_splits(d.count, d.n);
+    // column-norm partials: on the tensor path B^T P writes one per 32 rows of R
+    p.nsplit = o.kernel_path == DION_PATH_TENSOR ? (int)(4 * ((d.n + 127) / 128))
+                                                 : dion::colnorm_splits(d.count, d.n);
     const size_t c = (size_t)d.count;
     p.off_Bg = take(c * d.m * d.n * ge);
     p.off_Qg = take(c * d.n * d.r * ge);

@@ -49,14 +49,18 @@ cudaError_t launch_prep_q_split(const float* Q, void* Qs, int count, int64_t n, 
 // tile counters of the bucket's dynamically scheduled kernels.
 cudaError_t launch_init_flags(int32_t* flags, float* stats, int* sched, int count,
                               int32_t init_bits, cudaStream_t s);
-// mode 0: fp32 P only; 1: + bf16 copy Pg; 2: + three-way bf16 split Pg
+// mode 0: fp32 P only; 1: + bf16 copy Pg; 2: + three-way bf16 split Pg.  pg_ready: Pg
+// already holds the first pass's P; only second-pass and fallback matrices are written.
 cudaError_t launch_finalize_p(const float* P2, void* Pg, int mode, const int32_t* flags,
-                              int count, int64_t m, int64_t r, float* P, cudaStream_t s);
+                              int count, int64_t m, int64_t r, float* P, bool pg_ready,
+                              cudaStream_t s);
 int colnorm_splits(int count, int64_t n);
-// mode 0: Q only; 1: + bf16 R, Q; 2: + three-way bf16 splits of R, Q
+// mode 0: Q only; 1: + bf16 R, Q; 2: + three-way bf16 splits of R, Q.  part holds nsplit
+// partial column sums of squares per matrix ([count][nsplit][r]); part_ready: B^T P wrote
+// them already (else a first kernel does, over nsplit row ranges).
 cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, int mode,
-                           float* part, int nsplit, int32_t* flags, int count, int64_t n,
-                           int64_t r, cudaStream_t s);
+                           float* part, int nsplit, bool part_ready, int32_t* flags, int count,
+                           int64_t n, int64_t r, cudaStream_t s);
 cudaError_t launch_split3(const float* src, void* dst, int64_t n, int64_t dst_stride,
                           cudaStream_t s);
 cudaError_t launch_write_status(const int32_t* flags, int32_t* d_status, int count,

@@ -231,17 +231,20 @@ cudaError_t launch_write_status(const int32_t* flags, int32_t* d_status, int cou
 }
 
 // ------------------------------------------------------------- final P
-// P holds the first Cholesky-QR pass or the Householder result; P2 the
+// P holds the first Cholesky-QR pass or the fallback's result; P2 the
 // second pass.  Picks per matrix, then writes the GEMM copy Pg (bf16 mode).
+// pg_ready: the first pass already wrote Pg, so only matrices that took the second
+// pass or the fallback are touched.
 // MODE 0: fp32 only; 1: + bf16 copy; 2: + three-way bf16 split (planes of count*m*r)
 template <int MODE>
 __global__ void k_finalize_p(float* __restrict__ P, const float* __restrict__ P2,
                              void* __restrict__ Pg, const int32_t* __restrict__ flags,
-                             int64_t mr4, int64_t plane) {
+                             int64_t mr4, int64_t plane, int pg_ready) {
   const int64_t b = blockIdx.y;
   const int32_t f = flags[b];
   const bool take2 = (f & F_CHOLQR2) && !(f & F_FALLBACK);
   if (!take2 && MODE == 0) return;
+  if (pg_ready && !take2 && !(f & F_FALLBACK)) return;
   float4* p = reinterpret_cast<float4*>(P) + b * mr4;
   const float4* p2 = reinterpret_cast<const float4*>(P2) + b * mr4;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < mr4;
@@ -269,18 +272,19 @@ __global__ void k_finalize_p(float* __restrict__ P, const float* __restrict__ P2
 }
 
 cudaError_t launch_finalize_p(const float* P2, void* Pg, int mode, const int32_t* flags,
-                              int count, int64_t m, int64_t r, float* P, cudaStream_t s) {
+                              int count, int64_t m, int64_t r, float* P, bool pg_ready,
+                              cudaStream_t s) {
   const int64_t mr4 = m * r / 4;
   int64_t gx = (mr4 + 255) / 256;
   if (gx > 64) gx = 64;
   dim3 grid((unsigned)gx, (unsigned)count);
   const int64_t plane = (int64_t)count * m * r;
   if (mode == 2)
-    k_finalize_p<2><<<grid, 256, 0, s>>>(P, P2, Pg, flags, mr4, plane);
+    k_finalize_p<2><<<grid, 256, 0, s>>>(P, P2, Pg, flags, mr4, plane, pg_ready ? 1 : 0);
   else if (mode == 1)
-    k_finalize_p<1><<<grid, 256, 0, s>>>(P, P2, Pg, flags, mr4, plane);
+    k_finalize_p<1><<<grid, 256, 0, s>>>(P, P2, Pg, flags, mr4, plane, pg_ready ? 1 : 0);
   else
-    k_finalize_p<0><<<grid, 256, 0, s>>>(P, P2, Pg, flags, mr4, plane);
+    k_finalize_p<0><<<grid, 256, 0, s>>>(P, P2, Pg, flags, mr4, plane, 0);
   return cudaGetLastError();
 }
 
@@ -330,6 +334,19 @@ __global__ void __launch_bounds__(256) k_colnorm_partial(const float* __restrict
   }
 }
 
+// Many partials (one per 32 rows of R, from B^T P): add them once per column, in
+// row-block order, into partial 0, so that the apply kernel's blocks read one value.
+__global__ void __launch_bounds__(256) k_colnorm_fold(float* __restrict__ part, int64_t r,
+                                                       int nsplit) {
+  const int64_t b = blockIdx.y;
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= r) return;
+  float* pb = part + b * nsplit * r;
+  float ss = 0.f;
+  for (int s2 = 0; s2 < nsplit; ++s2) ss += pb[s2 * r + j];
+  pb[j] = ss;
+}
+
 // MODE 0: Q only; 1: + bf16 R and Q; 2: + three-way bf16 splits of R and Q
 template <int MODE>
 __global__ void __launch_bounds__(256) k_colnorm_apply(const float* __restrict__ R,
@@ -338,14 +355,14 @@ __global__ void __launch_bounds__(256) k_colnorm_apply(const float* __restrict__
                                                         void* __restrict__ Qg,
                                                         const float* __restrict__ part,
                                                         int32_t* __restrict__ flags, int64_t n,
-                                                        int64_t r, int nsplit,
+                                                        int64_t r, int nsplit, int64_t part_bs,
                                                         int64_t rows_per_block) {
   extern __shared__ float norm_s[];  // r floats
   const int64_t b = blockIdx.y;
   bool zero = false;
   for (int64_t j = threadIdx.x; j < r; j += blockDim.x) {
     float ss = 0.f;
-    for (int s2 = 0; s2 < nsplit; ++s2) ss += part[(b * nsplit + s2) * r + j];
+    for (int s2 = 0; s2 < nsplit; ++s2) ss += part[b * part_bs + s2 * r + j];
     const float nrm = sqrtf(ss);
     norm_s[j] = nrm;
     zero |= !(nrm > 0.f);
@@ -407,12 +424,19 @@ int colnorm_splits(int count, int64_t n) {
 }
 
 cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, int mode, float* part,
-                           int nsplit, int32_t* flags, int count, int64_t n, int64_t r,
-                           cudaStream_t s) {
+                           int nsplit, bool part_ready, int32_t* flags, int count, int64_t n,
+                           int64_t r, cudaStream_t s) {
   const int64_t vc = r / 4;
-  const size_t red_bytes = (size_t)(vc >= 256 ? 256 : 256 / vc * vc) * sizeof(float4);
-  k_colnorm_partial<<<dim3((unsigned)nsplit, (unsigned)count), 256, red_bytes, s>>>(R, part, n, r,
-                                                                                  nsplit);
+  if (!part_ready) {
+    const size_t red_bytes = (size_t)(vc >= 256 ? 256 : 256 / vc * vc) * sizeof(float4);
+    k_colnorm_partial<<<dim3((unsigned)nsplit, (unsigned)count), 256, red_bytes, s>>>(R, part, n,
+                                                                                    r, nsplit);
+  } else {
+    k_colnorm_fold<<<dim3((unsigned)((r + 255) / 256), (unsigned)count), 256, 0, s>>>(part, r,
+                                                                                   nsplit);
+  }
+  const int64_t part_bs = (int64_t)nsplit * r;  // partials of one matrix
+  if (part_ready) nsplit = 1;                    // folded into the first
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t target_blocks = 8 * (int64_t)sm_count();
@@ -428,11 +452,14 @@ cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, int mod
   }
   const dim3 grid((unsigned)gx, (unsigned)count);
   if (mode == 2)
-    k_colnorm_apply<2><<<grid, 256, smem, s>>>(R, Q, Rg, Qg, part, flags, n, r, nsplit, rows);
+    k_colnorm_apply<2><<<grid, 256, smem, s>>>(R, Q, Rg, Qg, part, flags, n, r, nsplit, part_bs,
+                                               rows);
   else if (mode == 1)
-    k_colnorm_apply<1><<<grid, 256, smem, s>>>(R, Q, Rg, Qg, part, flags, n, r, nsplit, rows);
+    k_colnorm_apply<1><<<grid, 256, smem, s>>>(R, Q, Rg, Qg, part, flags, n, r, nsplit, part_bs,
+                                               rows);
   else
-    k_colnorm_apply<0><<<grid, 256, smem, s>>>(R, Q, Rg, Qg, part, flags, n, r, nsplit, rows);
+    k_colnorm_apply<0><<<grid, 256, smem, s>>>(R, Q, Rg, Qg, part, flags, n, r, nsplit, part_bs,
+                                               rows);
   return cudaGetLastError();
 }
 

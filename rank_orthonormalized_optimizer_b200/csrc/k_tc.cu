@@ -174,6 +174,9 @@ struct GemmP {
   int64_t ldc, c_bs;
   bf16* Cs;                          // three-way bf16 split of the result (may be null)
   int64_t cs_stride;                 // elements between the split parts
+  bf16* Cb;                          // bf16 copy of the result (may be null)
+  float* colsq;                      // per-warp column sums of squares (may be null):
+                                     // [batch][tiles_m * 4][N], row block tm*4 + warp
   int32_t* flags;
   int32_t need_mask, skip_mask;      // matrices whose flags fail this are skipped
   int lower_only;                    // skip tiles above the diagonal (symmetric results)
@@ -392,8 +395,9 @@ __global__ void __launch_bounds__(NT, 1)
           float v[16];
           tmem_ld16(tbase + c, v);
           tmem_wait_ld();
-          if (row < p.M && n0 + c < p.N) {
-            if (epi != 0) {
+          if (n0 + c < p.N) {  // uniform across the warp
+            const bool valid = row < p.M;
+            if (valid && epi != 0) {
               float old[16];
               if (epi == 2) {
                 const float4* src = reinterpret_cast<const float4*>(p.C + off + n0 + c);
@@ -406,13 +410,21 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
               for (int q = 0; q < 16; ++q) v[q] = epi == 2 ? fmaf(alpha, v[q], old[q]) : alpha * v[q];
             }
-            if (p.C) {
+            if (valid && p.C) {
               float4* dst = reinterpret_cast<float4*>(p.C + off + n0 + c);
 #pragma unroll
               for (int q = 0; q < 4; ++q)
                 dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
             }
-            if (p.Cs && last) {
+            if (valid && p.Cb && last) {
+              __align__(16) bf16 h[16];
+#pragma unroll
+              for (int q = 0; q < 16; ++q) h[q] = __float2bfloat16_rn(v[q]);
+              uint4* d0 = reinterpret_cast<uint4*>(p.Cb + off + n0 + c);
+              d0[0] = reinterpret_cast<const uint4*>(h)[0];
+              d0[1] = reinterpret_cast<const uint4*>(h)[1];
+            }
+            if (valid && p.Cs && last) {
               __align__(16) bf16 h[16], mi[16], lo[16];
 #pragma unroll
               for (int q = 0; q < 16; ++q) split3_bf16(v[q], h[q], mi[q], lo[q]);
@@ -426,6 +438,28 @@ __global__ void __launch_bounds__(NT, 1)
               d0[0] = sh[0]; d0[1] = sh[1];
               d1[0] = sm[0]; d1[1] = sm[1];
               d2[0] = sl[0]; d2[1] = sl[1];
+            }
+            if (p.colsq && last) {
+              // the sum of squares of this warp's 32 rows for the 16 columns by a fixed
+              // butterfly (16 shuffles, every lane takes part); lane 2j ends with column
+              // j's sum, j's bits being lane bits 1..4
+              float w[16];
+#pragma unroll
+              for (int q = 0; q < 16; ++q) w[q] = valid ? v[q] * v[q] : 0.f;
+#pragma unroll
+              for (int h = 8; h >= 1; h >>= 1) {
+                const bool hi = (lane & (2 * h)) != 0;
+#pragma unroll
+                for (int j = 0; j < h; ++j) {
+                  const float recv = __shfl_xor_sync(0xffffffffu, hi ? w[j] : w[j + h], 2 * h);
+                  w[j] = (hi ? w[j + h] : w[j]) + recv;
+                }
+              }
+              w[0] += __shfl_xor_sync(0xffffffffu, w[0], 1);
+              if (!(lane & 1)) {
+                const int64_t rb = (int64_t)b * p.tiles_m * 4 + (rem / p.tiles_n) * 4 + ew;
+                p.colsq[rb * p.N + n0 + c + (lane >> 1)] = w[0];
+              }
             }
           }
         }
@@ -514,9 +548,9 @@ cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, bf16* P0s, int
   return e;
 }
 
-cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, int count, int64_t m, int64_t n,
-                        int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
-                        bool* done) {
+cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, float* colsq, int count,
+                        int64_t m, int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
+                        cudaStream_t s, int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
@@ -533,6 +567,7 @@ cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, int count, int
   p.num_kb = (int)((m + BK - 1) / BK);
   p.idesc = idesc_bf16(BM, bn, true, true);
   p.C = R; p.ldc = r; p.c_bs = n * r;
+  p.colsq = colsq;
   p.flags = flags;
   p.max_spins = max_spins;
   cudaError_t e = launch_gemm<true, true, 1>(ma, mb, p, s);
@@ -568,8 +603,8 @@ cudaError_t tc_gemm_bq_split(const bf16* Bs, const bf16* Qs, bf16* P0s, int coun
   return e;
 }
 
-cudaError_t tc_gemm_btp_split(const bf16* Bs, const bf16* Ps, float* R, int count, int64_t m,
-                              int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
+cudaError_t tc_gemm_btp_split(const bf16* Bs, const bf16* Ps, float* R, float* colsq, int count,
+                              int64_t m, int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
                               cudaStream_t s, int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
@@ -587,6 +622,7 @@ cudaError_t tc_gemm_btp_split(const bf16* Bs, const bf16* Ps, float* R, int coun
   p.num_kb = (int)((m + BK - 1) / BK);
   p.idesc = idesc_bf16(BM, bn, true, true);
   p.C = R; p.ldc = r; p.c_bs = n * r;
+  p.colsq = colsq;
   p.flags = flags;
   p.max_spins = max_spins;
   cudaError_t e = launch_gemm<true, true, 3>(ma, mb, p, s);
@@ -624,9 +660,9 @@ cudaError_t tc_gram(const bf16* Xs, float* W, bf16* Ws, int count, int64_t m, in
   return e;
 }
 
-cudaError_t tc_apply(const bf16* Xs, const bf16* Ls, float* Y, bf16* Ys, int count, int64_t m,
-                     int64_t r, int32_t* flags, int32_t need, int32_t skip, int64_t max_spins,
-                     cudaStream_t s, int* nlaunch, bool* done) {
+cudaError_t tc_apply(const bf16* Xs, const bf16* Ls, float* Y, bf16* Ys, bf16* Yb, int count,
+                     int64_t m, int64_t r, int32_t* flags, int32_t need, int32_t skip,
+                     int64_t max_spins, cudaStream_t s, int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
@@ -644,6 +680,7 @@ cudaError_t tc_apply(const bf16* Xs, const bf16* Ls, float* Y, bf16* Ys, int cou
   p.idesc = idesc_bf16(BM, bn, false, false);
   p.C = Y; p.ldc = r; p.c_bs = m * r;
   p.Cs = Ys; p.cs_stride = (int64_t)count * m * r;
+  p.Cb = Yb;
   p.flags = flags; p.need_mask = need; p.skip_mask = skip;
   p.kr = TC_KR_B_LOWER_NK;  // L^-1 is lower triangular: column tile j needs k <= j only
   p.max_spins = max_spins;

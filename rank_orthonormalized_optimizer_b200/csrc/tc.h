@@ -24,10 +24,12 @@ cudaError_t tc_formb_bq(const float* M, const float* G, const void* Qg, void* Bg
                         __nv_bfloat16* P0s, int count, int64_t m, int64_t n, int64_t r,
                         int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
                         bool* done);
-// R[b] (n x r, fp32) = Bg[b]^T (n x m) * Pg[b] (m x r, bf16).
-cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, int count, int64_t m,
-                        int64_t n, int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s,
-                        int* nlaunch, bool* done);
+// R[b] (n x r, fp32) = Bg[b]^T (n x m) * Pg[b] (m x r, bf16).  When colsq is not null it
+// receives the sums of squares of R's columns over each 32-row block of R, fixed order:
+// colsq[b][i][j] for row block i < 4 ceil(n / 128) (the partials of Q = colnorm(R)).
+cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, float* colsq, int count,
+                        int64_t m, int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
+                        cudaStream_t s, int* nlaunch, bool* done);
 // M <- (M + G) - (1 - mu) Pg Rg^T and X <- X - lr_scale Pg Qg^T (Pg: m x r, Rg, Qg: n x r, bf16).
 // tile_counter: one int in device memory, zero before the call (tiles are taken from it).
 // split: Pg, Rg, Qg are three-way bf16 splits ([3][count][...]) of fp32 operands.
@@ -41,8 +43,9 @@ cudaError_t tc_gemm_bq_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Qs,
                              int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
                              bool* done);
 cudaError_t tc_gemm_btp_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Ps, float* R,
-                              int count, int64_t m, int64_t n, int64_t r, int64_t max_spins,
-                              int32_t* flags, cudaStream_t s, int* nlaunch, bool* done);
+                              float* colsq, int count, int64_t m, int64_t n, int64_t r,
+                              int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
+                              bool* done);
 
 // W[b] (r x r, fp32) = X[b]^T X[b] from the three-way split Xs ([3][count][m][r] bf16),
 // six split products; matrices failing (flags & need) == need && !(flags & skip) skipped.
@@ -52,13 +55,14 @@ cudaError_t tc_gram(const __nv_bfloat16* Xs, float* W, __nv_bfloat16* Ws, int co
                     int64_t r, int32_t* flags, int32_t need, int32_t skip, int64_t max_spins,
                     cudaStream_t s, int* nlaunch, bool* done);
 // Y[b] (m x r, fp32) = X[b] L[b]^T from the splits Xs ([3][count][m][r]) and Ls
-// ([3][count][r][r], L lower triangular), optionally writing Y's split to Ys.  Column
+// ([3][count][r][r], L lower triangular), optionally writing Y's split to Ys and its
+// bf16 rounding to Yb ([count][m][r]).  Column
 // tile j reads L[j][k] for k below the end of its 128-wide window only: the entries of
 // L above the diagonal inside that window must be zero, those further right are not read.
 cudaError_t tc_apply(const __nv_bfloat16* Xs, const __nv_bfloat16* Ls, float* Y,
-                     __nv_bfloat16* Ys, int count, int64_t m, int64_t r, int32_t* flags,
-                     int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s, int* nlaunch,
-                     bool* done);
+                     __nv_bfloat16* Ys, __nv_bfloat16* Yb, int count, int64_t m, int64_t r,
+                     int32_t* flags, int32_t need, int32_t skip, int64_t max_spins,
+                     cudaStream_t s, int* nlaunch, bool* done);
 
 // Triangular operands: K blocks that can only multiply zeros are skipped.
 enum {

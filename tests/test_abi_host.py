@@ -116,15 +116,22 @@ def test_workspace_covers_the_layout():
 def test_workspace_recursive_factorisation_scratch():
     # r > 256 on the tensor path: two more [3][count][r][r] bf16 splits (the Gram's and
     # L21's) for the recursive Cholesky factorisation; none at r <= 256, none on the
-    # CUDA-core path (bf16 GEMM inputs: the two plans differ in nothing else)
+    # CUDA-core path.  With bf16 GEMM inputs the plans differ otherwise only in the
+    # column-norm partials: 4 per 128 rows of R (written by B^T P) on the tensor path,
+    # min(ceil(8 * 148 / count), ceil(n / 16), 256) row ranges on the CUDA-core path.
     def ws_of(r, path):
         c, h, ws = _init([(8, 1024, 1024, r)], kernel_path=path)
         assert c == dion.OK
         dion.dion_free(h)
         return ws
 
-    assert ws_of(512, 0) - ws_of(512, 1) == 2 * 8 * 512 * 512 * 6
-    assert ws_of(256, 0) == ws_of(256, 1)
+    def parts(r, path):
+        ns = 4 * 8 if path == 0 else min(-(-8 * 148 // 8), 1024 // 16, 256)
+        return -(-8 * ns * r * 4 // 1024) * 1024
+
+    for r in (256, 512):
+        extra = 2 * 8 * r * r * 6 if r > 256 else 0
+        assert ws_of(r, 0) - ws_of(r, 1) == extra + parts(r, 0) - parts(r, 1)
 
 
 def test_step_argument_checks_without_device():
