@@ -32,6 +32,7 @@ namespace tc {
 
 constexpr int BM = 128;       // tile rows = TMEM lanes
 constexpr int KCHUNK_SUMSQ = 8;  // K blocks per accumulation chunk of sums of squares
+constexpr int EPI_LD = 17;       // row stride (floats) of the epilogue's staging blocks
 constexpr int BK = 64;        // bf16 elements per 128-byte swizzle row
 constexpr int NT = 256;       // threads per CTA
 constexpr int UPD_BN = 128;   // update tile columns (acc uses 2 * UPD_BN TMEM columns)
@@ -234,6 +235,7 @@ __global__ void __launch_bounds__(NT, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* escr = reinterpret_cast<float*>(tmem_slot + 4);  // 4 warps x [32][EPI_LD]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_per_mat = p.tiles_m * p.tiles_n;
@@ -365,10 +367,16 @@ __global__ void __launch_bounds__(NT, 1)
     mma_commit(drain);
     wait_drain(drain, 0);
   } else if (warp >= 4) {
-    // ---------------- epilogue: TMEM -> registers -> global (fp32 and/or bf16 split)
-    // chunk 0 stores (or accumulates when p.epi == 2); later chunks of the tile add into
-    // C; the split Cs is written from the final value, after the last chunk
+    // ---------------- epilogue: TMEM -> shared -> global (fp32 and/or bf16 copies)
+    // Each warp owns 32 rows.  A 32 x 16 block read from TMEM (lane = row) is passed
+    // through shared memory so that global memory is touched row-contiguously: lane
+    // l then holds columns 4 (l % 4) .. + 3 of rows l / 4 + 8 k, k < 4 (four lanes
+    // write one row's 64 bytes).  Chunk 0 stores (or accumulates when p.epi == 2);
+    // later chunks of the tile add into C; the copies Cb, Cs and the column sums of
+    // squares are written from the final value, after the last chunk.
     const int ew = warp - 4;
+    float* scr = escr + ew * 32 * EPI_LD;
+    const int sub_r = lane >> 2, sub_c = (lane & 3) * 4;
     int lt = 0;
     int t = blockIdx.x;
     bool ok = true;
@@ -376,9 +384,8 @@ __global__ void __launch_bounds__(NT, 1)
       if (!tile_active(p, t, tiles_per_mat)) continue;
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
-      const int64_t row = (int64_t)(rem / p.tiles_n) * BM + ew * 32 + lane;
+      const int64_t row0 = (int64_t)(rem / p.tiles_n) * BM + ew * 32;  // this warp's rows
       const int64_t n0 = (int64_t)(rem % p.tiles_n) * p.block_n;
-      const int64_t off = (int64_t)b * p.c_bs + row * p.ldc;
       int kb0, kb1;
       k_range(p, (rem / p.tiles_n) * BM, (int)n0, kb0, kb1);
       const int nch = n_chunks(p, kb0, kb1);
@@ -395,73 +402,63 @@ __global__ void __launch_bounds__(NT, 1)
           float v[16];
           tmem_ld16(tbase + c, v);
           tmem_wait_ld();
-          if (n0 + c < p.N) {  // uniform across the warp
-            const bool valid = row < p.M;
-            if (valid && epi != 0) {
-              float old[16];
-              if (epi == 2) {
-                const float4* src = reinterpret_cast<const float4*>(p.C + off + n0 + c);
+          if (n0 + c >= p.N) continue;  // uniform across the warp
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const float4 o4 = src[q];
-                  old[4 * q] = o4.x; old[4 * q + 1] = o4.y; old[4 * q + 2] = o4.z; old[4 * q + 3] = o4.w;
+          for (int q = 0; q < 16; ++q) scr[lane * EPI_LD + q] = v[q];
+          __syncwarp();
+          float sq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int rl = sub_r + 8 * k;
+            const int64_t row = row0 + rl;
+            float a[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) a[j] = scr[rl * EPI_LD + sub_c + j];
+            if (row < p.M) {
+              const int64_t at = (int64_t)b * p.c_bs + row * p.ldc + n0 + c + sub_c;
+              if (epi != 0) {
+                float o[4] = {0.f, 0.f, 0.f, 0.f};
+                if (epi == 2) {
+                  const float4 o4 = *reinterpret_cast<const float4*>(p.C + at);
+                  o[0] = o4.x; o[1] = o4.y; o[2] = o4.z; o[3] = o4.w;
                 }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) a[j] = epi == 2 ? fmaf(alpha, a[j], o[j]) : alpha * a[j];
+              }
+              if (p.C) *reinterpret_cast<float4*>(p.C + at) = make_float4(a[0], a[1], a[2], a[3]);
+              if (last && p.Cb) {
+                __align__(8) bf16 h[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) h[j] = __float2bfloat16_rn(a[j]);
+                *reinterpret_cast<uint2*>(p.Cb + at) = *reinterpret_cast<const uint2*>(h);
+              }
+              if (last && p.Cs) {
+                __align__(8) bf16 h[4], mi[4], lo[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) split3_bf16(a[j], h[j], mi[j], lo[j]);
+                *reinterpret_cast<uint2*>(p.Cs + at) = *reinterpret_cast<const uint2*>(h);
+                *reinterpret_cast<uint2*>(p.Cs + at + p.cs_stride) = *reinterpret_cast<const uint2*>(mi);
+                *reinterpret_cast<uint2*>(p.Cs + at + 2 * p.cs_stride) =
+                    *reinterpret_cast<const uint2*>(lo);
               }
 #pragma unroll
-              for (int q = 0; q < 16; ++q) v[q] = epi == 2 ? fmaf(alpha, v[q], old[q]) : alpha * v[q];
-            }
-            if (valid && p.C) {
-              float4* dst = reinterpret_cast<float4*>(p.C + off + n0 + c);
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-            }
-            if (valid && p.Cb && last) {
-              __align__(16) bf16 h[16];
-#pragma unroll
-              for (int q = 0; q < 16; ++q) h[q] = __float2bfloat16_rn(v[q]);
-              uint4* d0 = reinterpret_cast<uint4*>(p.Cb + off + n0 + c);
-              d0[0] = reinterpret_cast<const uint4*>(h)[0];
-              d0[1] = reinterpret_cast<const uint4*>(h)[1];
-            }
-            if (valid && p.Cs && last) {
-              __align__(16) bf16 h[16], mi[16], lo[16];
-#pragma unroll
-              for (int q = 0; q < 16; ++q) split3_bf16(v[q], h[q], mi[q], lo[q]);
-              bf16* base = p.Cs + off + n0 + c;
-              uint4* d0 = reinterpret_cast<uint4*>(base);
-              uint4* d1 = reinterpret_cast<uint4*>(base + p.cs_stride);
-              uint4* d2 = reinterpret_cast<uint4*>(base + 2 * p.cs_stride);
-              const uint4* sh = reinterpret_cast<const uint4*>(h);
-              const uint4* sm = reinterpret_cast<const uint4*>(mi);
-              const uint4* sl = reinterpret_cast<const uint4*>(lo);
-              d0[0] = sh[0]; d0[1] = sh[1];
-              d1[0] = sm[0]; d1[1] = sm[1];
-              d2[0] = sl[0]; d2[1] = sl[1];
-            }
-            if (p.colsq && last) {
-              // the sum of squares of this warp's 32 rows for the 16 columns by a fixed
-              // butterfly (16 shuffles, every lane takes part); lane 2j ends with column
-              // j's sum, j's bits being lane bits 1..4
-              float w[16];
-#pragma unroll
-              for (int q = 0; q < 16; ++q) w[q] = valid ? v[q] * v[q] : 0.f;
-#pragma unroll
-              for (int h = 8; h >= 1; h >>= 1) {
-                const bool hi = (lane & (2 * h)) != 0;
-#pragma unroll
-                for (int j = 0; j < h; ++j) {
-                  const float recv = __shfl_xor_sync(0xffffffffu, hi ? w[j] : w[j + h], 2 * h);
-                  w[j] = (hi ? w[j + h] : w[j]) + recv;
-                }
-              }
-              w[0] += __shfl_xor_sync(0xffffffffu, w[0], 1);
-              if (!(lane & 1)) {
-                const int64_t rb = (int64_t)b * p.tiles_m * 4 + (rem / p.tiles_n) * 4 + ew;
-                p.colsq[rb * p.N + n0 + c + (lane >> 1)] = w[0];
-              }
+              for (int j = 0; j < 4; ++j) sq[j] = fmaf(a[j], a[j], sq[j]);
             }
           }
+          if (p.colsq && last) {
+            // column sums of squares over the warp's 32 rows in a fixed order: the
+            // lane's four rows, then the eight lanes of one column group by butterfly
+#pragma unroll
+            for (int o = 4; o <= 16; o <<= 1)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) sq[j] += __shfl_xor_sync(0xffffffffu, sq[j], o);
+            if (lane < 4) {
+              const int64_t rb = (int64_t)b * p.tiles_m * 4 + (rem / p.tiles_n) * 4 + ew;
+              *reinterpret_cast<float4*>(p.colsq + rb * p.N + n0 + c + sub_c) =
+                  make_float4(sq[0], sq[1], sq[2], sq[3]);
+            }
+          }
+          __syncwarp();
         }
         tc_fence_before();
         __syncwarp();
@@ -497,7 +494,8 @@ static cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Gem
   p.stages = stages;
   p.acc_stride = (uint32_t)p.block_n;
   p.tmem_cols = pow2_cols(2 * p.block_n);
-  const size_t smem = 1024 + stages * stage_bytes + (2 * stages + 5) * 8 + 16;
+  const size_t smem = 1024 + stages * stage_bytes + (2 * stages + 5) * 8 + 16 +
+                      4 * 32 * EPI_LD * sizeof(float);
   auto kern = k_tc_gemm<A_MN, B_MN, SPLIT>;
   // the device's limit rather than this launch's need: a launch captured into a graph
   // is checked against the attribute when the graph runs, after later launches of the
