@@ -171,7 +171,7 @@ dion_status fb_iteration(const Plan& p, const dion_options& o, const FbBufs& f,
   const int32_t skip = dion::F_SDONE | dion::F_SFAIL | DION_MAT_NONFINITE;
   int nl = 0;
   bool done = false;
-  cudaError_t e = dion::tc_gram(src, f.W, f.Ws, p.count, p.m, p.r, f.flags, need, skip,
+  cudaError_t e = dion::tc_gram(src, f.W, f.Ws, nullptr, 0, p.count, p.m, p.r, f.flags, need, skip,
                                 o.max_wait_spins, s, &nl, &done);
   if (e != cudaSuccess || !done)
     return fail(DION_ERR_CUDA, "shifted iteration, Gram: %s",
@@ -464,7 +464,8 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
         return DION_OK;
       };
       if (!p0s_ready) DION_LAUNCH(c, 1, dion::launch_split3(P0, P0s, mr, mr, s));
-      e = dion::tc_gram(P0s, W, Ws, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s,
+      e = dion::tc_gram(P0s, W, Ws, nullptr, 0, cnt, m, r, flags, 0, DION_MAT_FALLBACK,
+                        o.max_wait_spins, s,
                         &nl, &done);
       if ((st = tc_check(e, "tc_gram")) != DION_OK) return st;
       ca.pass = 1; ca.orth_tol = o.orth_tol;
@@ -478,11 +479,16 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
       if ((st = tc_check(e, "tc_apply")) != DION_OK) return st;
       pg_ready = true;
       if (o.orth_mode != DION_ORTH_CHOLQR) {
-        e = dion::tc_gram(P1s, W, Ws, cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s,
+        // the second pass's Gram also measures max|W - I| per matrix (statistics slot 2,
+        // zero since the step began), so that its factorisation can skip matrices the
+        // first pass left orthonormal without reading W
+        e = dion::tc_gram(P1s, W, Ws, r <= 256 ? stats + 2 : nullptr, dion::ST, cnt, m, r, flags,
+                          0, DION_MAT_FALLBACK, o.max_wait_spins, s,
                           &nl, &done);
         if ((st = tc_check(e, "tc_gram")) != DION_OK) return st;
         ca.pass = 2;
         ca.orth_tol = o.orth_mode == DION_ORTH_CHOLQR2 ? -1.f : o.orth_tol;
+        ca.dev_ready = r <= 256 ? 1 : 0;
         if ((st = chol()) != DION_OK) return st;
         e = dion::tc_apply(P1s, Linvs, P2, nullptr, nullptr, cnt, m, r, flags, DION_MAT_CHOLQR2,
                            DION_MAT_FALLBACK, o.max_wait_spins, s, &nl, &done);

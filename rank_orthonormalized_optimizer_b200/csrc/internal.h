@@ -88,6 +88,7 @@ struct CholArgs {
   float orth_tol;      // pass 2: skip the second pass when max|W - I| <= orth_tol
   int64_t o, nl;       // leaf of the recursive factorisation: block (o, o) of size nl
   int64_t m;           // rows of P0 (pass 3: scales the shift)
+  int dev_ready;       // pass 2, r <= 256: stats[ST b + 2] holds max|W - I| already
 };
 // pass 3 = one step of the shifted Cholesky-QR iteration (launch_chol_inv_rec only)
 // r <= 256: one kernel; larger r: the blocked CUDA-core factorisation (many launches).

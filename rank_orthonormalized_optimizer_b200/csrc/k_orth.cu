@@ -39,69 +39,162 @@ __device__ __forceinline__ int32_t fail_bits(int pass, bool nonfinite) {
 
 // ------------------------------------ r <= 256: one CTA, 32 x 32 blocks in shared memory
 // Right-looking blocked Cholesky with the triangular inverse, all on chip:
-//   for each block column k: factor L_kk (one warp), D_k = L_kk^-1 (one warp),
-//   panel L_ik = W_ik D_k^T (a thread per row), trailing W_ij -= L_ik L_jk^T
-//   (a warp per block pair, a lane per row, the row of L_ik in registers);
-//   then L^-1 block row by block row: X_ij = -D_i sum_{k=j}^{i-1} L_ik X_kj, X_ii = D_i.
-// Rows and columns past r are padded with the identity, which factors and inverts
-// to itself.  Padded stride 33 keeps row-per-lane accesses free of bank conflicts.
+//   for each block column k: factor L_kk (one warp, rows in registers, columns by
+//   shuffle, one template step per column so that every index is a constant); panel
+//   L_ik = W_ik L_kk^-T by forward substitution (a thread per row); trailing
+//   W_ij -= L_ik L_jk^T (a warp per block pair, a lane per row);
+//   then D_k = L_kk^-1 for all k at once (a warp per block, a column per lane), and
+//   L^-1 block row by block row: X_ij = -D_i sum_{k=j}^{i-1} L_ik X_kj, X_ii = D_i,
+//   each block product shared by two warps (16 columns each).
+// Only the factorisation of the diagonal blocks is serial across k, and it keeps the
+// one warp that does it short: the triangular inverses are off that path.
+// Rows of a block are LD = 36 floats apart: rows start on 16-byte boundaries, so rows are
+// read and written as float4 -- a lane's own row without bank conflicts (8 lanes cover
+// the 32 banks once), a row shared by the warp as a broadcast -- which cuts the
+// shared-memory instructions of the block products four-fold.  Rows and columns past r
+// are padded with the identity, which factors and inverts to itself.
 // With a.nl > 0 the kernel factors the diagonal block of size nl at (a.o, a.o) of each
 // matrix as a leaf of the recursive factorisation: the pass-2 test against I was made
 // for the whole matrix before, the diagonal statistics are merged by atomics, and the
 // diagonal-ratio test is left to the end of the recursion.
 namespace {
-constexpr int CB = 32, CBS = 33, CBLK = CB * CBS;
+constexpr int CB = 32, LD = 36, BLK = CB * LD;
 __device__ __forceinline__ float* blk_at(float* base, int i, int j) {
-  return base + (i * (i + 1) / 2 + j) * CBLK;
+  return base + (i * (i + 1) / 2 + j) * BLK;
+}
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ float dot4(float4 a, float4 b, float s) {
+  return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, s))));
+}
+// a row held as 8 float4 in registers dotted with a row of a block (a broadcast read)
+__device__ __forceinline__ float dot32(const float4 (&a)[8], const float* row) {
+  float s = 0.f;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) s = dot4(a[q], ld4(row + 4 * q), s);
+  return s;
+}
+// Column J of the in-register Cholesky of a 32 x 32 block (lane u holds row u), then
+// the columns after it.  A template step per column keeps every row index a
+// compile-time constant, so the row stays in registers.
+template <int J>
+__device__ __forceinline__ void chol_col(float (&row)[CB], int lane, int base, int r, bool& fail,
+                                         float& my_inv, float& dmin, float& dmax) {
+  if constexpr (J < CB) {
+    const float d = __shfl_sync(0xffffffffu, row[J], J);
+    fail |= !(d > 0.f) || !isfinite(d);
+    const float dd = fmaxf(d, 1e-30f);
+    const float inv = rsqrtf(dd);
+    const float ljj = dd * inv;
+    if (base + J < r) { dmin = fminf(dmin, ljj); dmax = fmaxf(dmax, ljj); }
+    if (lane == J) { row[J] = ljj; my_inv = inv; }
+    if (lane > J) row[J] *= inv;
+#pragma unroll
+    for (int c = J + 1; c < CB; ++c) {
+      const float lcj = __shfl_sync(0xffffffffu, row[J], c);  // L[c][J]
+      if (lane >= c) row[c] = fmaf(-row[J], lcj, row[c]);
+    }
+    chol_col<J + 1>(row, lane, base, r, fail, my_inv, dmin, dmax);
+  }
+}
+
+// Forward substitution of one row w against L_kk: w <- w L_kk^-T, right-looking over
+// columns; Lt holds L_kk^T (row t = column t of L_kk, read as a broadcast), rinv 1/L_tt.
+template <int J>
+__device__ __forceinline__ void trsv_col(float (&w)[CB], const float* Lt, const float* rinv) {
+  if constexpr (J < CB) {
+    const float lt = w[J] * rinv[J];
+    w[J] = lt;
+    if constexpr (J + 1 < CB) {
+#pragma unroll
+      for (int q = (J + 1) / 4; q < 8; ++q) {
+        const float4 c4 = ld4(Lt + J * LD + 4 * q);
+        const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (4 * q + e > J) w[4 * q + e] = fmaf(-lt, cv[e], w[4 * q + e]);
+      }
+    }
+    trsv_col<J + 1>(w, Lt, rinv);
+  }
+}
+
+// Column lane of L^-1 for the 32 x 32 lower-triangular L whose row u is in lane u's
+// registers: right-looking, x_t /= L_tt, then x_i -= L_it x_t for i > t (L_it by shuffle).
+template <int J>
+__device__ __forceinline__ void trinv_col(const float (&row)[CB], float (&x)[CB], float my_inv) {
+  if constexpr (J < CB) {
+    const float xt = x[J] * __shfl_sync(0xffffffffu, my_inv, J);
+    x[J] = xt;
+#pragma unroll
+    for (int i = J + 1; i < CB; ++i) x[i] = fmaf(-__shfl_sync(0xffffffffu, row[J], i), xt, x[i]);
+    trinv_col<J + 1>(row, x, my_inv);
+  }
+}
+
+// the diagonal entry of the row held by this lane (row u: entry u)
+__device__ __forceinline__ float diag_of(const float (&row)[CB], int lane) {
+  float d = 0.f;
+#pragma unroll
+  for (int c = 0; c < CB; ++c) d = (c == lane) ? row[c] : d;
+  return d;
 }
 }  // namespace
 
+
 size_t chol_blocked_smem_bytes(int64_t r) {
   const int T = (int)((r + CB - 1) / CB);
-  return (size_t)(T * (T + 1) / 2 + T + (T > 1 ? T - 1 : 1)) * CBLK * sizeof(float) + 64 * sizeof(float);
+  return (size_t)(T * (T + 1) / 2 + (T > 2 ? T - 1 : 2)) * BLK * sizeof(float) + 64 * sizeof(float);
 }
 
 template <int NT>
-__global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
-  extern __shared__ float sm[];
+__global__ void __launch_bounds__(NT, 1) k_chol_blocked(CholArgs a) {
+  extern __shared__ __align__(16) float sm[];
   const bool leaf = a.nl > 0;
   const int r = (int)(leaf ? a.nl : a.r);  // size of the factored block
   const int64_t ld = a.r;                  // row stride of W and L^-1
   const int64_t org = a.o * ld + a.o;      // block origin inside each matrix
   const int T = (r + CB - 1) / CB;
-  float* blk = sm;                                  // T(T+1)/2 lower blocks
-  float* dinv = blk + (T * (T + 1) / 2) * CBLK;     // T inverses of the diagonal blocks
-  float* tmp = dinv + T * CBLK;                     // T-1 blocks of partial sums
-  float* red = tmp + (T > 1 ? T - 1 : 1) * CBLK;    // 64 floats
+  float* blk = sm;                                  // T(T+1)/2 lower blocks; the diagonal
+                                                    // ones end as D_k = L_kk^-1
+  float* tmp = blk + (T * (T + 1) / 2) * BLK;       // max(T-1, 2) blocks: partial sums
+  float* red = tmp + (T > 2 ? T - 1 : 2) * BLK;     // of the inverse, scratch; 64 floats
   __shared__ int s_fail;
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = NT / 32;
   const int32_t f0 = a.flags[b];
   if ((leaf || a.pass == 3) ? skip_matrix(f0, a.pass) : (f0 & F_FALLBACK) != 0) return;
+  // second pass: the Gram's epilogue measured max|W - I| already (a NaN fails the test)
+  if (a.pass == 2 && !leaf && a.dev_ready && a.stats[ST * b + 2] <= a.orth_tol) return;
   const float* W = a.W + (int64_t)b * ld * ld + org;
 
-  // load the lower blocks, padding with the identity; check finiteness and |W - I|
+  // load the lower blocks, padding with the identity; check finiteness and |W - I|.
+  // Block row bi is read row by row over its bi + 1 blocks as float4 (rows of W are
+  // contiguous there; r % 16 == 0 keeps a float4 either inside r or past it).
   float dev = 0.f;
   bool nonfin = false;
-  const int nlow = T * (T + 1) / 2;
-  for (int e = tid; e < nlow * CB * CB; e += NT) {
-    const int bl = e / (CB * CB), w = e % (CB * CB), u = w / CB, v = w % CB;
-    int bi = 0;
-    while ((bi + 1) * (bi + 2) / 2 <= bl) ++bi;
-    const int bj = bl - bi * (bi + 1) / 2;
-    const int gi = bi * CB + u, gj = bj * CB + v;
-    float val;
-    if (gi < r && gj < r) {
-      val = W[(int64_t)gi * ld + gj];
-      if (gj <= gi) {
-        nonfin |= !isfinite(val);
-        dev = fmaxf(dev, fabsf(val - (gi == gj ? 1.f : 0.f)));
+  for (int bi = 0; bi < T; ++bi) {
+    const int per_row = 8 * (bi + 1);  // float4 per row of the block row
+    for (int e = tid; e < CB * per_row; e += NT) {
+      const int u = e / per_row, gj = 4 * (e - u * per_row);
+      const int gi = bi * CB + u;
+      float vv[4];
+      if (gi < r && gj < r) {
+        const float4 v4 = *reinterpret_cast<const float4*>(W + (int64_t)gi * ld + gj);
+        vv[0] = v4.x; vv[1] = v4.y; vv[2] = v4.z; vv[3] = v4.w;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (gj + q <= gi) {
+            nonfin |= !isfinite(vv[q]);
+            dev = fmaxf(dev, fabsf(vv[q] - (gi == gj + q ? 1.f : 0.f)));
+          }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) vv[q] = (gi == gj + q) ? 1.f : 0.f;
       }
-    } else {
-      val = (gi == gj) ? 1.f : 0.f;
+      st4(blk_at(blk, bi, gj / CB) + u * LD + (gj % CB), make_float4(vv[0], vv[1], vv[2], vv[3]));
     }
-    blk[bl * CBLK + u * CBS + v] = val;
   }
   if (tid == 0) s_fail = 0;
   nonfin = __syncthreads_or(nonfin);
@@ -116,72 +209,54 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
 
   float dmin = 3.0e38f, dmax = 0.f;  // meaningful in warp 0
   for (int k = 0; k < T; ++k) {
-    float* Lkk = blk_at(blk, k, k);
-    float* Dk = dinv + k * CBLK;
+    float* Dk = blk_at(blk, k, k);
     if (warp == 0) {
-      // Cholesky of the diagonal block in registers: lane u holds row u; entries of
-      // other rows come by warp shuffle (fully unrolled, so the row stays in registers)
-      const int u = lane;
+      // Cholesky of the diagonal block: lane u holds row u in registers; column j of
+      // the other rows comes by warp shuffle (fully unrolled, static indices)
       float row[CB];
 #pragma unroll
-      for (int c = 0; c < CB; ++c) row[c] = Lkk[u * CBS + c];
+      for (int q = 0; q < 8; ++q) {
+        const float4 v4 = ld4(Dk + lane * LD + 4 * q);
+        row[4 * q] = v4.x; row[4 * q + 1] = v4.y; row[4 * q + 2] = v4.z; row[4 * q + 3] = v4.w;
+      }
       bool fail = false;
+      float my_inv = 0.f;  // 1 / L_uu of this lane's row
+      chol_col<0>(row, lane, k * CB, r, fail, my_inv, dmin, dmax);
+      // L_kk (zeros above the diagonal) into the block, its transpose into scratch for
+      // the panel, the reciprocals of its diagonal into red
 #pragma unroll
-      for (int j = 0; j < CB; ++j) {
-        const float d = __shfl_sync(0xffffffffu, row[j], j);
-        fail |= !(d > 0.f) || !isfinite(d);
-        const float ljj = sqrtf(fmaxf(d, 1e-30f));
-        if (k * CB + j < r) { dmin = fminf(dmin, ljj); dmax = fmaxf(dmax, ljj); }
-        if (u == j) row[j] = ljj;
-        if (u > j) row[j] = row[j] / ljj;
+      for (int q = 0; q < 8; ++q)
+        st4(Dk + lane * LD + 4 * q,
+            make_float4(4 * q <= lane ? row[4 * q] : 0.f, 4 * q + 1 <= lane ? row[4 * q + 1] : 0.f,
+                        4 * q + 2 <= lane ? row[4 * q + 2] : 0.f,
+                        4 * q + 3 <= lane ? row[4 * q + 3] : 0.f));
 #pragma unroll
-        for (int c = j + 1; c < CB; ++c) {
-          const float lcj = __shfl_sync(0xffffffffu, row[j], c);  // L[c][j]
-          if (u >= c) row[c] = fmaf(-row[j], lcj, row[c]);
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < CB; ++c) Lkk[u * CBS + c] = (c <= u) ? row[c] : 0.f;
-      if (fail) {
-        if (lane == 0) s_fail = 1;
-      } else {
-        // D_k = L_kk^-1, lane v computes column v by forward substitution; row i of L
-        // is broadcast from lane i
-        const int v = lane;
-        float x[CB];
-#pragma unroll
-        for (int i = 0; i < CB; ++i) {
-          float sacc = (i == v) ? 1.f : 0.f;
-#pragma unroll
-          for (int t = 0; t < i; ++t) sacc = fmaf(-__shfl_sync(0xffffffffu, row[t], i), x[t], sacc);
-          const float lii = __shfl_sync(0xffffffffu, row[i], i);
-          x[i] = (i < v) ? 0.f : sacc / lii;
-        }
-#pragma unroll
-        for (int i = 0; i < CB; ++i) Dk[i * CBS + v] = x[i];
-      }
+      for (int c = 0; c < CB; ++c) tmp[c * LD + lane] = (c <= lane) ? row[c] : 0.f;
+      red[lane] = my_inv;
+      if (fail && lane == 0) s_fail = 1;
     }
     __syncthreads();
     if (s_fail) {
       if (tid == 0) atomicOr(a.flags + b, fail_bits(a.pass, false));
       return;
     }
-    // panel: L_ik = W_ik D_k^T, one thread per row of the panel
+    // panel: L_ik = W_ik L_kk^-T by forward substitution, one thread per row of the
+    // panel, the row in registers; column t of L_kk is row t of the transpose in tmp
     const int prow = (T - 1 - k) * CB;
     for (int rr = tid; rr < prow; rr += NT) {
-      float* row = blk_at(blk, k + 1 + rr / CB, k) + (rr % CB) * CBS;
+      float* rowp = blk_at(blk, k + 1 + rr / CB, k) + (rr % CB) * LD;
       float w[CB];
 #pragma unroll
-      for (int t = 0; t < CB; ++t) w[t] = row[t];
-#pragma unroll
-      for (int c = 0; c < CB; ++c) {
-        float sacc = 0.f;
-        for (int t = 0; t <= c; ++t) sacc = fmaf(w[t], Dk[c * CBS + t], sacc);
-        row[c] = sacc;
+      for (int q = 0; q < 8; ++q) {
+        const float4 v4 = ld4(rowp + 4 * q);
+        w[4 * q] = v4.x; w[4 * q + 1] = v4.y; w[4 * q + 2] = v4.z; w[4 * q + 3] = v4.w;
       }
+      trsv_col<0>(w, tmp, red);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) st4(rowp + 4 * q, make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
     }
     __syncthreads();
-    // trailing update: W_ij -= L_ik L_jk^T for k < j <= i
+    // trailing update: W_ij -= L_ik L_jk^T for k < j <= i, a warp per block pair
     const int nt = T - 1 - k;
     const int npairs = nt * (nt + 1) / 2;
     for (int pi = warp; pi < npairs; pi += NW) {
@@ -189,17 +264,20 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
       while ((ii + 1) * (ii + 2) / 2 <= pi) ++ii;
       const int jj = pi - ii * (ii + 1) / 2;
       const int i = k + 1 + ii, j = k + 1 + jj;
-      const float* Lik = blk_at(blk, i, k) + lane * CBS;
+      const float* Lik = blk_at(blk, i, k) + lane * LD;
       const float* Ljk = blk_at(blk, j, k);
-      float* Wij = blk_at(blk, i, j) + lane * CBS;
-      float av[CB];
+      float* Wij = blk_at(blk, i, j) + lane * LD;
+      float4 av[8];
 #pragma unroll
-      for (int t = 0; t < CB; ++t) av[t] = Lik[t];
-      for (int c = 0; c < CB; ++c) {
-        float sacc = 0.f;
-#pragma unroll
-        for (int t = 0; t < CB; ++t) sacc = fmaf(av[t], Ljk[c * CBS + t], sacc);
-        Wij[c] -= sacc;
+      for (int q = 0; q < 8; ++q) av[q] = ld4(Lik + 4 * q);
+#pragma unroll 1
+      for (int cg = 0; cg < 8; ++cg) {
+        float4 wv = ld4(Wij + 4 * cg);
+        wv.x -= dot32(av, Ljk + (4 * cg) * LD);
+        wv.y -= dot32(av, Ljk + (4 * cg + 1) * LD);
+        wv.z -= dot32(av, Ljk + (4 * cg + 2) * LD);
+        wv.w -= dot32(av, Ljk + (4 * cg + 3) * LD);
+        st4(Wij + 4 * cg, wv);
       }
     }
     __syncthreads();
@@ -221,39 +299,89 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
     }
   }
 
-  // L^-1 block row by block row; X_ij overwrites L_ij once row i is done
+  // D_k = L_kk^-1 for every diagonal block at once, a warp per block: lane u loads row u
+  // of L_kk, lane v computes column v of D_k (entries of L come by shuffle), and the
+  // column replaces the block after the whole warp has read it
+  for (int kk = warp; kk < T; kk += NW) {
+    float* Dk = blk_at(blk, kk, kk);
+    float row[CB], x[CB];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 v4 = ld4(Dk + lane * LD + 4 * q);
+      row[4 * q] = v4.x; row[4 * q + 1] = v4.y; row[4 * q + 2] = v4.z; row[4 * q + 3] = v4.w;
+    }
+    const float my_inv = 1.f / diag_of(row, lane);
+#pragma unroll
+    for (int i = 0; i < CB; ++i) x[i] = (i == lane) ? 1.f : 0.f;
+    trinv_col<0>(row, x, my_inv);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < CB; ++i) Dk[i * LD + lane] = (i >= lane) ? x[i] : 0.f;
+  }
+  __syncthreads();
+  // L^-1 block row by block row; X_ij overwrites L_ij once row i is done.  Each block
+  // product is shared by two warps, 16 columns each; the lane owns a row.
   for (int i = 1; i < T; ++i) {
-    for (int j = warp; j < i; j += NW) {
-      float acc[CB];
+    for (int wj = warp; wj < 2 * i; wj += NW) {
+      const int j = wj >> 1, c0 = (wj & 1) * 16;
+      float acc[16];
 #pragma unroll
-      for (int c = 0; c < CB; ++c) acc[c] = 0.f;
+      for (int c = 0; c < 16; ++c) acc[c] = 0.f;
       for (int k = j; k < i; ++k) {
-        const float* Lik = blk_at(blk, i, k) + lane * CBS;
-        const float* Xkj = (k == j) ? dinv + j * CBLK : blk_at(blk, k, j);
-        float av[CB];
+        const float* Lik = blk_at(blk, i, k) + lane * LD;
+        const float* Xkj = blk_at(blk, k, j) + c0;  // X_jj = D_j on the diagonal
+#pragma unroll 1
+        for (int tg = 0; tg < 8; ++tg) {
+          const float4 l4 = ld4(Lik + 4 * tg);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-        for (int t = 0; t < CB; ++t) av[t] = Lik[t];
+          for (int tt = 0; tt < 4; ++tt) {
+            const float* xr = Xkj + (4 * tg + tt) * LD;
 #pragma unroll
-        for (int t = 0; t < CB; ++t) {
-          const float* xr = Xkj + t * CBS;
-#pragma unroll
-          for (int c = 0; c < CB; ++c) acc[c] = fmaf(av[t], xr[c], acc[c]);
+            for (int q = 0; q < 4; ++q) {
+              const float4 x4 = ld4(xr + 4 * q);
+              acc[4 * q] = fmaf(lv[tt], x4.x, acc[4 * q]);
+              acc[4 * q + 1] = fmaf(lv[tt], x4.y, acc[4 * q + 1]);
+              acc[4 * q + 2] = fmaf(lv[tt], x4.z, acc[4 * q + 2]);
+              acc[4 * q + 3] = fmaf(lv[tt], x4.w, acc[4 * q + 3]);
+            }
+          }
         }
       }
-      float* Sj = tmp + j * CBLK + lane * CBS;
+      float* Sj = tmp + j * BLK + lane * LD + c0;
 #pragma unroll
-      for (int c = 0; c < CB; ++c) Sj[c] = acc[c];
+      for (int q = 0; q < 4; ++q)
+        st4(Sj + 4 * q, make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]));
     }
     __syncthreads();
-    for (int j = warp; j < i; j += NW) {
-      const float* Di = dinv + i * CBLK + lane * CBS;
-      const float* Sj = tmp + j * CBLK;
-      float* Xij = blk_at(blk, i, j) + lane * CBS;
-      for (int c = 0; c < CB; ++c) {
-        float sacc = 0.f;
-        for (int t = 0; t <= lane; ++t) sacc = fmaf(Di[t], Sj[t * CBS + c], sacc);
-        Xij[c] = -sacc;
+    for (int wj = warp; wj < 2 * i; wj += NW) {
+      const int j = wj >> 1, c0 = (wj & 1) * 16;
+      const float* Di = blk_at(blk, i, i) + lane * LD;
+      const float* Sj = tmp + j * BLK + c0;
+      float acc[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) acc[c] = 0.f;
+#pragma unroll 1
+      for (int tg = 0; tg < 8; ++tg) {
+        const float4 d4 = ld4(Di + 4 * tg);
+        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+        for (int tt = 0; tt < 4; ++tt) {
+          const float* sr = Sj + (4 * tg + tt) * LD;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float4 s4 = ld4(sr + 4 * q);
+            acc[4 * q] = fmaf(dv[tt], s4.x, acc[4 * q]);
+            acc[4 * q + 1] = fmaf(dv[tt], s4.y, acc[4 * q + 1]);
+            acc[4 * q + 2] = fmaf(dv[tt], s4.z, acc[4 * q + 2]);
+            acc[4 * q + 3] = fmaf(dv[tt], s4.w, acc[4 * q + 3]);
+          }
+        }
       }
+      float* Xij = blk_at(blk, i, j) + lane * LD + c0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        st4(Xij + 4 * q, make_float4(-acc[4 * q], -acc[4 * q + 1], -acc[4 * q + 2], -acc[4 * q + 3]));
     }
     __syncthreads();
   }
@@ -262,22 +390,29 @@ __global__ void __launch_bounds__(NT) k_chol_blocked(CholArgs a) {
   const int64_t mo = (int64_t)b * ld * ld + org;
   float* Li = a.Linv + mo;
   const int64_t part = (int64_t)a.count * ld * ld;
-  for (int64_t e = tid; e < (int64_t)r * r; e += NT) {
-    const int gi = (int)(e / r), gj = (int)(e % r);
-    float val = 0.f;
-    if (gj <= gi) {
-      const int bi = gi / CB, bj = gj / CB, u = gi % CB, v = gj % CB;
-      val = (bi == bj) ? dinv[bi * CBLK + u * CBS + v] : blk_at(blk, bi, bj)[u * CBS + v];
-    }
-    const int64_t at = (int64_t)gi * ld + gj;
-    Li[at] = val;
-    if (a.Linvs) {
-      bf16 h, mi, lo;
-      split3_bf16(val, h, mi, lo);
-      bf16* d = a.Linvs + mo + at;
-      d[0] = h;
-      d[part] = mi;
-      d[2 * part] = lo;
+  // block row bi, row by row over all T blocks (zeros right of the diagonal), float4
+  for (int bi = 0; bi < T; ++bi) {
+    const int per_row = 8 * T;
+    for (int e = tid; e < CB * per_row; e += NT) {
+      const int u = e / per_row, gj = 4 * (e - u * per_row);
+      const int gi = bi * CB + u, bj = gj / CB, v = gj % CB;
+      if (gi >= r || gj >= r) continue;
+      float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (bj <= bi) {
+        val = ld4(blk_at(blk, bi, bj) + u * LD + v);
+      }
+      const int64_t at = (int64_t)gi * ld + gj;
+      *reinterpret_cast<float4*>(Li + at) = val;
+      if (a.Linvs) {
+        const float vv[4] = {val.x, val.y, val.z, val.w};
+        __align__(8) bf16 h[4], mi[4], lo[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) split3_bf16(vv[q], h[q], mi[q], lo[q]);
+        bf16* d = a.Linvs + mo + at;
+        *reinterpret_cast<uint2*>(d) = *reinterpret_cast<const uint2*>(h);
+        *reinterpret_cast<uint2*>(d + part) = *reinterpret_cast<const uint2*>(mi);
+        *reinterpret_cast<uint2*>(d + 2 * part) = *reinterpret_cast<const uint2*>(lo);
+      }
     }
   }
   if (!leaf && a.pass == 2 && tid == 0) atomicOr(a.flags + b, F_CHOLQR2);
@@ -898,3 +1033,4 @@ cudaError_t launch_householder(const float* P0, const void* P0s, float* work_cm,
 }
 
 }  // namespace dion
+

@@ -178,6 +178,8 @@ struct GemmP {
   bf16* Cb;                          // bf16 copy of the result (may be null)
   float* colsq;                      // per-warp column sums of squares (may be null):
                                      // [batch][tiles_m * 4][N], row block tm*4 + warp
+  float* devmax;                     // max |C_ij - I_ij| over j <= i, per matrix (may be
+  int dev_stride;                    // null): atomic max into devmax[b * dev_stride]
   int32_t* flags;
   int32_t need_mask, skip_mask;      // matrices whose flags fail this are skipped
   int lower_only;                    // skip tiles above the diagonal (symmetric results)
@@ -194,6 +196,11 @@ struct GemmP {
 // out (about 2.5e-5 relative at K = 4096 with six split products per step).  Long K
 // ranges are therefore cut into chunks of kchunk blocks, each accumulated from zero in
 // TMEM, and the epilogue adds the chunks in fp32 registers (round to nearest) into C.
+// max that keeps a NaN (fmaxf would drop it)
+__device__ __forceinline__ float max_keep_nan(float a, float b) {
+  return (isnan(a) || isnan(b)) ? a + b : fmaxf(a, b);
+}
+
 __device__ __forceinline__ int n_chunks(const GemmP& p, int kb0, int kb1) {
   return p.kchunk > 0 ? (kb1 - kb0 + p.kchunk - 1) / p.kchunk : 1;
 }
@@ -377,6 +384,7 @@ __global__ void __launch_bounds__(NT, 1)
     const int ew = warp - 4;
     float* scr = escr + ew * 32 * EPI_LD;
     const int sub_r = lane >> 2, sub_c = (lane & 3) * 4;
+    float dev = 0.f;  // max |C - I| over this warp's rows of the current tile (lower part)
     int lt = 0;
     int t = blockIdx.x;
     bool ok = true;
@@ -443,6 +451,14 @@ __global__ void __launch_bounds__(NT, 1)
               }
 #pragma unroll
               for (int j = 0; j < 4; ++j) sq[j] = fmaf(a[j], a[j], sq[j]);
+              if (p.devmax && last) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const int64_t col = n0 + c + sub_c + j;
+                  const float e = fabsf(a[j] - (col == row ? 1.f : 0.f));
+                  if (col <= row) dev = max_keep_nan(dev, e);
+                }
+              }
             }
           }
           if (p.colsq && last) {
@@ -466,6 +482,16 @@ __global__ void __launch_bounds__(NT, 1)
         ++lt;
       }
       if (!ok) break;
+      if (p.devmax) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dev = max_keep_nan(dev, __shfl_xor_sync(0xffffffffu, dev, o));
+        // non-negative floats order like their bits; a NaN is stored as the positive
+        // quiet NaN, whose bits exceed every finite value's
+        if (lane == 0 && !(dev <= 0.f))
+          atomicMax(reinterpret_cast<int*>(p.devmax + (int64_t)b * p.dev_stride),
+                    isnan(dev) ? 0x7fc00000 : __float_as_int(dev));
+        dev = 0.f;
+      }
     }
     if (t < ntiles && lane == 0) mark_unfinished(p.flags, t, ntiles, tiles_per_mat, gridDim.x);
   }
@@ -628,9 +654,9 @@ cudaError_t tc_gemm_btp_split(const bf16* Bs, const bf16* Ps, float* R, float* c
   return e;
 }
 
-cudaError_t tc_gram(const bf16* Xs, float* W, bf16* Ws, int count, int64_t m, int64_t r,
-                    int32_t* flags, int32_t need, int32_t skip, int64_t max_spins, cudaStream_t s,
-                    int* nlaunch, bool* done) {
+cudaError_t tc_gram(const bf16* Xs, float* W, bf16* Ws, float* devmax, int dev_stride, int count,
+                    int64_t m, int64_t r, int32_t* flags, int32_t need, int32_t skip,
+                    int64_t max_spins, cudaStream_t s, int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
@@ -652,6 +678,7 @@ cudaError_t tc_gram(const bf16* Xs, float* W, bf16* Ws, int count, int64_t m, in
   p.flags = flags; p.need_mask = need; p.skip_mask = skip;
   p.lower_only = bn == BM;
   p.kchunk = KCHUNK_SUMSQ;  // the diagonal sums squares: keep the accumulation unbiased
+  p.devmax = devmax; p.dev_stride = dev_stride;
   p.max_spins = max_spins;
   cudaError_t e = launch_gemm<true, true, 3>(ma, mb, p, s);
   if (e == cudaSuccess) { *done = true; *nlaunch = 1; }

@@ -50,10 +50,12 @@ cudaError_t tc_gemm_btp_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Ps, 
 // W[b] (r x r, fp32) = X[b]^T X[b] from the three-way split Xs ([3][count][m][r] bf16),
 // six split products; matrices failing (flags & need) == need && !(flags & skip) skipped.
 // Only the 128 x 128 tiles on and below the diagonal are written (r > 64), and, when Ws
-// is not null, their split ([3][count][r][r]) as well.
-cudaError_t tc_gram(const __nv_bfloat16* Xs, float* W, __nv_bfloat16* Ws, int count, int64_t m,
-                    int64_t r, int32_t* flags, int32_t need, int32_t skip, int64_t max_spins,
-                    cudaStream_t s, int* nlaunch, bool* done);
+// is not null, their split ([3][count][r][r]) as well.  When devmax is not null,
+// max_{j <= i} |W_ij - I_ij| of matrix b is max-ed into devmax[b * dev_stride] (which must
+// hold a non-negative value before the call; NaN wins).
+cudaError_t tc_gram(const __nv_bfloat16* Xs, float* W, __nv_bfloat16* Ws, float* devmax,
+                    int dev_stride, int count, int64_t m, int64_t r, int32_t* flags, int32_t need,
+                    int32_t skip, int64_t max_spins, cudaStream_t s, int* nlaunch, bool* done);
 // Y[b] (m x r, fp32) = X[b] L[b]^T from the splits Xs ([3][count][m][r]) and Ls
 // ([3][count][r][r], L lower triangular), optionally writing Y's split to Ys and its
 // bf16 rounding to Yb ([count][m][r]).  Column
