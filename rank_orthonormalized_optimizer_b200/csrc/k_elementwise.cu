@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(256) k_colnorm_apply(const float* __restrict__
                                                         int32_t* __restrict__ flags, int64_t n,
                                                         int64_t r, int nsplit, int64_t part_bs,
                                                         int64_t rows_per_block) {
-  extern __shared__ float norm_s[];  // r floats
+  extern __shared__ __align__(16) float norm_s[];  // r floats
   const int64_t b = blockIdx.y;
   bool zero = false;
   for (int64_t j = threadIdx.x; j < r; j += blockDim.x) {
@@ -375,10 +375,16 @@ __global__ void __launch_bounds__(256) k_colnorm_apply(const float* __restrict__
   const int64_t e0 = (b * n + i0) * vc, e1 = (b * n + i1) * vc;
   const float4* R4 = reinterpret_cast<const float4*>(R);
   float4* Q4 = reinterpret_cast<float4*>(Q);
+  // the thread's column group advances by blockDim % vc per iteration (no division)
+  const int vci = (int)vc, step = (int)(blockDim.x % vc);
+  int jg = (int)(threadIdx.x % vc);
   for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
-    const int j = (int)((e - e0) % vc) * 4;
+    const int j = jg * 4;
+    jg += step;
+    if (jg >= vci) jg -= vci;
     const float4 rv = R4[e];
-    const float n0 = norm_s[j], n1 = norm_s[j + 1], n2 = norm_s[j + 2], n3 = norm_s[j + 3];
+    const float4 nv = *reinterpret_cast<const float4*>(norm_s + j);
+    const float n0 = nv.x, n1 = nv.y, n2 = nv.z, n3 = nv.w;
     float4 qv;
     qv.x = n0 > 0.f ? rv.x / n0 : 0.f;
     qv.y = n1 > 0.f ? rv.y / n1 : 0.f;
