@@ -748,9 +748,10 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
     p.scale = d.scale > 0.f ? d.scale : (float)std::sqrt((double)d.m / (double)d.n);
     p.mat0 = mats;
     mats += d.count;
-    // column-norm partials: on the tensor path B^T P writes one per 32 rows of R
-    p.nsplit = o.kernel_path == DION_PATH_TENSOR ? (int)(4 * ((d.n + 127) / 128))
-                                                 : dion::colnorm_splits(d.count, d.n);
+    // column-norm partials: on the tensor path B^T P writes them, one per block of
+    // R's rows (256 rows with bf16 operands, 32 rows from splits)
+    p.nsplit = o.kernel_path != DION_PATH_TENSOR ? dion::colnorm_splits(d.count, d.n)
+               : (bf ? dion::tc_btp_col_splits(d.n) : (int)(4 * ((d.n + 127) / 128)));
     const size_t c = (size_t)d.count;
     p.off_Bg = take(c * d.m * d.n * ge);
     p.off_Qg = take(c * d.n * d.r * ge);

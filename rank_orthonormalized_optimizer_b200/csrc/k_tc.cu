@@ -180,6 +180,9 @@ struct GemmP {
                                      // [batch][tiles_m * 4][N], row block tm*4 + warp
   float* devmax;                     // max |C_ij - I_ij| over j <= i, per matrix (may be
   int dev_stride;                    // null): atomic max into devmax[b * dev_stride]
+  int c_trans;                       // store C transposed: C[j * ldc + i] (no Cs, Cb); colsq
+                                     // then holds row sums of squares [batch][tiles_n][M]
+  int m_fast;                        // tile order: M tiles of one N tile next to each other
   int32_t* flags;
   int32_t need_mask, skip_mask;      // matrices whose flags fail this are skipped
   int lower_only;                    // skip tiles above the diagonal (symmetric results)
@@ -216,10 +219,18 @@ __device__ __forceinline__ void k_range(const GemmP& p, int m0, int n0, int& kb0
   if (kb1 <= kb0) kb1 = kb0 + 1;  // never empty: a block past K loads as zeros
 }
 
+// M and N tile of tile rem within a matrix
+__device__ __forceinline__ int tile_mi(const GemmP& p, int rem) {
+  return p.m_fast ? rem % p.tiles_m : rem / p.tiles_n;
+}
+__device__ __forceinline__ int tile_ni(const GemmP& p, int rem) {
+  return p.m_fast ? rem / p.tiles_m : rem % p.tiles_n;
+}
+
 __device__ __forceinline__ bool tile_active(const GemmP& p, int t, int tiles_per_mat) {
   if (p.lower_only) {
     const int rem = t % tiles_per_mat;
-    if ((rem % p.tiles_n) * p.block_n > (rem / p.tiles_n) * BM) return false;
+    if (tile_ni(p, rem) * p.block_n > tile_mi(p, rem) * BM) return false;
   }
   if (p.need_mask == 0 && p.skip_mask == 0) return true;
   const int32_t f = p.flags[t / tiles_per_mat];
@@ -281,8 +292,8 @@ __global__ void __launch_bounds__(NT, 1)
       if (!tile_active(p, t, tiles_per_mat)) continue;
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
-      const int m0 = (rem / p.tiles_n) * BM;
-      const int n0 = (rem % p.tiles_n) * p.block_n;
+      const int m0 = tile_mi(p, rem) * BM;
+      const int n0 = tile_ni(p, rem) * p.block_n;
       int kb0, kb1;
       k_range(p, m0, n0, kb0, kb1);
       bool ok = true;
@@ -335,7 +346,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (!tile_active(p, t, tiles_per_mat)) continue;
       const int rem = t % tiles_per_mat;
       int kb0, kb1;
-      k_range(p, (rem / p.tiles_n) * BM, (rem % p.tiles_n) * p.block_n, kb0, kb1);
+      k_range(p, tile_mi(p, rem) * BM, tile_ni(p, rem) * p.block_n, kb0, kb1);
       const int nch = n_chunks(p, kb0, kb1);
       for (int ch = 0; ch < nch && ok; ++ch) {
       const int acc = lt & 1;
@@ -392,10 +403,11 @@ __global__ void __launch_bounds__(NT, 1)
       if (!tile_active(p, t, tiles_per_mat)) continue;
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
-      const int64_t row0 = (int64_t)(rem / p.tiles_n) * BM + ew * 32;  // this warp's rows
-      const int64_t n0 = (int64_t)(rem % p.tiles_n) * p.block_n;
+      const int64_t row0 = (int64_t)tile_mi(p, rem) * BM + ew * 32;  // this warp's rows
+      const int64_t n0 = (int64_t)tile_ni(p, rem) * p.block_n;
       int kb0, kb1;
-      k_range(p, (rem / p.tiles_n) * BM, (int)n0, kb0, kb1);
+      k_range(p, tile_mi(p, rem) * BM, (int)n0, kb0, kb1);
+      float rsq = 0.f;  // transposed store: this lane's row sum of squares over the tile
       const int nch = n_chunks(p, kb0, kb1);
       for (int ch = 0; ch < nch; ++ch) {
         const int acc = lt & 1;
@@ -411,6 +423,20 @@ __global__ void __launch_bounds__(NT, 1)
           tmem_ld16(tbase + c, v);
           tmem_wait_ld();
           if (n0 + c >= p.N) continue;  // uniform across the warp
+          if (p.c_trans) {
+            // C[j][i]: for each column j the warp's 32 rows are 32 consecutive floats
+            const int64_t row = row0 + lane;
+            if (row < p.M) {
+              float* dst = p.C + (int64_t)b * p.c_bs + (n0 + c) * p.ldc + row;
+#pragma unroll
+              for (int q = 0; q < 16; ++q)
+                if (n0 + c + q < p.N) {
+                  dst[q * p.ldc] = v[q];
+                  rsq = fmaf(v[q], v[q], rsq);
+                }
+            }
+            continue;
+          }
 #pragma unroll
           for (int q = 0; q < 16; ++q) scr[lane * EPI_LD + q] = v[q];
           __syncwarp();
@@ -469,7 +495,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
               for (int j = 0; j < 4; ++j) sq[j] += __shfl_xor_sync(0xffffffffu, sq[j], o);
             if (lane < 4) {
-              const int64_t rb = (int64_t)b * p.tiles_m * 4 + (rem / p.tiles_n) * 4 + ew;
+              const int64_t rb = (int64_t)b * p.tiles_m * 4 + tile_mi(p, rem) * 4 + ew;
               *reinterpret_cast<float4*>(p.colsq + rb * p.N + n0 + c + sub_c) =
                   make_float4(sq[0], sq[1], sq[2], sq[3]);
             }
@@ -482,6 +508,8 @@ __global__ void __launch_bounds__(NT, 1)
         ++lt;
       }
       if (!ok) break;
+      if (p.c_trans && p.colsq && row0 + lane < p.M)
+        p.colsq[((int64_t)b * p.tiles_n + tile_ni(p, rem)) * p.M + row0 + lane] = rsq;
       if (p.devmax) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) dev = max_keep_nan(dev, __shfl_xor_sync(0xffffffffu, dev, o));
@@ -572,25 +600,35 @@ cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, bf16* P0s, int
   return e;
 }
 
+int tc_btp_col_splits(int64_t n) {
+  return (int)((n + tc::pick_block_n(n, 64) - 1) / tc::pick_block_n(n, 64));
+}
+
 cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, float* colsq, int count,
                         int64_t m, int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
                         cudaStream_t s, int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
-  const int bn = pick_block_n(r, 64);  // MN-major B: whole 64-wide atoms (zero-filled past r)
+  // computed as R^T = P^T B: tiles of r x up to 256 columns of B (both operands read
+  // MN-major), so each 48 KB stage brings 32 KB of B from DRAM (the stream this kernel
+  // waits on) and 16 KB of P (L2-resident); the two r halves of a column block run on
+  // neighbouring CTAs (tile order M-fast) and share B in L2; R is stored transposed
+  const int bn = pick_block_n(n, 64);  // MN-major B: whole 64-wide atoms (zero-filled past n)
   CUtensorMap ma, mb;
-  if (!map3d(&ma, Bg, true, n, m, count, 64, BK)) return cudaSuccess;
-  if (!map3d(&mb, Pg, true, r, m, count, 64, BK)) return cudaSuccess;
+  if (!map3d(&ma, Pg, true, r, m, count, 64, BK)) return cudaSuccess;
+  if (!map3d(&mb, Bg, true, n, m, count, 64, BK)) return cudaSuccess;
   GemmP p{};
-  p.M = n; p.N = r; p.K = m;
+  p.M = r; p.N = n; p.K = m;
   p.batch = count;
   p.block_n = bn;
-  p.tiles_m = (int)((n + BM - 1) / BM);
-  p.tiles_n = (int)((r + bn - 1) / bn);
+  p.tiles_m = (int)((r + BM - 1) / BM);
+  p.tiles_n = (int)((n + bn - 1) / bn);
   p.num_kb = (int)((m + BK - 1) / BK);
   p.idesc = idesc_bf16(BM, bn, true, true);
   p.C = R; p.ldc = r; p.c_bs = n * r;
+  p.c_trans = 1;
+  p.m_fast = 1;
   p.colsq = colsq;
   p.flags = flags;
   p.max_spins = max_spins;

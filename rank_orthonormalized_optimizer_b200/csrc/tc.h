@@ -25,11 +25,13 @@ cudaError_t tc_formb_bq(const float* M, const float* G, const void* Qg, void* Bg
                         int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
                         bool* done);
 // R[b] (n x r, fp32) = Bg[b]^T (n x m) * Pg[b] (m x r, bf16).  When colsq is not null it
-// receives the sums of squares of R's columns over each 32-row block of R, fixed order:
-// colsq[b][i][j] for row block i < 4 ceil(n / 128) (the partials of Q = colnorm(R)).
+// receives the sums of squares of R's columns over blocks of R's rows, fixed order:
+// colsq[b][i][j] for row block i < tc_btp_col_splits(n) (the partials of Q = colnorm(R)).
 cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, float* colsq, int count,
                         int64_t m, int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
                         cudaStream_t s, int* nlaunch, bool* done);
+int tc_btp_col_splits(int64_t n);
+// As tc_gemm_btp from three-way splits; colsq blocks of 32 rows: 4 ceil(n / 128) of them.
 // M <- (M + G) - (1 - mu) Pg Rg^T and X <- X - lr_scale Pg Qg^T (Pg: m x r, Rg, Qg: n x r, bf16).
 // tile_counter: one int in device memory, zero before the call (tiles are taken from it).
 // split: Pg, Rg, Qg are three-way bf16 splits ([3][count][...]) of fp32 operands.

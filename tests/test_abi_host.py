@@ -117,8 +117,9 @@ def test_workspace_recursive_factorisation_scratch():
     # r > 256 on the tensor path: two more [3][count][r][r] bf16 splits (the Gram's and
     # L21's) for the recursive Cholesky factorisation; none at r <= 256, none on the
     # CUDA-core path.  With bf16 GEMM inputs the plans differ otherwise only in the
-    # column-norm partials: 4 per 128 rows of R (written by B^T P) on the tensor path,
-    # min(ceil(8 * 148 / count), ceil(n / 16), 256) row ranges on the CUDA-core path.
+    # column-norm partials: one per block of up to 256 rows of R (written by B^T P) on
+    # the tensor path, min(ceil(8 * 148 / count), ceil(n / 16), 256) row ranges on the
+    # CUDA-core path.
     def ws_of(r, path):
         c, h, ws = _init([(8, 1024, 1024, r)], kernel_path=path)
         assert c == dion.OK
@@ -126,7 +127,7 @@ def test_workspace_recursive_factorisation_scratch():
         return ws
 
     def parts(r, path):
-        ns = 4 * 8 if path == 0 else min(-(-8 * 148 // 8), 1024 // 16, 256)
+        ns = 1024 // 256 if path == 0 else min(-(-8 * 148 // 8), 1024 // 16, 256)
         return -(-8 * ns * r * 4 // 1024) * 1024
 
     for r in (256, 512):
