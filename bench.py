@@ -182,9 +182,13 @@ def update_kernel_hash():
 def oracle_sample(wl: W.Workload, steps: int, budget_s: float = 20.0):
     """Time the fp64 oracle on one matrix per bucket; returns (params/s, seconds, cores, note)."""
     import oracle
+    blas = "unknown"
     try:
         from threadpoolctl import threadpool_info
-        cores = max((i.get("num_threads", 0) for i in threadpool_info()), default=os.cpu_count())
+        info = threadpool_info()
+        cores = max((i.get("num_threads", 0) for i in info), default=os.cpu_count())
+        blas = ", ".join(sorted({f"{i.get('internal_api')} {i.get('version')}" for i in info
+                                 if i.get("user_api") == "blas"})) or "unknown"
     except Exception:
         cores = os.cpu_count()
     per_bucket = []
@@ -204,7 +208,7 @@ def oracle_sample(wl: W.Workload, steps: int, budget_s: float = 20.0):
                 break
         per_bucket.append(statistics.median(times))
     step_s = sum(b.count * t for b, t in zip(wl.buckets, per_bucket))
-    note = (f"fp64 NumPy oracle, one matrix per bucket "
+    note = (f"fp64 NumPy oracle (BLAS: {blas}; host has {os.cpu_count()} logical cores), one matrix per bucket "
             f"({', '.join(f'{b.m}x{b.n}' for b in wl.buckets)}), median of up to {steps} steps each, "
             f"scaled by bucket counts ({', '.join(str(b.count) for b in wl.buckets)}) to the full "
             f"{wl.params:.4g}-parameter step ({step_s:.1f} s extrapolated)")
