@@ -365,7 +365,7 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     int nl = 0;
     bool done = false;
     cudaError_t e = dion::tc_formb_bq(bp.M, bp.G, Qg, Bg, P0s, cnt, m, n, r, o.max_wait_spins,
-                                      flags, s, &nl, &done);
+                                      flags, sched + 1, s, &nl, &done);
     c.launches += nl;
     if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_formb_bq: %s", cudaGetErrorString(e));
     if (!done) return fail(DION_ERR_CUDA, "tc_formb_bq: %s", dion::tc_map_error());

@@ -810,6 +810,10 @@ namespace tc {
 //   warp 2       TMEM allocator
 //   warps 4..7   epilogue: P0's three-way bf16 split
 //   warps 8..11  converters
+// Tiles of the fused kernel come in order from a global counter through a ring of
+// FB_TILE_RING ids in shared memory: dealt round-robin instead, CTAs drift apart over a
+// long launch and stop sharing DRAM pages.
+constexpr int FB_TILE_RING = 4;
 constexpr int FB_STAGES = 2;
 constexpr int FB_NT = 384;
 constexpr uint32_t FB_F32_BYTES = 2 * 2 * BM * 32 * 4;  // M and G, two 32-column boxes: 64 KB
@@ -822,8 +826,12 @@ struct FusedP {
   bf16* P0s;
   int64_t cs_stride;
   int32_t* flags;
+  int* tile_counter;  // zero before the launch; tiles are taken from it in order
   int64_t max_spins;
 };
+// consumers of the fused kernel's tile ring: MMA issuer, four converter warps, four
+// epilogue warps (the TMA producer fills it)
+constexpr int FB_RING_CONSUMERS = 9;
 
 __global__ void __launch_bounds__(FB_NT, 1)
     k_tc_formb_bq(const __grid_constant__ CUtensorMap tmM, const __grid_constant__ CUtensorMap tmG,
@@ -843,8 +851,11 @@ __global__ void __launch_bounds__(FB_NT, 1)
   uint64_t* tfull = a_empty + FB_STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ring_full = drain + 1;
+  uint64_t* ring_empty = ring_full + FB_TILE_RING;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring_empty + FB_TILE_RING);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);  // FB_TILE_RING tile ids
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_per_mat = p.tiles_m * p.tiles_n;
@@ -864,9 +875,28 @@ __global__ void __launch_bounds__(FB_NT, 1)
       mbar_init(tempty + a, 4);
     }
     mbar_init(drain, 1);
+    for (int s = 0; s < FB_TILE_RING; ++s) {
+      mbar_init(ring_full + s, 1);
+      mbar_init(ring_empty + s, FB_RING_CONSUMERS);
+    }
     *abort = 0;
     fence_mbar_init();
   }
+  // next tile id from the ring (-1: none left); a warp-wide call when `warp_wide`
+  int ring_slot = 0;
+  uint32_t ring_phase = 0;
+  auto next_tile = [&](bool warp_wide) -> int {
+    int t = -2;
+    if (!warp_wide || lane == 0) {
+      if (wait_bounded(ring_full + ring_slot, ring_phase, p.max_spins, abort)) {
+        t = ring[ring_slot];
+        mbar_arrive(ring_empty + ring_slot);
+      }
+    }
+    if (warp_wide) t = __shfl_sync(0xffffffffu, t, 0);
+    if (++ring_slot == FB_TILE_RING) { ring_slot = 0; ring_phase ^= 1; }
+    return t;  // -2: gave up
+  };
   if (warp == 2) {
     tmem_alloc(tmem_slot, p.tmem_cols);
     tmem_relinquish();
@@ -881,9 +911,17 @@ __global__ void __launch_bounds__(FB_NT, 1)
     prefetch_map(&tmM);
     prefetch_map(&tmG);
     prefetch_map(&tmQ);
-    int stage = 0, used = 0;
-    uint32_t phase = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    int stage = 0, used = 0, slot = 0;
+    uint32_t phase = 0, rphase = 0;
+    while (true) {
+      // take the next tile in order and publish it to the other roles
+      if (!wait_bounded(ring_empty + slot, rphase ^ 1, p.max_spins, abort)) break;
+      int t = atomicAdd(p.tile_counter, 1);
+      if (t >= ntiles) t = -1;
+      ring[slot] = t;
+      mbar_arrive(ring_full + slot);
+      if (++slot == FB_TILE_RING) { slot = 0; rphase ^= 1; }
+      if (t < 0) break;
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
       const int m0 = (rem / p.tiles_n) * BM;
@@ -917,7 +955,7 @@ __global__ void __launch_bounds__(FB_NT, 1)
     // ---------------- MMA issuer
     int stage = 0, lt = 0;
     uint32_t phase = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+    for (int t = next_tile(false); t >= 0; t = next_tile(false), ++lt) {
       const int acc = lt & 1;
       if (!wait_bounded(tempty + acc, ((lt >> 1) & 1) ^ 1, p.max_spins, abort)) break;
       tc_fence_after();
@@ -948,14 +986,16 @@ __global__ void __launch_bounds__(FB_NT, 1)
     const int row = cw * 32 + lane;
     int stage = 0;
     uint32_t phase = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    for (int t = next_tile(true); t >= 0; t = next_tile(true)) {
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
       const int m0 = (rem / p.tiles_n) * BM;
       bool ok = true;
       for (int kb = 0; kb < p.num_kb; ++kb) {
-        if (!wait_bounded(f_full + stage, phase, p.max_spins, abort) ||
-            !wait_bounded(a_empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
+        // warp-uniform outcome: the tile ring is read with warp shuffles
+        const bool w = wait_bounded(f_full + stage, phase, p.max_spins, abort) &&
+                       wait_bounded(a_empty + stage, phase ^ 1, p.max_spins, abort);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         // the store issued from this A stage two k-blocks ago must have read it
         if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
         __syncwarp();
@@ -1002,10 +1042,15 @@ __global__ void __launch_bounds__(FB_NT, 1)
     // ---------------- epilogue: P0's three-way bf16 split
     const int ew = warp - 4;
     int lt = 0;
-    int t = blockIdx.x;
-    for (; t < ntiles; t += gridDim.x, ++lt) {
+    bool ok = true;
+    for (int t = next_tile(true); ; t = next_tile(true), ++lt) {
+      if (t < 0) {
+        ok = t == -1;
+        break;
+      }
       const int acc = lt & 1;
-      if (!wait_bounded(tfull + acc, (lt >> 1) & 1, p.max_spins, abort)) break;
+      const bool w = wait_bounded(tfull + acc, (lt >> 1) & 1, p.max_spins, abort);
+      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }  // warp-uniform
       tc_fence_after();
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
@@ -1037,7 +1082,9 @@ __global__ void __launch_bounds__(FB_NT, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + acc);
     }
-    if (t < ntiles && lane == 0) mark_unfinished(p.flags, t, ntiles, tiles_per_mat, gridDim.x);
+    // tiles are handed out dynamically, so after a give-up every matrix is suspect
+    if ((!ok || *abort) && lane == 0)
+      for (int b = 0; b < p.batch; ++b) atomicOr(p.flags + b, F_TIMEOUT);
   }
   __syncthreads();
   if (warp == 2) {
@@ -1050,7 +1097,8 @@ __global__ void __launch_bounds__(FB_NT, 1)
 
 cudaError_t tc_formb_bq(const float* M, const float* G, const void* Qg, void* Bg, bf16* P0s,
                         int count, int64_t m, int64_t n, int64_t r, int64_t max_spins,
-                        int32_t* flags, cudaStream_t s, int* nlaunch, bool* done) {
+                        int32_t* flags, int* tile_counter, cudaStream_t s, int* nlaunch,
+                        bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
@@ -1073,9 +1121,10 @@ cudaError_t tc_formb_bq(const float* M, const float* G, const void* Qg, void* Bg
   p.P0s = P0s;
   p.cs_stride = (int64_t)count * m * r;
   p.flags = flags;
+  p.tile_counter = tile_counter;
   p.max_spins = max_spins;
   const size_t smem = 1024 + FB_STAGES * (FB_F32_BYTES + FB_A_BYTES + p.b_bytes) +
-                      (6 * FB_STAGES + 5) * 8 + 16;
+                      (6 * FB_STAGES + 5 + 2 * FB_TILE_RING) * 8 + 16 + 4 * FB_TILE_RING;
   cudaError_t e = cudaFuncSetAttribute(k_tc_formb_bq, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

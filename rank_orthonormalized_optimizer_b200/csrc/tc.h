@@ -20,10 +20,11 @@ cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, __nv_bfloat16*
                        cudaStream_t s, int* nlaunch, bool* done);
 // Steps 1 and 2 fused: Bg[b] = bf16(M[b] + G[b]) (written for B^T P) and the
 // three-way bf16 split of P0[b] = Bg[b] Qg[b]^T into P0s ([3][count][m][r]).
+// tile_counter: one int in device memory, zero before the call (tiles are taken from it).
 cudaError_t tc_formb_bq(const float* M, const float* G, const void* Qg, void* Bg,
                         __nv_bfloat16* P0s, int count, int64_t m, int64_t n, int64_t r,
-                        int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
-                        bool* done);
+                        int64_t max_spins, int32_t* flags, int* tile_counter, cudaStream_t s,
+                        int* nlaunch, bool* done);
 // R[b] (n x r, fp32) = Bg[b]^T (n x m) * Pg[b] (m x r, bf16).  When colsq is not null it
 // receives the sums of squares of R's columns over blocks of R's rows, fixed order:
 // colsq[b][i][j] for row block i < tc_btp_col_splits(n) (the partials of Q = colnorm(R)).
