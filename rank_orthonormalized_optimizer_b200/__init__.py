@@ -31,7 +31,7 @@ c_int32, c_int64, c_float, c_void_p, c_size_t = (ctypes.c_int32, ctypes.c_int64,
 
 # status codes and bits, mirrored from include/dion.h
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_WORKSPACE_TOO_SMALL, ERR_CUDA, \
-    ERR_NOT_INITIALIZED, ERR_DEVICE, ERR_MISALIGNED = range(8)
+    ERR_NOT_INITIALIZED, ERR_DEVICE, ERR_MISALIGNED, ERR_HOST = range(9)
 MAT_OK, MAT_FALLBACK, MAT_CHOLQR2, MAT_NONFINITE, MAT_TIMEOUT, MAT_ZERO_COLUMN = 0, 1, 2, 4, 8, 16
 PRECISIONS = {"fp32": 0, "bf16": 1}
 ORTH_MODES = {"auto": 0, "cholqr": 1, "cholqr2": 2, "householder": 3}

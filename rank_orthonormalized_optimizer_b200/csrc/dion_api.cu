@@ -23,16 +23,27 @@
 
 namespace {
 
-thread_local std::string tl_error;
+thread_local char tl_error[512];  // a fixed buffer: recording an error never allocates
 
 dion_status fail(dion_status s, const char* fmt, ...) {
-  char buf[512];
   va_list ap;
   va_start(ap, fmt);
-  vsnprintf(buf, sizeof(buf), fmt, ap);
+  vsnprintf(tl_error, sizeof(tl_error), fmt, ap);
   va_end(ap);
-  tl_error = buf;
   return s;
+}
+
+// No C++ exception crosses the C ABI: the entry points that allocate host memory (plans,
+// events, streams, graphs) catch what escapes and report it.
+template <class F>
+dion_status guarded(const char* where, F&& f) {
+  try {
+    return f();
+  } catch (const std::exception& e) {
+    return fail(DION_ERR_HOST, "%s: host-side failure: %s", where, e.what());
+  } catch (...) {
+    return fail(DION_ERR_HOST, "%s: host-side failure", where);
+  }
 }
 
 constexpr uint64_t kMagic = 0x44494f4e42323030ull;  // "DIONB200"
@@ -670,12 +681,10 @@ dion_status check_step_args(dion_handle h, const dion_bucket_ptrs* ptrs, int32_t
 namespace dion {
 
 dion_status set_error(dion_status s, const char* fmt, ...) {
-  char buf[512];
   va_list ap;
   va_start(ap, fmt);
-  vsnprintf(buf, sizeof(buf), fmt, ap);
+  vsnprintf(tl_error, sizeof(tl_error), fmt, ap);
   va_end(ap);
-  tl_error = buf;
   return s;
 }
 
@@ -701,7 +710,7 @@ dion_status dion_default_options(dion_options* opt) {
   return DION_OK;
 }
 
-dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const dion_options* opt,
+static dion_status dion_init_impl(const dion_bucket_desc* buckets, int32_t nbuckets, const dion_options* opt,
                       dion_handle* out, size_t* workspace_bytes) {
   if (!out || !workspace_bytes) return fail(DION_ERR_INVALID_ARG, "out or workspace_bytes is NULL");
   *out = nullptr;
@@ -801,7 +810,7 @@ dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const d
   return DION_OK;
 }
 
-dion_status dion_step_batched(dion_handle h, const dion_bucket_ptrs* ptrs, int32_t nbuckets,
+static dion_status dion_step_batched_impl(dion_handle h, const dion_bucket_ptrs* ptrs, int32_t nbuckets,
                               float lr, void* d_workspace, size_t workspace_bytes,
                               int32_t* d_status, void* stream) {
   dion_status st = check_step_args(h, ptrs, nbuckets, d_workspace, workspace_bytes, d_status);
@@ -857,7 +866,7 @@ dion_status dion_step_batched(dion_handle h, const dion_bucket_ptrs* ptrs, int32
   return finish(DION_OK);
 }
 
-dion_status dion_step_batched_from_host(dion_handle h, const dion_bucket_ptrs* ptrs,
+static dion_status dion_step_batched_from_host_impl(dion_handle h, const dion_bucket_ptrs* ptrs,
                                         const float* const* host_grads, int32_t nbuckets,
                                         float lr, void* d_workspace, size_t workspace_bytes,
                                         int32_t* d_status, int32_t* host_status, void* stream) {
@@ -884,7 +893,7 @@ dion_status dion_step_batched_from_host(dion_handle h, const dion_bucket_ptrs* p
   return DION_OK;
 }
 
-dion_status dion_free(dion_handle h) {
+static dion_status dion_free_impl(dion_handle h) {
   if (!h) return DION_OK;
   if (!valid(h)) return fail(DION_ERR_NOT_INITIALIZED, "invalid or freed handle");
   for (auto& ep : h->events) {
@@ -912,18 +921,19 @@ const char* dion_status_string(dion_status s) {
     case DION_ERR_NOT_INITIALIZED: return "handle not initialized";
     case DION_ERR_DEVICE: return "unsupported device";
     case DION_ERR_MISALIGNED: return "misaligned pointer";
+    case DION_ERR_HOST: return "host-side failure (host memory)";
   }
   return "unknown status";
 }
 
-const char* dion_last_error(void) { return tl_error.c_str(); }
+const char* dion_last_error(void) { return tl_error; }
 
 int64_t dion_num_matrices(dion_handle h) { return valid(h) ? h->total_mats : -1; }
 
 int32_t dion_last_launch_count(dion_handle h) { return valid(h) ? h->last_launches : -1; }
 
-dion_status dion_workspace_view(dion_handle h, int32_t bucket, int32_t which, void* d_workspace,
-                                void** d_ptr, size_t* bytes) {
+static dion_status dion_workspace_view_impl(dion_handle h, int32_t bucket, int32_t which,
+                                            void* d_workspace, void** d_ptr, size_t* bytes) {
   if (!valid(h)) return fail(DION_ERR_NOT_INITIALIZED, "invalid or freed handle");
   if (!d_ptr || !bytes || !d_workspace) return fail(DION_ERR_INVALID_ARG, "NULL argument");
   if (bucket < 0 || bucket >= (int32_t)h->plans.size())
@@ -942,7 +952,7 @@ dion_status dion_workspace_view(dion_handle h, int32_t bucket, int32_t which, vo
   return DION_OK;
 }
 
-dion_status dion_profile_enable(dion_handle h, int32_t on) {
+static dion_status dion_profile_enable_impl(dion_handle h, int32_t on) {
   if (!valid(h)) return fail(DION_ERR_NOT_INITIALIZED, "invalid or freed handle");
   h->profiling = on != 0;
   h->events_used = 0;
@@ -950,7 +960,8 @@ dion_status dion_profile_enable(dion_handle h, int32_t on) {
   return DION_OK;
 }
 
-dion_status dion_profile_read(dion_handle h, double* ms, int64_t* launches, int32_t nclasses) {
+static dion_status dion_profile_read_impl(dion_handle h, double* ms, int64_t* launches,
+                                          int32_t nclasses) {
   if (!valid(h)) return fail(DION_ERR_NOT_INITIALIZED, "invalid or freed handle");
   if (!ms || nclasses < 1) return fail(DION_ERR_INVALID_ARG, "ms is NULL or nclasses < 1");
   for (size_t i = 0; i < h->events_used; ++i) {
@@ -969,6 +980,50 @@ dion_status dion_profile_read(dion_handle h, double* ms, int64_t* launches, int3
     if (launches) launches[i] = h->prof_launches[i];
   }
   return DION_OK;
+}
+
+dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const dion_options* opt,
+                      dion_handle* out, size_t* workspace_bytes) {
+  return guarded("dion_init",
+                 [&] { return dion_init_impl(buckets, nbuckets, opt, out, workspace_bytes); });
+}
+
+dion_status dion_step_batched(dion_handle h, const dion_bucket_ptrs* ptrs, int32_t nbuckets,
+                              float lr, void* d_workspace, size_t workspace_bytes,
+                              int32_t* d_status, void* stream) {
+  return guarded("dion_step_batched", [&] {
+    return dion_step_batched_impl(h, ptrs, nbuckets, lr, d_workspace, workspace_bytes, d_status,
+                                  stream);
+  });
+}
+
+dion_status dion_step_batched_from_host(dion_handle h, const dion_bucket_ptrs* ptrs,
+                                        const float* const* host_grads, int32_t nbuckets,
+                                        float lr, void* d_workspace, size_t workspace_bytes,
+                                        int32_t* d_status, int32_t* host_status, void* stream) {
+  return guarded("dion_step_batched_from_host", [&] {
+    return dion_step_batched_from_host_impl(h, ptrs, host_grads, nbuckets, lr, d_workspace,
+                                            workspace_bytes, d_status, host_status, stream);
+  });
+}
+
+dion_status dion_free(dion_handle h) {
+  return guarded("dion_free", [&] { return dion_free_impl(h); });
+}
+
+dion_status dion_workspace_view(dion_handle h, int32_t bucket, int32_t which, void* d_workspace,
+                                void** out, size_t* bytes) {
+  return guarded("dion_workspace_view",
+                 [&] { return dion_workspace_view_impl(h, bucket, which, d_workspace, out, bytes); });
+}
+
+dion_status dion_profile_enable(dion_handle h, int32_t on) {
+  return guarded("dion_profile_enable", [&] { return dion_profile_enable_impl(h, on); });
+}
+
+dion_status dion_profile_read(dion_handle h, double* ms, int64_t* launches, int32_t nclasses) {
+  return guarded("dion_profile_read",
+                 [&] { return dion_profile_read_impl(h, ms, launches, nclasses); });
 }
 
 }  // extern "C"

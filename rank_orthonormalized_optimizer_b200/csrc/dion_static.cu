@@ -47,9 +47,8 @@ dion_status scratch_for_current_device(void** out) {
 
 }  // namespace
 
-extern "C" dion_status dion_step_batched_noalloc(dion_handle h, const dion_bucket_ptrs* ptrs,
-                                                 int32_t nbuckets, float lr, int32_t* d_status,
-                                                 void* stream) {
+static dion_status noalloc_impl(dion_handle h, const dion_bucket_ptrs* ptrs, int32_t nbuckets,
+                                float lr, int32_t* d_status, void* stream) {
   size_t need = 0;
   dion_status st = dion::plan_workspace_bytes(h, &need);
   if (st != DION_OK) return st;
@@ -63,4 +62,14 @@ extern "C" dion_status dion_step_batched_noalloc(dion_handle h, const dion_bucke
   if (st != DION_OK) return st;
   return dion_step_batched(h, ptrs, nbuckets, lr, scratch, DION_STATIC_SCRATCH_BYTES, d_status,
                            stream);
+}
+
+extern "C" dion_status dion_step_batched_noalloc(dion_handle h, const dion_bucket_ptrs* ptrs,
+                                                 int32_t nbuckets, float lr, int32_t* d_status,
+                                                 void* stream) {
+  try {  // no C++ exception leaves the library (the lock can throw)
+    return noalloc_impl(h, ptrs, nbuckets, lr, d_status, stream);
+  } catch (...) {
+    return dion::set_error(DION_ERR_HOST, "dion_step_batched_noalloc: host-side failure");
+  }
 }

@@ -165,8 +165,8 @@ def test_step_argument_checks_without_device():
 
 
 def test_status_strings_and_views():
-    for code in range(8):
-        assert dion.dion_status_string(code)
+    for code in range(9):
+        assert dion.dion_status_string(code) and dion.dion_status_string(code) != b"unknown status"
     c, h, ws = _init([(3, 64, 32, 16)])
     ptr, nb = ctypes.c_void_p(), ctypes.c_size_t()
     assert dion.dion_workspace_view(h, 0, dion.VIEW_P, 1 << 20, ctypes.byref(ptr),
