@@ -128,6 +128,9 @@ EDGE = [
     # r > 256: the recursive factorisation, with a last block of 16 (272 = 256 + 16;
     # 784 = 512 + 272) and row counts that are not multiples of the 128-row tiles
     ("recursive_chol", [(2, 600, 560, 272), (2, 1100, 800, 784)]),
+    # r <= 256 with m over 512 rows: the Gram adds 512-row K chunks in fp32 (3 chunks,
+    # the last ragged; 5 chunks over a 2 x 2 tile grid with r = 144)
+    ("chunked_gram", [(3, 1300, 96, 64), (2, 2100, 256, 144)]),
 ]
 
 
