@@ -179,6 +179,11 @@ dion_status dion_step_batched(dion_handle h, const dion_bucket_ptrs* ptrs,
  * device buffer ptrs[b].G (which this call therefore overwrites), runs the
  * step, copies d_status back to host_status (one int32 per matrix), and
  * synchronises `stream` before returning, so host_status is valid on return.
+ * The copies run on a stream owned by the handle, ordered after the work already
+ * on `stream`, one bucket at a time with the largest gradient first; each bucket's
+ * whole step starts on `stream` as soon as its own gradients are on the device, so
+ * the steps of the early buckets overlap the uploads of the later ones (the
+ * results are those of dion_step_batched: buckets are independent).
  */
 dion_status dion_step_batched_from_host(dion_handle h, const dion_bucket_ptrs* ptrs,
                                         const float* const* host_grads, int32_t nbuckets,

@@ -8,11 +8,13 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <new>
+#include <numeric>
 #include <string>
 #include <vector>
 
@@ -98,6 +100,12 @@ struct dion_ctx {
   std::vector<FbGraph> fb;
   cudaStream_t cap;  // stream the loop body is captured on
   int cap_device;
+  // gradient uploads of dion_step_batched_from_host: a copy stream, an event when the
+  // caller's stream lets the uploads start, one event per uploaded bucket
+  int up_device;
+  cudaStream_t up;
+  cudaEvent_t up_start;
+  std::vector<cudaEvent_t> up_done;
 };
 
 namespace {
@@ -637,6 +645,41 @@ bool ensure_side_streams(dion_handle h, size_t want) {
   return true;
 }
 
+void release_upload(dion_handle h) {
+  for (auto ev : h->up_done) cudaEventDestroy(ev);
+  h->up_done.clear();
+  if (h->up_start) cudaEventDestroy(h->up_start);
+  if (h->up) cudaStreamDestroy(h->up);
+  h->up_start = nullptr;
+  h->up = nullptr;
+  h->up_device = -1;
+}
+
+// The copy stream and events of the overlapped gradient upload on the current device.
+bool ensure_upload(dion_handle h, size_t want) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (h->up_device != dev) {
+    release_upload(h);
+    if (cudaStreamCreateWithFlags(&h->up, cudaStreamNonBlocking) != cudaSuccess) {
+      h->up = nullptr;
+      return false;
+    }
+    if (cudaEventCreateWithFlags(&h->up_start, cudaEventDisableTiming) != cudaSuccess) {
+      h->up_start = nullptr;
+      release_upload(h);
+      return false;
+    }
+    h->up_device = dev;
+  }
+  while (h->up_done.size() < want) {
+    cudaEvent_t ev;
+    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return false;
+    h->up_done.push_back(ev);
+  }
+  return true;
+}
+
 dion_status check_device(dion_handle h) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -805,6 +848,9 @@ static dion_status dion_init_impl(const dion_bucket_desc* buckets, int32_t nbuck
   h->fork_ev = nullptr;
   h->cap = nullptr;
   h->cap_device = -1;
+  h->up_device = -1;
+  h->up = nullptr;
+  h->up_start = nullptr;
   *out = h;
   *workspace_bytes = off;
   return DION_OK;
@@ -866,6 +912,64 @@ static dion_status dion_step_batched_impl(dion_handle h, const dion_bucket_ptrs*
   return finish(DION_OK);
 }
 
+// The step with the gradients uploaded bucket by bucket on a copy stream: each bucket's
+// whole step (B Q to update) starts as soon as its own gradients have arrived, so it runs
+// while the later buckets' gradients cross the host link.  Buckets are uploaded largest
+// first, so what is left after the last copy is the step of the smallest bucket.
+static dion_status step_overlapped(dion_handle h, const dion_bucket_ptrs* ptrs,
+                                   const float* const* host_grads, int32_t nbuckets, float lr,
+                                   char* ws, int32_t* d_status, cudaStream_t main) {
+  std::vector<int32_t> order((size_t)nbuckets);
+  std::iota(order.begin(), order.end(), 0);
+  auto grad_bytes = [&](int32_t b) {
+    const Plan& p = h->plans[b];
+    return (size_t)p.count * p.m * p.n * sizeof(float);
+  };
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int32_t a, int32_t b) { return grad_bytes(a) > grad_bytes(b); });
+  // the previous work on the caller's stream (an earlier step) may still read G
+  cudaError_t e = cudaEventRecord(h->up_start, main);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->up, h->up_start, 0);
+  if (e != cudaSuccess) return fail(DION_ERR_CUDA, "upload ordering: %s", cudaGetErrorString(e));
+  for (int32_t k = 0; k < nbuckets; ++k) {
+    const int32_t b = order[k];
+    e = cudaMemcpyAsync(const_cast<float*>(ptrs[b].G), host_grads[b], grad_bytes(b),
+                        cudaMemcpyHostToDevice, h->up);
+    if (e == cudaSuccess) e = cudaEventRecord(h->up_done[k], h->up);
+    if (e != cudaSuccess) {
+      // the caller's stream stays ordered after the copies already issued
+      if (cudaEventRecord(h->up_start, h->up) == cudaSuccess)
+        cudaStreamWaitEvent(main, h->up_start, 0);
+      return fail(DION_ERR_CUDA, "gradient upload: %s", cudaGetErrorString(e));
+    }
+  }
+  StepCtx c{h, main, 0, -1, nullptr, 0, std::vector<int>(nbuckets, 0)};
+  int32_t waited = 0;  // uploads [0, waited) the caller's stream is ordered after
+  auto finish = [&](dion_status result) -> dion_status {
+    end_cls(c);
+    if (waited < nbuckets) cudaStreamWaitEvent(main, h->up_done[nbuckets - 1], 0);
+    h->last_launches = c.launches;
+    return result;
+  };
+  dion_status st;
+  for (int phase : {PH_INIT, PH_PREPQ})
+    for (int32_t b = 0; b < nbuckets; ++b)
+      if ((st = run_bucket(c, b, phase, h->plans[b], ptrs[b], lr, ws, d_status)) != DION_OK)
+        return finish(st);
+  for (int32_t k = 0; k < nbuckets; ++k) {
+    const int32_t b = order[k];
+    if ((e = cudaStreamWaitEvent(main, h->up_done[k], 0)) != cudaSuccess)
+      return finish(fail(DION_ERR_CUDA, "upload wait: %s", cudaGetErrorString(e)));
+    waited = k + 1;
+    for (int phase : {PH_FORMB, PH_BQ, PH_ORTH, PH_BTP, PH_COLNORM, PH_UPDATE, PH_STATUS}) {
+      c.s = main;
+      if ((st = run_bucket(c, b, phase, h->plans[b], ptrs[b], lr, ws, d_status)) != DION_OK)
+        return finish(st);
+    }
+  }
+  return finish(DION_OK);
+}
+
 static dion_status dion_step_batched_from_host_impl(dion_handle h, const dion_bucket_ptrs* ptrs,
                                         const float* const* host_grads, int32_t nbuckets,
                                         float lr, void* d_workspace, size_t workspace_bytes,
@@ -874,16 +978,27 @@ static dion_status dion_step_batched_from_host_impl(dion_handle h, const dion_bu
   if (st != DION_OK) return st;
   if (!host_grads || !host_status || !d_status)
     return fail(DION_ERR_INVALID_ARG, "host_grads, host_status and d_status are required");
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  for (int32_t b = 0; b < nbuckets; ++b) {
+  if (!std::isfinite(lr)) return fail(DION_ERR_INVALID_ARG, "lr is not finite");
+  for (int32_t b = 0; b < nbuckets; ++b)
     if (!host_grads[b]) return fail(DION_ERR_INVALID_ARG, "host_grads[%d] is NULL", b);
-    const Plan& p = h->plans[b];
-    const size_t bytes = (size_t)p.count * p.m * p.n * sizeof(float);
-    cudaError_t e = cudaMemcpyAsync(const_cast<float*>(ptrs[b].G), host_grads[b], bytes,
-                                    cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return fail(DION_ERR_CUDA, "gradient upload: %s", cudaGetErrorString(e));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (ensure_upload(h, (size_t)nbuckets)) {
+    st = step_overlapped(h, ptrs, host_grads, nbuckets, lr, static_cast<char*>(d_workspace),
+                         d_status, s);
+  } else {
+    // no copy stream: upload everything, then step
+    cudaGetLastError();
+    for (int32_t b = 0; b < nbuckets; ++b) {
+      const Plan& p = h->plans[b];
+      const size_t bytes = (size_t)p.count * p.m * p.n * sizeof(float);
+      cudaError_t e = cudaMemcpyAsync(const_cast<float*>(ptrs[b].G), host_grads[b], bytes,
+                                      cudaMemcpyHostToDevice, s);
+      if (e != cudaSuccess)
+        return fail(DION_ERR_CUDA, "gradient upload: %s", cudaGetErrorString(e));
+    }
+    st = dion_step_batched_impl(h, ptrs, nbuckets, lr, d_workspace, workspace_bytes, d_status,
+                                stream);
   }
-  st = dion_step_batched(h, ptrs, nbuckets, lr, d_workspace, workspace_bytes, d_status, stream);
   if (st != DION_OK) return st;
   cudaError_t e = cudaMemcpyAsync(host_status, d_status, (size_t)h->total_mats * sizeof(int32_t),
                                   cudaMemcpyDeviceToHost, s);
@@ -906,6 +1021,7 @@ static dion_status dion_free_impl(dion_handle h) {
   for (auto& g : h->fb)
     if (g.exec) cudaGraphExecDestroy(g.exec);
   if (h->cap) cudaStreamDestroy(h->cap);
+  release_upload(h);
   h->magic = 0;
   delete h;
   return DION_OK;

@@ -282,6 +282,33 @@ def test_deterministic_and_resumable():
         assert torch.equal(a.X[i], d.X[i]) and torch.equal(a.M[i], d.M[i])
 
 
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_step_from_host_equals_device_step(precision):
+    """The host-gradient entry point uploads bucket by bucket (largest first) and steps
+    each bucket as soon as its gradients arrive; over several steps, each overwriting G
+    that the previous step's update read, it gives bitwise the device step's state and
+    status.  The buckets are listed smallest first, so the upload order is not theirs;
+    r = 272 takes the recursive factorisation and the fallback graph."""
+    wl = W.custom("from_host", [(2, 256, 128, 32), (3, 600, 560, 272), (4, 1024, 512, 64)],
+                  precision=precision, steps=3)
+    a = GpuRun(wl)
+    b = GpuRun(wl)
+    nb = len(wl.buckets)
+    host_status = torch.zeros(b.opt.num_matrices, dtype=torch.int32).pin_memory()
+    for t in range(3):
+        grads = [W.gradient(wl, i, t, "cpu") for i in range(nb)]
+        a.step(1, G_override=[g.cuda() for g in grads])
+        pinned = [g.pin_memory() for g in grads]
+        b.opt.step_from_host(b.X, b.M, b.G, b.Q, pinned, wl.lr, b.ws, b.status, host_status)
+        torch.cuda.synchronize()
+        for i in range(nb):
+            assert torch.equal(a.X[i], b.X[i]) and torch.equal(a.M[i], b.M[i]), (t, i)
+            assert torch.equal(a.Q[i], b.Q[i]), (t, i)
+            assert torch.equal(b.G[i].cpu(), grads[i])
+        assert torch.equal(host_status, a.status.cpu()), t
+        assert torch.equal(b.status.cpu(), a.status.cpu()), t
+
+
 def test_tensor_and_simt_paths_agree():
     wl = W.custom("paths", [(6, 1024, 512, 64), (4, 512, 1024, 128)], precision="bf16", steps=3)
     a = GpuRun(wl, kernel_path="tensor")
