@@ -324,7 +324,10 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
   float* P0 = reinterpret_cast<float*>(ws + p.off_P0);
   float* P = reinterpret_cast<float*>(ws + p.off_P);
   float* P2 = reinterpret_cast<float*>(ws + p.off_P2);
-  void* Pg = (bf || split) ? (void*)(ws + p.off_Pg) : (void*)P;
+  // the GEMM copy of P: bf16 on the tensor path is the leading plane of P's three-way
+  // split (both are P rounded to nearest bf16), the split itself in fp32 mode
+  void* Pg = (bf && tensor) ? (void*)(ws + p.off_Ps)
+             : (bf || split) ? (void*)(ws + p.off_Pg) : (void*)P;
   float* W = reinterpret_cast<float*>(ws + p.off_W);
   float* Linv = reinterpret_cast<float*>(ws + p.off_Linv);
   float* dinv = reinterpret_cast<float*>(ws + p.off_dinv);
@@ -489,12 +492,12 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
       if ((st = tc_check(e, "tc_gram")) != DION_OK) return st;
       ca.pass = 1; ca.orth_tol = o.orth_tol;
       if ((st = chol()) != DION_OK) return st;
-      // the first pass writes P and its GEMM copy Pg at once (in split mode Pg is the
-      // split the second pass reads); the finalize then touches only the matrices that
+      // the first pass writes P and its split, which is also the GEMM copy Pg (bf16:
+      // the split's leading plane); the finalize then touches only the matrices that
       // took the second pass or the fallback
       __nv_bfloat16* P1s = split ? reinterpret_cast<__nv_bfloat16*>(Pg) : Ps;
-      e = dion::tc_apply(P0s, Linvs, P, P1s, bf ? reinterpret_cast<__nv_bfloat16*>(Pg) : nullptr,
-                         cnt, m, r, flags, 0, DION_MAT_FALLBACK, o.max_wait_spins, s, &nl, &done);
+      e = dion::tc_apply(P0s, Linvs, P, P1s, nullptr, cnt, m, r, flags, 0, DION_MAT_FALLBACK,
+                         o.max_wait_spins, s, &nl, &done);
       if ((st = tc_check(e, "tc_apply")) != DION_OK) return st;
       pg_ready = true;
       if (o.orth_mode != DION_ORTH_CHOLQR) {
@@ -810,7 +813,8 @@ static dion_status dion_init_impl(const dion_bucket_desc* buckets, int32_t nbuck
     p.off_P0 = take(c * d.m * d.r * 4);
     p.off_P = take(c * d.m * d.r * 4);
     p.off_P2 = take(c * d.m * d.r * 4);
-    p.off_Pg = (bf || split) ? take(c * d.m * d.r * ge) : 0;
+    p.off_Pg = (bf || split) && !(bf && o.kernel_path == DION_PATH_TENSOR)
+                   ? take(c * d.m * d.r * ge) : 0;
     p.off_W = take(c * d.r * d.r * 4);
     p.off_Linv = take(c * d.r * d.r * 4);
     p.off_dinv = take(dion::chol_dinv_floats(d.count, d.r) * 4);

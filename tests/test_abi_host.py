@@ -103,7 +103,9 @@ def test_workspace_covers_the_layout():
     c, h, ws = _init(c4)
     assert c == dion.OK
     bf16_b = sum(k * m * n * 2 for k, m, n, r in c4)
-    factors = sum(k * (m * r * (4 * 3 + 2 + 12) + n * r * (4 + 2 + 2 + 2) + r * r * 14)
+    # per m x r element: P0, P, P2 (fp32) and the splits of P0 and P (the bf16 GEMM
+    # copy of P is the leading plane of P's split)
+    factors = sum(k * (m * r * (4 * 3 + 12) + n * r * (4 + 2 + 2 + 2) + r * r * 14)
                   for k, m, n, r in c4)
     assert bf16_b + factors <= ws < 1.1 * (bf16_b + factors) + (1 << 24)
     assert dion.dion_num_matrices(h) == 224
@@ -116,8 +118,9 @@ def test_workspace_covers_the_layout():
 def test_workspace_recursive_factorisation_scratch():
     # r > 256 on the tensor path: two more [3][count][r][r] bf16 splits (the Gram's and
     # L21's) for the recursive Cholesky factorisation; none at r <= 256, none on the
-    # CUDA-core path.  With bf16 GEMM inputs the plans differ otherwise only in the
-    # column-norm partials: one per block of up to 256 rows of R (written by B^T P) on
+    # CUDA-core path.  With bf16 GEMM inputs the plans differ otherwise only in the bf16
+    # copy of P (on the tensor path the leading plane of P's split) and the column-norm
+    # partials: one per block of up to 256 rows of R (written by B^T P) on
     # the tensor path, min(ceil(8 * 148 / count), ceil(n / 16), 256) row ranges on the
     # CUDA-core path.
     def ws_of(r, path):
@@ -132,7 +135,8 @@ def test_workspace_recursive_factorisation_scratch():
 
     for r in (256, 512):
         extra = 2 * 8 * r * r * 6 if r > 256 else 0
-        assert ws_of(r, 0) - ws_of(r, 1) == extra + parts(r, 0) - parts(r, 1)
+        pg = 8 * 1024 * r * 2               # the CUDA-core path's own bf16 copy of P
+        assert ws_of(r, 0) - ws_of(r, 1) == extra - pg + parts(r, 0) - parts(r, 1)
 
 
 def test_step_argument_checks_without_device():
