@@ -329,6 +329,11 @@ def run_ours(args):
         del Gh
         _ = time.perf_counter() - t_start
 
+    if not args.no_vector:
+        del ws
+        torch.cuda.empty_cache()
+        result["vector_step"] = measure_vector_step(dev, stream, peaks)
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, step_s, cores, note = oracle_sample(wl, steps=2)
         result["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -339,6 +344,61 @@ def run_ours(args):
     import torch.distributed as dist
     if dist.is_initialized():
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------ vector (1-D) parameters
+VEC_BYTES = {"adamw": 28, "lion": 20}   # per element: AdamW reads x, g, m, v and writes
+                                        # x, m, v; Lion reads x, g, m and writes x, m
+
+
+def measure_vector_step(dev, stream, peaks, warmup=3, iters=10):
+    """AdamW and Lion over the vector parameters (dion_vec_step): a bank of 64 x 4 Mi
+    elements (4 GiB of state, far larger than L2) against the copy bandwidth, and the
+    65 RMSNorm gains of the 7B-like decoder (L2-resident, launch-bound)."""
+    import torch
+
+    from rank_orthonormalized_optimizer_b200 import vec_step
+    out = {}
+    for name, reps in (("vectors_64x4Mi", iters), ("norms_h4096_l32", 20 * iters)):
+        vw = W.VECTOR_WORKLOADS[name]
+        n = vw.params
+        flat = {k: torch.empty(n, dtype=torch.float32, device=dev) for k in "xgmv"}
+        views = {k: [] for k in "xgmv"}
+        off = 0
+        for i, sz in enumerate(vw.sizes):
+            vals = W.vector_state(vw, i, 0, dev)
+            for k, t in zip("xgmv", vals):
+                flat[k][off:off + sz].copy_(t)
+                views[k].append(flat[k][off:off + sz])
+            off += sz
+        rec = {"elements": n, "tensors": len(vw.sizes)}
+        for rule in ("adamw", "lion"):
+            v = views["v"] if rule == "adamw" else None
+            with torch.cuda.stream(stream):
+                for t in range(warmup):
+                    vec_step(views["x"], views["g"], views["m"], v, rule=rule, step=t + 1,
+                             stream=stream)
+                barrier(dev)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                launches = 0
+                for t in range(reps):
+                    launches += vec_step(views["x"], views["g"], views["m"], v, rule=rule,
+                                         step=warmup + t + 1, stream=stream)
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = max_over_ranks(e0.elapsed_time(e1) / reps, dev)
+            gbs = VEC_BYTES[rule] * n / (ms * 1e-3) / 1e9
+            rec[rule] = {"us": ms * 1e3, "launches_per_step": launches // reps,
+                         "bytes_per_element": VEC_BYTES[rule], "achieved_GBs": gbs,
+                         "frac_of_measured_copy": gbs / peaks["hbm_gbs"]}
+        rec["l2"] = ("state (%.1f GB) far larger than L2" % (16 * n / 1e9) if n * 16 > 1 << 30
+                     else "state resident in L2 (%.1f MB); launch-bound" % (16 * n / 1e6))
+        out[name] = rec
+        del flat, views
+        torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------------------ the oracle arm
@@ -380,6 +440,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-vector", action="store_true",
+                    help="skip the AdamW / Lion step of the vector parameters")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -264,6 +264,73 @@ dion_status dion_profile_enable(dion_handle h, int32_t on);
 dion_status dion_profile_read(dion_handle h, double* ms, int64_t* launches,
                               int32_t nclasses);
 
+/*
+ * ---------------------------------------------------------------------------
+ * The step of the vector (1-D) parameters.  Dion takes only the 2-D weight
+ * matrices; biases and normalisation gains go to AdamW or Lion (paragraph 5 of
+ * the rivista.ai article).  The article names the two rules without writing them;
+ * they are taken as published:
+ *
+ *   DION_VEC_ADAMW -- "Decoupled Weight Decay Regularization" (Loshchilov and
+ *   Hutter), decoupled decay first, then the bias-corrected Adam step, t >= 1:
+ *     x <- x (1 - lr wd)
+ *     m <- b1 m + (1 - b1) g;        v <- b2 v + (1 - b2) g^2
+ *     x <- x - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ *
+ *   DION_VEC_LION -- "Symbolic Discovery of Optimization Algorithms" (Chen et
+ *   al.), the sign of an interpolation of momentum and gradient:
+ *     c = b1 m + (1 - b1) g
+ *     x <- x (1 - lr wd) - lr sign(c)            sign(0) = 0
+ *     m <- b2 m + (1 - b2) g
+ *   Because sign(c) is a discrete decision, c is fixed to fp32 arithmetic with
+ *   no fused multiply-add: 1 - b1 is rounded to fp32, then each product and the
+ *   sum are rounded to fp32 (round to nearest even).
+ *
+ * State and arithmetic are fp32.  One call updates a list of tensors, each a
+ * contiguous array with its own state; the elements are independent.  Non-finite
+ * gradients are not checked: they make the affected elements non-finite.
+ */
+typedef enum dion_vec_rule { DION_VEC_ADAMW = 0, DION_VEC_LION = 1 } dion_vec_rule;
+
+typedef struct dion_vec_tensor {
+  float* x;         /* parameter, updated in place                                */
+  const float* g;   /* gradient, read only                                        */
+  float* m;         /* first moment (both rules), updated in place                */
+  float* v;         /* second moment (AdamW; not read by Lion, may be NULL there)  */
+  int64_t numel;    /* elements; a tensor with 0 elements is skipped (its pointers
+                       may then be NULL)                                          */
+} dion_vec_tensor;
+
+typedef struct dion_vec_options {
+  int32_t rule;        /* DION_VEC_ADAMW or DION_VEC_LION                         */
+  float lr;            /* learning rate, finite                                   */
+  float beta1, beta2;  /* in [0, 1)                                               */
+  float eps;           /* AdamW: added to the bias-corrected sqrt(v), > 0         */
+  float weight_decay;  /* decoupled decay, finite and >= 0                        */
+  int64_t step;        /* AdamW: this step's number t >= 1 (bias correction)      */
+} dion_vec_options;
+
+/* Defaults of the two papers: AdamW lr 1e-3, betas (0.9, 0.999), eps 1e-8,
+ * weight decay 0.01, step 1; Lion lr 1e-4, betas (0.9, 0.99), weight decay 0. */
+dion_status dion_vec_default_options(int32_t rule, dion_vec_options* o);
+
+/*
+ * One step of every tensor of tensors[0 .. ntensors), enqueued on `stream` of the
+ * current device; returns as soon as the work is enqueued.  tensors is a host
+ * array of device pointer sets.  Every pointer must be 4-byte aligned (16-byte
+ * alignment of x, g, m, v at the same offset takes a vectorised path); x, g, m
+ * and v of one tensor, and different tensors, must not overlap.  The arguments
+ * are checked before anything is enqueued (DION_ERR_INVALID_ARG,
+ * DION_ERR_MISALIGNED, DION_ERR_DEVICE); no handle and no workspace are needed.
+ * Up to 64 tensors go into one kernel launch; longer lists take several
+ * launches on the same stream.
+ */
+dion_status dion_vec_step(const dion_vec_tensor* tensors, int32_t ntensors,
+                          const dion_vec_options* o, void* stream);
+
+/* Kernel launches made by the most recent dion_vec_step on this thread. */
+int32_t dion_vec_last_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -56,6 +56,19 @@ class BucketPtrs(ctypes.Structure):
     _fields_ = [("X", c_void_p), ("M", c_void_p), ("G", c_void_p), ("Q", c_void_p)]
 
 
+VEC_RULES = {"adamw": 0, "lion": 1}
+
+
+class VecTensor(ctypes.Structure):
+    _fields_ = [("x", c_void_p), ("g", c_void_p), ("m", c_void_p), ("v", c_void_p),
+                ("numel", c_int64)]
+
+
+class VecOptions(ctypes.Structure):
+    _fields_ = [("rule", c_int32), ("lr", c_float), ("beta1", c_float), ("beta2", c_float),
+                ("eps", c_float), ("weight_decay", c_float), ("step", c_int64)]
+
+
 def _sig(name, restype, *args):
     f = getattr(_lib, name)
     f.restype = restype
@@ -74,6 +87,11 @@ dion_step_batched_from_host = _sig("dion_step_batched_from_host", c_int32, c_voi
 dion_step_batched_noalloc = _sig("dion_step_batched_noalloc", c_int32, c_void_p,
                                  ctypes.POINTER(BucketPtrs), c_int32, c_float, c_void_p, c_void_p)
 dion_free = _sig("dion_free", c_int32, c_void_p)
+dion_vec_default_options = _sig("dion_vec_default_options", c_int32, c_int32,
+                                ctypes.POINTER(VecOptions))
+dion_vec_step = _sig("dion_vec_step", c_int32, ctypes.POINTER(VecTensor), c_int32,
+                     ctypes.POINTER(VecOptions), c_void_p)
+dion_vec_last_launch_count = _sig("dion_vec_last_launch_count", c_int32)
 dion_status_string = _sig("dion_status_string", ctypes.c_char_p, c_int32)
 dion_last_error = _sig("dion_last_error", ctypes.c_char_p)
 dion_num_matrices = _sig("dion_num_matrices", c_int64, c_void_p)
@@ -88,7 +106,8 @@ dion_profile_read = _sig("dion_profile_read", c_int32, c_void_p, ctypes.POINTER(
 EXPORTED = ["dion_default_options", "dion_init", "dion_step_batched",
             "dion_step_batched_from_host", "dion_step_batched_noalloc", "dion_free", "dion_status_string", "dion_last_error",
             "dion_num_matrices", "dion_last_launch_count", "dion_workspace_view",
-            "dion_profile_enable", "dion_profile_read"]
+            "dion_profile_enable", "dion_profile_read", "dion_vec_default_options",
+            "dion_vec_step", "dion_vec_last_launch_count"]
 
 
 class DionError(RuntimeError):
@@ -252,3 +271,49 @@ class DionB200:
             self.close()
         except Exception:
             pass
+
+
+# ---------------------------------------------------------------- vector parameters
+def vec_default_options(rule: str = "adamw") -> VecOptions:
+    o = VecOptions()
+    _check(dion_vec_default_options(VEC_RULES[rule], ctypes.byref(o)), "dion_vec_default_options")
+    return o
+
+
+def vec_step(x, g, m, v=None, *, rule="adamw", lr=None, betas=None, eps=None,
+             weight_decay=None, step=1, stream=None):
+    """One AdamW or Lion step of the vector (1-D) parameters, on the CUDA library.
+
+    ``x``, ``g``, ``m`` (and ``v`` for AdamW): equal-length lists of contiguous fp32
+    CUDA tensors, one entry per parameter; x, m, v are updated in place.  Options left
+    as None take the defaults of include/dion.h (dion_vec_default_options); ``step`` is
+    the AdamW step number t >= 1.  Returns the number of kernel launches.
+    """
+    import torch
+    o = vec_default_options(rule)
+    if lr is not None:
+        o.lr = lr
+    if betas is not None:
+        o.beta1, o.beta2 = betas
+    if eps is not None:
+        o.eps = eps
+    if weight_decay is not None:
+        o.weight_decay = weight_decay
+    o.step = int(step)
+    n = len(x)
+    if v is None:
+        v = [None] * n
+    if not (len(g) == len(m) == len(v) == n):
+        raise ValueError("x, g, m and v must have one entry per parameter")
+    arr = (VecTensor * max(n, 1))()
+    for i in range(n):
+        for name, t in (("x", x[i]), ("g", g[i]), ("m", m[i])) + ((("v", v[i]),) if rule == "adamw" else ()):
+            if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 \
+                    or not t.is_contiguous() or t.numel() != x[i].numel():
+                raise ValueError(f"parameter {i}: {name} must be a contiguous fp32 CUDA tensor "
+                                 f"of {x[i].numel()} elements")
+        arr[i].x, arr[i].g, arr[i].m = x[i].data_ptr(), g[i].data_ptr(), m[i].data_ptr()
+        arr[i].v = v[i].data_ptr() if v[i] is not None else None
+        arr[i].numel = x[i].numel()
+    _check(dion_vec_step(arr, n, ctypes.byref(o), DionB200._stream(stream)), "dion_vec_step")
+    return dion_vec_last_launch_count()

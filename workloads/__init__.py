@@ -102,7 +102,7 @@ WORKLOADS = {
 #: the workload a throughput figure is quoted on (7B-like transformer shapes)
 HEADLINE = "transformer_h4096_l32_ff11008_r256"
 
-_KINDS = {"X": 1, "Q": 2, "G": 3, "U": 4, "V": 5, "M": 6}
+_KINDS = {"X": 1, "Q": 2, "G": 3, "U": 4, "V": 5, "M": 6, "S": 7}
 
 
 def seed_for(workload: str, bucket: int, slot: int, kind: str, step: int = 0) -> int:
@@ -209,3 +209,36 @@ def custom(name: str, buckets, precision="fp32", mu=0.95, lr=0.01, steps=3,
     """A small ad-hoc workload (odd shapes for edge-case tests)."""
     return Workload(name=name, buckets=tuple(Bucket(*b) for b in buckets),
                     precision=precision, mu=mu, lr=lr, steps=steps, grad=grad)
+
+
+# ------------------------------------------------------------ vector (1-D) parameters
+@dataclass(frozen=True)
+class VectorWorkload:
+    """The 1-D parameters of a model (biases, normalisation gains), one entry per
+    parameter tensor, stepped by AdamW or Lion beside the Dion step of its matrices."""
+    name: str
+    sizes: tuple
+    lr: float = 1e-3
+
+    @property
+    def params(self) -> int:
+        return sum(self.sizes)
+
+
+VECTOR_WORKLOADS = {
+    # the RMSNorm gains of the 7B-like decoder: two per layer and the final one
+    "norms_h4096_l32": VectorWorkload("norms_h4096_l32", (4096,) * 65),
+    # a bank larger than L2 (64 x 4 Mi elements, 1 GiB per state array)
+    "vectors_64x4Mi": VectorWorkload("vectors_64x4Mi", (4 << 20,) * 64),
+}
+
+
+def vector_state(vw: VectorWorkload, i: int, step: int = 0, device="cpu"):
+    """(x, g, m, v) of parameter i, fp32 1-D: x ~ N(0, 1), g ~ 1e-3 N(0, 1) fresh each
+    step, m ~ 1e-3 N(0, 1), v = (1e-3 N(0, 1))^2 (non-negative, as a second moment)."""
+    n = vw.sizes[i]
+    x = _randn((n,), seed_for(vw.name, i, 0, "X"), device)
+    g = _randn((n,), seed_for(vw.name, i, 0, "G", step), device) * 1e-3
+    m = _randn((n,), seed_for(vw.name, i, 0, "M"), device) * 1e-3
+    v = (_randn((n,), seed_for(vw.name, i, 0, "S"), device) * 1e-3) ** 2
+    return x, g, m, v
