@@ -352,12 +352,15 @@ VEC_BYTES = {"adamw": 28, "lion": 20}   # per element: AdamW reads x, g, m, v an
 
 
 def measure_vector_step(dev, stream, peaks, warmup=3, iters=10):
-    """AdamW and Lion over the vector parameters (dion_vec_step): a bank of 64 x 4 Mi
-    elements (4 GiB of state, far larger than L2) against the copy bandwidth, and the
-    65 RMSNorm gains of the 7B-like decoder (L2-resident, launch-bound)."""
+    """AdamW and Lion over the vector parameters (dion_vec_step through a prepared
+    VecStepPlan): a bank of 64 x 4 Mi elements (4 GiB of state, far larger than L2)
+    against the copy bandwidth, and the 65 RMSNorm gains of the 7B-like decoder
+    (L2-resident): per call through the C ABI, where the host's call and launch cost
+    dominates, and with the calls enqueued ahead of the device, which leaves the
+    device time."""
     import torch
 
-    from rank_orthonormalized_optimizer_b200 import vec_step
+    from rank_orthonormalized_optimizer_b200 import VecStepPlan
     out = {}
     for name, reps in (("vectors_64x4Mi", iters), ("norms_h4096_l32", 20 * iters)):
         vw = W.VECTOR_WORKLOADS[name]
@@ -373,26 +376,37 @@ def measure_vector_step(dev, stream, peaks, warmup=3, iters=10):
             off += sz
         rec = {"elements": n, "tensors": len(vw.sizes)}
         for rule in ("adamw", "lion"):
-            v = views["v"] if rule == "adamw" else None
-            with torch.cuda.stream(stream):
-                for t in range(warmup):
-                    vec_step(views["x"], views["g"], views["m"], v, rule=rule, step=t + 1,
-                             stream=stream)
-                barrier(dev)
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                launches = 0
-                for t in range(reps):
-                    launches += vec_step(views["x"], views["g"], views["m"], v, rule=rule,
-                                         step=warmup + t + 1, stream=stream)
-                e1.record(stream)
+            plan = VecStepPlan(views["x"], views["g"], views["m"],
+                               views["v"] if rule == "adamw" else None, rule=rule)
+            for t in range(warmup):
+                plan.step(t + 1, stream)
+            barrier(dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            launches = 0
+            for t in range(reps):
+                launches += plan.step(warmup + t + 1, stream)
+            e1.record(stream)
             torch.cuda.synchronize(dev)
             ms = max_over_ranks(e0.elapsed_time(e1) / reps, dev)
             gbs = VEC_BYTES[rule] * n / (ms * 1e-3) / 1e9
-            rec[rule] = {"us": ms * 1e3, "launches_per_step": launches // reps,
-                         "bytes_per_element": VEC_BYTES[rule], "achieved_GBs": gbs,
-                         "frac_of_measured_copy": gbs / peaks["hbm_gbs"]}
+            r = {"us": ms * 1e3, "launches_per_step": launches // reps,
+                 "bytes_per_element": VEC_BYTES[rule], "achieved_GBs": gbs,
+                 "frac_of_measured_copy": gbs / peaks["hbm_gbs"]}
+            if n * 16 <= 1 << 30:
+                # the same calls with the host ahead of the device: a bounded spin kernel
+                # (about 20 ms) holds the stream while every call is enqueued, so the
+                # events bracket the launches back to back (device time per call)
+                with torch.cuda.stream(stream):
+                    torch.cuda._sleep(40_000_000)
+                e0.record(stream)
+                for t in range(reps):
+                    plan.step(warmup + reps + t + 1, stream)
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                r["queued_us"] = max_over_ranks(e0.elapsed_time(e1) / reps, dev) * 1e3
+            rec[rule] = r
         rec["l2"] = ("state (%.1f GB) far larger than L2" % (16 * n / 1e9) if n * 16 > 1 << 30
                      else "state resident in L2 (%.1f MB); launch-bound" % (16 * n / 1e6))
         out[name] = rec

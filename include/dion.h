@@ -322,7 +322,7 @@ dion_status dion_vec_default_options(int32_t rule, dion_vec_options* o);
  * and v of one tensor, and different tensors, must not overlap.  The arguments
  * are checked before anything is enqueued (DION_ERR_INVALID_ARG,
  * DION_ERR_MISALIGNED, DION_ERR_DEVICE); no handle and no workspace are needed.
- * Up to 64 tensors go into one kernel launch; longer lists take several
+ * Up to 128 tensors go into one kernel launch; longer lists take several
  * launches on the same stream.
  */
 dion_status dion_vec_step(const dion_vec_tensor* tensors, int32_t ntensors,

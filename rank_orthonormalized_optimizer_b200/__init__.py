@@ -280,40 +280,59 @@ def vec_default_options(rule: str = "adamw") -> VecOptions:
     return o
 
 
-def vec_step(x, g, m, v=None, *, rule="adamw", lr=None, betas=None, eps=None,
-             weight_decay=None, step=1, stream=None):
-    """One AdamW or Lion step of the vector (1-D) parameters, on the CUDA library.
+class VecStepPlan:
+    """A fixed list of vector (1-D) parameters and their state, marshalled once.
 
     ``x``, ``g``, ``m`` (and ``v`` for AdamW): equal-length lists of contiguous fp32
-    CUDA tensors, one entry per parameter; x, m, v are updated in place.  Options left
-    as None take the defaults of include/dion.h (dion_vec_default_options); ``step`` is
-    the AdamW step number t >= 1.  Returns the number of kernel launches.
+    CUDA tensors, one entry per parameter; they must stay allocated while the plan is
+    used.  ``step`` then costs one C call (dion_vec_step) and its launches.  Options
+    left as None take the defaults of include/dion.h (dion_vec_default_options).
     """
-    import torch
-    o = vec_default_options(rule)
-    if lr is not None:
-        o.lr = lr
-    if betas is not None:
-        o.beta1, o.beta2 = betas
-    if eps is not None:
-        o.eps = eps
-    if weight_decay is not None:
-        o.weight_decay = weight_decay
-    o.step = int(step)
-    n = len(x)
-    if v is None:
-        v = [None] * n
-    if not (len(g) == len(m) == len(v) == n):
-        raise ValueError("x, g, m and v must have one entry per parameter")
-    arr = (VecTensor * max(n, 1))()
-    for i in range(n):
-        for name, t in (("x", x[i]), ("g", g[i]), ("m", m[i])) + ((("v", v[i]),) if rule == "adamw" else ()):
-            if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 \
-                    or not t.is_contiguous() or t.numel() != x[i].numel():
-                raise ValueError(f"parameter {i}: {name} must be a contiguous fp32 CUDA tensor "
-                                 f"of {x[i].numel()} elements")
-        arr[i].x, arr[i].g, arr[i].m = x[i].data_ptr(), g[i].data_ptr(), m[i].data_ptr()
-        arr[i].v = v[i].data_ptr() if v[i] is not None else None
-        arr[i].numel = x[i].numel()
-    _check(dion_vec_step(arr, n, ctypes.byref(o), DionB200._stream(stream)), "dion_vec_step")
-    return dion_vec_last_launch_count()
+
+    def __init__(self, x, g, m, v=None, *, rule="adamw", lr=None, betas=None, eps=None,
+                 weight_decay=None):
+        import torch
+        o = vec_default_options(rule)
+        if lr is not None:
+            o.lr = lr
+        if betas is not None:
+            o.beta1, o.beta2 = betas
+        if eps is not None:
+            o.eps = eps
+        if weight_decay is not None:
+            o.weight_decay = weight_decay
+        n = len(x)
+        if v is None:
+            v = [None] * n
+        if not (len(g) == len(m) == len(v) == n):
+            raise ValueError("x, g, m and v must have one entry per parameter")
+        arr = (VecTensor * max(n, 1))()
+        for i in range(n):
+            named = (("x", x[i]), ("g", g[i]), ("m", m[i]))
+            if rule == "adamw":
+                named += (("v", v[i]),)
+            for name, t in named:
+                if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 \
+                        or not t.is_contiguous() or t.numel() != x[i].numel():
+                    raise ValueError(f"parameter {i}: {name} must be a contiguous fp32 CUDA "
+                                     f"tensor of {x[i].numel()} elements")
+            arr[i].x, arr[i].g, arr[i].m = x[i].data_ptr(), g[i].data_ptr(), m[i].data_ptr()
+            arr[i].v = v[i].data_ptr() if v[i] is not None else None
+            arr[i].numel = x[i].numel()
+        self.options, self.n, self._arr = o, n, arr
+        self._keep = (list(x), list(g), list(m), list(v))
+
+    def step(self, step: int = 1, stream=None) -> int:
+        """One step (AdamW step number ``step`` >= 1); returns the kernel launches."""
+        self.options.step = int(step)
+        _check(dion_vec_step(self._arr, self.n, ctypes.byref(self.options),
+                             DionB200._stream(stream)), "dion_vec_step")
+        return dion_vec_last_launch_count()
+
+
+def vec_step(x, g, m, v=None, *, rule="adamw", lr=None, betas=None, eps=None,
+             weight_decay=None, step=1, stream=None):
+    """One AdamW or Lion step of the vector (1-D) parameters, on the CUDA library
+    (a one-off VecStepPlan; keep a plan for repeated steps).  Returns the launches."""
+    return VecStepPlan(x, g, m, v, rule=rule, lr=lr, betas=betas, eps=eps,
+                       weight_decay=weight_decay).step(step, stream)

@@ -24,7 +24,7 @@
 
 namespace {
 
-constexpr int kPerLaunch = 64;
+constexpr int kPerLaunch = 128;  // 7.2 KB of kernel parameters (sm_70+ takes up to 32 KB)
 constexpr int kChunk = 8192;  // elements per work item (a multiple of 4 * kThreads)
 constexpr int kThreads = 256;
 constexpr int kCtasPerSm = 8;

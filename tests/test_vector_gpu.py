@@ -129,11 +129,11 @@ def test_lion_matches_oracle_step_by_step(wd):
 
 
 def test_many_tensors_take_several_launches():
-    sizes = [5 + (i % 7) * 300 for i in range(150)] + [0] * 10
+    sizes = [5 + (i % 7) * 300 for i in range(300)] + [0] * 10
     s = _state(sizes, 31)
     xs, gs, ms, vs = (_np(s[k]) for k in "xgmv")
     nl = dion.vec_step(s["x"], s["g"], s["m"], s["v"], rule="adamw", lr=1e-3, step=3)
-    assert nl == 3                                    # 150 non-empty tensors, 64 per launch
+    assert nl == 3                                    # 300 non-empty tensors, 128 per launch
     xr, mr, vr, bound = _adamw_ref(xs, gs, ms, vs, t=3, lr=1e-3, **HP)
     torch.cuda.synchronize()
     for i in range(len(sizes)):
@@ -179,3 +179,20 @@ def test_norm_gains_workload_both_rules():
                                   b2=0.99, wd=0.0)
         assert np.all(np.abs(_np([x[i]])[0] - xr) <= 2.0 ** -22 * np.abs(xr) + 1e-10)
         assert _rel(_np([m[i]])[0], mr) <= 1e-6
+
+
+def test_prepared_plan_over_steps_matches_oracle():
+    """A VecStepPlan marshals the pointer table once; three steps through it equal three
+    one-off calls' oracle trajectory (the step number is passed per call)."""
+    sizes = [4096] * 65 + [7]                        # 66 tensors: one launch of up to 128
+    s = _state(sizes, 51)
+    xs, gs, ms, vs = (_np(s[k]) for k in "xgmv")
+    plan = dion.VecStepPlan(s["x"], s["g"], s["m"], s["v"], rule="adamw", lr=1e-3)
+    bound = [np.zeros(n) for n in sizes]
+    for t in range(1, 4):
+        assert plan.step(t) == 1
+        xs, ms, vs, b = _adamw_ref(xs, gs, ms, vs, t=t, lr=1e-3, **HP)
+        bound = [a + c for a, c in zip(bound, b)]
+    torch.cuda.synchronize()
+    for i in range(len(sizes)):
+        assert np.all(np.abs(_np([s["x"][i]])[0] - xs[i]) <= bound[i]), i
