@@ -347,11 +347,13 @@ def run_ours(args):
 
 
 # ------------------------------------------------------------ vector (1-D) parameters
+L2_BYTES = 126 << 20                    # B200 L2
 VEC_BYTES = {"adamw": 28, "lion": 20}   # per element: AdamW reads x, g, m, v and writes
                                         # x, m, v; Lion reads x, g, m and writes x, m
 
 
-def measure_vector_step(dev, stream, peaks, warmup=3, iters=10):
+def measure_vector_step(dev, stream, peaks, warmup=3, iters=10,
+                        names=("vectors_64x4Mi", "norms_h4096_l32")):
     """AdamW and Lion over the vector parameters (dion_vec_step through a prepared
     VecStepPlan): a bank of 64 x 4 Mi elements (4 GiB of state, far larger than L2)
     against the copy bandwidth, and the 65 RMSNorm gains of the 7B-like decoder
@@ -362,9 +364,11 @@ def measure_vector_step(dev, stream, peaks, warmup=3, iters=10):
 
     from rank_orthonormalized_optimizer_b200 import VecStepPlan
     out = {}
-    for name, reps in (("vectors_64x4Mi", iters), ("norms_h4096_l32", 20 * iters)):
+    for name in names:
         vw = W.VECTOR_WORKLOADS[name]
         n = vw.params
+        big = 16 * n > L2_BYTES        # the four state arrays do not fit in L2
+        reps = iters if big else 20 * iters
         flat = {k: torch.empty(n, dtype=torch.float32, device=dev) for k in "xgmv"}
         views = {k: [] for k in "xgmv"}
         off = 0
@@ -394,7 +398,7 @@ def measure_vector_step(dev, stream, peaks, warmup=3, iters=10):
             r = {"us": ms * 1e3, "launches_per_step": launches // reps,
                  "bytes_per_element": VEC_BYTES[rule], "achieved_GBs": gbs,
                  "frac_of_measured_copy": gbs / peaks["hbm_gbs"]}
-            if n * 16 <= 1 << 30:
+            if not big:
                 # the same calls with the host ahead of the device: a bounded spin kernel
                 # (about 20 ms) holds the stream while every call is enqueued, so the
                 # events bracket the launches back to back (device time per call)
@@ -407,12 +411,33 @@ def measure_vector_step(dev, stream, peaks, warmup=3, iters=10):
                 torch.cuda.synchronize(dev)
                 r["queued_us"] = max_over_ranks(e0.elapsed_time(e1) / reps, dev) * 1e3
             rec[rule] = r
-        rec["l2"] = ("state (%.1f GB) far larger than L2" % (16 * n / 1e9) if n * 16 > 1 << 30
+        rec["l2"] = ("state (%.2f GB) larger than L2" % (16 * n / 1e9) if big
                      else "state resident in L2 (%.1f MB); launch-bound" % (16 * n / 1e6))
         out[name] = rec
         del flat, views
         torch.cuda.empty_cache()
     return out
+
+
+def run_vector_only(args):
+    """The vector-parameter step alone: one JSON line with its timings."""
+    import torch
+
+    rank, world = dist_setup("nccl")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = measured_peaks()
+    rec = measure_vector_step(dev, torch.cuda.current_stream(dev), peaks, warmup=args.warmup,
+                              iters=args.steps, names=(args.vector_only,))
+    if rank == 0:
+        print(json.dumps({"metric": "vector-parameter step (AdamW, Lion)", "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "data": "synthetic",
+                          "peak_GBs": peaks["hbm_gbs"], "peak_source": peaks["source"],
+                          "vector_step": rec}), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
 
 
 # ------------------------------------------------------------------ the oracle arm
@@ -456,11 +481,16 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-vector", action="store_true",
                     help="skip the AdamW / Lion step of the vector parameters")
+    ap.add_argument("--vector-only", default=None, choices=sorted(W.VECTOR_WORKLOADS),
+                    help="time only the vector-parameter step on this workload (for profiling "
+                         "its kernel with little else on the device)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
+    elif args.vector_only:
+        run_vector_only(args)
     else:
         run_ours(args)
 

@@ -230,6 +230,8 @@ VECTOR_WORKLOADS = {
     "norms_h4096_l32": VectorWorkload("norms_h4096_l32", (4096,) * 65),
     # a bank larger than L2 (64 x 4 Mi elements, 1 GiB per state array)
     "vectors_64x4Mi": VectorWorkload("vectors_64x4Mi", (4 << 20,) * 64),
+    # the same with 16 tensors (256 MiB per state array, still twice L2): for profiling
+    "vectors_16x4Mi": VectorWorkload("vectors_16x4Mi", (4 << 20,) * 16),
 }
 
 
