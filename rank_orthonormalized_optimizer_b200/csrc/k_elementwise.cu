@@ -6,15 +6,16 @@
 
 namespace dion {
 
-static int g_sms = 0;
+// SM count of the first device asked (the library runs on B200s only); initialised once,
+// thread-safely, by the static local's initialiser
 static int sm_count() {
-  if (g_sms == 0) {
-    int dev = 0;
+  static const int sms = [] {
+    int dev = 0, n = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_sms <= 0) g_sms = 148;
-  }
-  return g_sms;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+  }();
+  return sms;
 }
 
 // ---------------------------------------------------------------- B = M + G

@@ -121,25 +121,25 @@ const char* tc_map_error() { return tc::tl_map_error; }
 
 namespace tc {
 
+// Device limits of the first device asked (the library runs on B200s only), each
+// initialised once, thread-safely, by its static local's initialiser.
 static int smem_optin() {
-  static int bytes = 0;
-  if (!bytes) {
-    int dev = 0;
+  static const int bytes = [] {
+    int dev = 0, b = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&bytes, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (bytes <= 0) bytes = 227 * 1024;
-  }
+    cudaDeviceGetAttribute(&b, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    return b > 0 ? b : 227 * 1024;
+  }();
   return bytes;
 }
 
 static int sm_count() {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
+  static const int sms = [] {
+    int dev = 0, n = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+  }();
   return sms;
 }
 
