@@ -55,7 +55,8 @@ typedef enum dion_status {
   DION_ERR_CUDA = 4,                /* a CUDA runtime call failed (message says which) */
   DION_ERR_NOT_INITIALIZED = 5,     /* null or freed handle                       */
   DION_ERR_DEVICE = 6,              /* current device is not sm_100 (B200)       */
-  DION_ERR_MISALIGNED = 7,          /* a device pointer is not 16-byte aligned    */
+  DION_ERR_MISALIGNED = 7,          /* a device pointer is not aligned as required
+                                       (16 bytes for the Dion step, 4 for dion_vec_step) */
   DION_ERR_HOST = 8                 /* host-side failure (out of host memory); no C++
                                        exception ever leaves the library             */
 } dion_status;
