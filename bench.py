@@ -275,6 +275,8 @@ def run_ours(args):
     if traffic_per_elem is not None and traffic_hash == update_kernel_hash():
         traffic = traffic_per_elem * sum(b.params for b in wl.buckets) / max(upd_launches, 1)
     roof_t = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_alg / (peaks["hbm_gbs"] * 1e9))
+    comp_bytes = sum(b.count * (20 * b.m * b.n + 8 * b.n * b.r) for b in wl.buckets)
+    comp_t = comp_bytes / (peaks["hbm_gbs"] * 1e9)
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -294,7 +296,12 @@ def run_ours(args):
                      "peak_source": peaks["source"],
                      "per_step_ms": upd_ms, "algorithmic_bytes_per_step": upd_bytes},
         "step_roofline": {"t_roofline_ms": roof_t * 1e3, "frac": roof_t * 1e3 / ms,
-                          "flops": flops, "bytes": bytes_alg},
+                          "flops": flops, "bytes": bytes_alg,
+                          # the state alone (read M, G, X, Q; write M, X, Q), as if the three
+                          # sweeps over B needed no more than one
+                          "compulsory_bytes": comp_bytes,
+                          "t_compulsory_ms": comp_t * 1e3,
+                          "frac_compulsory": comp_t * 1e3 / ms},
         "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items()},
         "gpu_launches": launches,
         "status_bits": int(np.bitwise_or.reduce(st.numpy())) if st.numel() else 0,
