@@ -85,3 +85,16 @@ def test_empty_tensors_need_no_pointers():
     if no_gpu:
         assert _call(arr, 2, _opts()) in (dion.ERR_CUDA, dion.ERR_DEVICE)
         assert dion.dion_vec_last_launch_count() == 0
+
+
+def test_plan_checks_its_tensors_on_the_host():
+    """VecStepPlan refuses what the C ABI could not take, before any call: CPU tensors,
+    other dtypes, non-contiguous views, mismatched sizes and list lengths."""
+    import torch
+    x = torch.zeros(8)
+    with pytest.raises(ValueError, match="CUDA"):
+        dion.VecStepPlan([x], [x.clone()], [x.clone()], [x.clone()])
+    with pytest.raises(ValueError, match="one entry per parameter"):
+        dion.VecStepPlan([x, x], [x], [x], [x])
+    with pytest.raises(KeyError):
+        dion.VecStepPlan([x], [x], [x], [x], rule="sgd")
