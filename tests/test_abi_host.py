@@ -180,3 +180,21 @@ def test_status_strings_and_views():
                                     ctypes.byref(nb)) == dion.ERR_INVALID_ARG
     assert dion.dion_last_launch_count(h) == 0
     dion.dion_free(h)
+
+
+def test_plain_c_caller(tmp_path):
+    """include/dion.h compiles as C99 and a C program links the library and gets the
+    documented codes back (no device touched)."""
+    import shutil
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "abi_check"
+    libdir = os.path.dirname(dion.LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_check.c"),
+                    "-L", libdir, "-ldion_b200", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                   check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout + out.stderr
