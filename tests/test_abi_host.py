@@ -198,3 +198,22 @@ def test_plain_c_caller(tmp_path):
                    check=True, capture_output=True, text=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout + out.stderr
+
+
+def test_product_and_oracle_share_nothing():
+    """The package (binding, build script, CUDA sources) never names the oracle, and the
+    oracle never names the package or its library: the two meet only through the seeded
+    inputs of `workloads`, which holds none of the method's arithmetic."""
+    import glob
+    pkg = os.path.join(ROOT, "rank_orthonormalized_optimizer_b200")
+    product = [f for pat in ("*.py", "csrc/*") for f in glob.glob(os.path.join(pkg, pat))]
+    product.append(os.path.join(ROOT, "include", "dion.h"))
+    for f in product:
+        text = open(f, errors="replace").read()
+        assert not re.search(r"\boracle\b", text, flags=re.I), f
+    for f in glob.glob(os.path.join(ROOT, "oracle", "*.py")):
+        text = open(f).read()
+        assert "rank_orthonormalized_optimizer_b200" not in text and "libdion" not in text, f
+        assert not re.search(r"^\s*(import|from)\s+(torch|rank_orth|ctypes)", text, flags=re.M), f
+    wl = open(os.path.join(ROOT, "workloads", "__init__.py")).read()
+    assert not re.search(r"^\s*(import|from)\s+(oracle|rank_orth)", wl, flags=re.M)
