@@ -145,6 +145,21 @@ def algorithmic(wl: W.Workload):
     return flops, bytes_, update_bytes
 
 
+def split_ceiling(wl: W.Workload, peaks):
+    """The ceiling of fp32 mode on the tensor path, whose contractions run as bf16
+    products of three-way splits: six for B Q, B^T P, the Gram and the apply, three for
+    the update (its two leading parts); B kept as its split, written once and read by
+    both sweeps (40 B per weight element with B = M + G fused into B Q).  The time of
+    those bf16 products at the measured bf16 peak, or of those bytes at the measured copy
+    bandwidth, whichever is longer."""
+    flops = sum(b.count * (36 * b.m * b.n * b.r + 18 * b.m * b.r ** 2 + b.r ** 3 / 3)
+                for b in wl.buckets)
+    bytes_ = sum(b.count * (40 * b.m * b.n + 4 * (3 * b.m * b.r + 6 * b.n * b.r))
+                 for b in wl.buckets)
+    t = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
+    return flops, bytes_, t
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -307,6 +322,11 @@ def run_ours(args):
         "status_bits": int(np.bitwise_or.reduce(st.numpy())) if st.numel() else 0,
         "clocks": clocks,
     }
+
+    if wl.precision == "fp32" and args.kernel_path == "tensor":
+        sf, sb, st_ = split_ceiling(wl, peaks)
+        result["split_roofline"] = {"t_ms": st_ * 1e3, "frac": st_ * 1e3 / ms,
+                                    "bf16_product_flops": sf, "bytes": sb}
 
     # end to end through the C ABI with the gradients in pinned host memory
     if not args.no_e2e:

@@ -74,3 +74,16 @@ def test_reference_arm_other_ranks_exit_quietly():
                           "--workload", "single_256x128_r32", "--steps", "1", "--warmup", "0"],
                          capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_split_ceiling_of_the_rank_sweep():
+    """fp32 mode's ceiling counts the bf16 products its splits issue (36 m n r + 18 m r^2)
+    and 40 B per weight element; at r = 1024 on 8 x 8192^2 the products dominate."""
+    wl = W.WORKLOADS["square_8x8192_r1024"]
+    peaks = {"bf16_tflops": 1672.0, "hbm_gbs": 6458.1}
+    f, b, t = bench.split_ceiling(wl, peaks)
+    m = n = 8192
+    r = 1024
+    assert f == 8 * (36 * m * n * r + 18 * m * r * r + r ** 3 / 3)
+    assert b == 8 * (40 * m * n + 4 * (3 * m * r + 6 * n * r))
+    assert t == f / 1672e12 and f / 1672e12 > b / 6458.1e9
