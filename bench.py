@@ -78,17 +78,65 @@ def whole_job_rate(units_per_rank: float, world: int, seconds_max: float) -> flo
 
 
 # ------------------------------------------------------------------ clocks sampler
+_REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+                ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+
+
 class Clocks:
+    """SM clock, power and clock-event reasons sampled DURING the timed region.
+
+    NVML is read from a background thread every 10 ms (read-only queries: nothing about
+    the GPU's settings is changed), so even a sub-second timed region gives dozens of
+    samples; without NVML, ``nvidia-smi -lms 200`` is polled instead."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.01
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, pci_bus_id: str | None = None):
         self.gpu = gpu_index
+        self.pci = pci_bus_id
+        self.rows = []          # (sm_mhz, sm_max_mhz, power_w, reasons_bitmask)
         self.proc = None
         self.path = None
+        self.thread = None
+        self.stop = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.pci:
+            try:
+                return pynvml.nvmlDeviceGetHandleByPciBusId(self.pci)
+            except Exception:
+                pass
+        return pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _sample_nvml(self, h):
+        import pynvml
+        smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            try:
+                self.rows.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), smax,
+                                  pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                  pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except Exception:
+                break
+            self.stop.wait(self.PERIOD_S)
 
     def __enter__(self):
+        import threading
+        try:
+            h = self._nvml_handle()
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._sample_nvml, args=(h,), daemon=True)
+            self.thread.start()
+            self.source = "nvml, 10 ms"
+            time.sleep(0.05)
+            return self
+        except Exception:
+            self.thread = None
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
@@ -96,12 +144,16 @@ class Clocks:
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi, 200 ms"
         except Exception:
             self.proc = None
         time.sleep(0.3)
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -109,27 +161,39 @@ class Clocks:
             except Exception:
                 self.proc.kill()
 
-    def summary(self):
+    def _smi_rows(self):
         rows = []
         try:
             for line in open(self.path):
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
-                    rows.append(parts)
+                    bits = sum(b for i, (_, b) in enumerate(_REASON_BITS)
+                               if parts[5 + i].lower() == "active")
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), bits))
         except Exception:
             pass
         finally:
             if self.path and os.path.exists(self.path):
                 os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clocks not sampled"]}
-        sm = [float(r[1]) for r in rows]
-        smax = max(float(r[2]) for r in rows)
-        loaded = [s for s, r in zip(sm, rows) if float(r[3]) > 200.0] or sm
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows)}
+        return rows
+
+    def summary(self):
+        rows = self.rows if self.thread is not None else self._smi_rows()
+        return summarize_clocks(rows, self.source)
+
+
+def summarize_clocks(rows, source=None):
+    """Median SM clock under load, the max clock and the throttle reasons seen, from
+    (sm_mhz, sm_max_mhz, power_w, reasons_bitmask) samples."""
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clocks not sampled"]}
+    sm = [float(r[0]) for r in rows]
+    smax = max(float(r[1]) for r in rows)
+    loaded = [s for s, r in zip(sm, rows) if float(r[2]) > 200.0] or sm
+    reasons = sorted({name for r in rows for name, bit in _REASON_BITS if int(r[3]) & bit})
+    return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+            "samples": len(rows), "power_w_max": max(float(r[2]) for r in rows),
+            "source": source}
 
 
 # ------------------------------------------------------------------ roofline figures
@@ -195,7 +259,9 @@ def update_kernel_hash():
 
 # ------------------------------------------------------------------ oracle timing
 def oracle_sample(wl: W.Workload, steps: int, budget_s: float = 20.0):
-    """Time the fp64 oracle on one matrix per bucket; returns (params/s, seconds, cores, note)."""
+    """Time the fp64 oracle on one matrix per bucket; returns (params/s, seconds, cores,
+    note).  The seconds are the whole workload's step extrapolated from the sample by
+    the bucket counts."""
     import oracle
     blas = "unknown"
     try:
@@ -231,6 +297,15 @@ def oracle_sample(wl: W.Workload, steps: int, budget_s: float = 20.0):
 
 
 # ------------------------------------------------------------------ the GPU arm
+def _pci_bus_id(dev):
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+    except Exception:
+        return None
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -260,7 +335,7 @@ def run_ours(args):
     # timed region: K steps, barrier + sync on both sides, device events
     opt.profile_enable(True)
     launches = 0
-    with Clocks(local) as clk:
+    with Clocks(local, _pci_bus_id(dev)) as clk:
         barrier(dev)
         torch.cuda.synchronize(dev)
         t0 = torch.cuda.Event(enable_timing=True)
@@ -484,11 +559,18 @@ def run_reference(args):
     wall = time.perf_counter() - t0
     step_s = statistics.median(vals)
     value = wl.params / step_s
+    sampled = len(wl.buckets)
+    total = sum(b.count for b in wl.buckets)
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": wl.name, "params": wl.params},
+        # each timed step runs one matrix per shape bucket; ms_per_step is that sample
+        # scaled by the bucket counts to the whole workload, not a measured step
+        "extrapolated": total != sampled,
+        "matrices_run_per_step": sampled, "matrices_per_workload_step": total,
+        "sample_ms_per_step": wall / max(args.steps, 1) * 1e3,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": note},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -498,12 +580,12 @@ def run_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE, choices=sorted(W.WORKLOADS))
     ap.add_argument("--kernel-path", default="tensor", choices=["tensor", "simt"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-vector", action="store_true",

@@ -201,22 +201,29 @@ dion_status dion_step_batched_from_host(dion_handle h, const dion_bucket_ptrs* p
 
 /*
  * dion_step_batched without a caller workspace, for callers that cannot allocate
- * device memory: code running while a stream is being captured into a CUDA graph
- * (where cudaMalloc is not allowed), plug-ins that are handed only the model's
- * buffers by a host program whose allocator they cannot reach, or loops that must
- * not allocate after start-up.  The pages describe nothing like it; it is a
- * convenience of this library.  Arguments are those of dion_step_batched; X, M, G,
- * Q and d_status remain caller buffers.
+ * device memory: a plug-in or extension that is handed only the model's buffers by a
+ * host program whose allocator it cannot reach, or a training loop whose device
+ * memory is sized once at start-up (a fixed pool, a budget the host program enforces)
+ * and that must not allocate afterwards.  The pages describe nothing like it; it is a
+ * convenience of this library.  Arguments are those of dion_step_batched; X, M, G, Q
+ * and d_status remain caller buffers.
  *  - Scratch comes from one array of DION_STATIC_SCRATCH_BYTES inside the library.
  *    A plan whose workspace (from dion_init) is larger is rejected with
  *    DION_ERR_WORKSPACE_TOO_SMALL and nothing runs.
- *  - The first call on a device looks the array's device address up once (with
- *    that device current); make that first call outside any stream capture.
+ *  - The first call on a device looks the array's device address up (with that
+ *    device current); make that first call outside any stream capture.  The address
+ *    is looked up again when the device's context has changed since the last call
+ *    (after cudaDeviceReset, for instance), since a new context holds a new copy.
  *  - Every call on a device shares the array.  It keeps whatever the last call
  *    left in it; the step writes every scratch word it reads, so nothing needs
  *    clearing.  Calls whose work overlaps on the GPU (two streams, two threads, two
  *    handles) race on it: serialise them.
- *  - The library allocates and frees no device memory in this call.
+ *  - This call makes no cudaMalloc or cudaFree and calls no allocating library
+ *    routine.  As with dion_step_batched, the first call on a handle and device
+ *    creates the handle's streams and events, and a plan with r > 256 on the tensor
+ *    path builds the fallback's CUDA graph, which is rebuilt whenever the same handle
+ *    switches between this entry point and dion_step_batched (their scratch differs);
+ *    the driver may set aside memory for those objects.
  */
 dion_status dion_step_batched_noalloc(dion_handle h, const dion_bucket_ptrs* ptrs,
                                       int32_t nbuckets, float lr, int32_t* d_status,

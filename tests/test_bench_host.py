@@ -66,6 +66,32 @@ def test_reference_arm_prints_one_json_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "params/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+    # one matrix is the whole workload here: nothing extrapolated
+    assert d["extrapolated"] is False and d["matrices_run_per_step"] == 1
+
+
+def test_reference_arm_marks_extrapolation():
+    """On a multi-matrix workload the oracle arm runs one matrix per bucket, scales it by
+    the bucket counts, and says so in fields of its own."""
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "fullrank_16x1024x1024", "--steps", "1", "--warmup", "0"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    d = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][0])
+    assert d["extrapolated"] is True
+    assert d["matrices_run_per_step"] == 1 and d["matrices_per_workload_step"] == 16
+    assert d["sample_ms_per_step"] < d["ms_per_step"]
+
+
+def test_clock_summary_flags_throttle_reasons():
+    """Samples (MHz, max MHz, W, reason bits): the median is taken over loaded samples
+    (power above 200 W) and every throttle reason seen is named."""
+    rows = [(1965, 1965, 150.0, 0), (1800, 1965, 900.0, 0x4), (1700, 1965, 950.0, 0x4),
+            (1900, 1965, 800.0, 0x40)]
+    s = bench.summarize_clocks(rows, "test")
+    assert s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965 and s["samples"] == 4
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert bench.summarize_clocks([])["reasons"] == ["clocks not sampled"]
 
 
 def test_reference_arm_other_ranks_exit_quietly():
