@@ -448,6 +448,86 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------ row-sharded step
+def run_rowshard(args):
+    """The workload's matrices split by rows over the ranks (dion_init_sharded): every
+    rank holds rows of every matrix, and each step all-reduces the Grams and R over NCCL
+    (strong scaling: the total work is fixed).  At one rank nothing is exchanged; the
+    line then measures what the sharded protocol itself costs (its host round trip)."""
+    import numpy as np
+    import torch
+
+    rank, world = dist_setup("nccl")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from rank_orthonormalized_optimizer_b200 import DionB200RowSharded
+
+    wl = W.WORKLOADS[args.workload]
+    opt = DionB200RowSharded([(b.count, b.m, b.n, b.r) for b in wl.buckets], rank, world,
+                             mu=wl.mu, precision=wl.precision)
+    nb = len(wl.buckets)
+
+    def rows(t, i):
+        r0, mk = opt.row_ranges[i]
+        return t[:, r0:r0 + mk].contiguous()
+
+    X, G = [], []
+    for i in range(nb):
+        X.append(rows(W.weights(wl, i, dev), i))
+        G.append(rows(W.gradient(wl, i, 0, dev), i))
+        torch.cuda.empty_cache()
+    M = [torch.zeros_like(x) for x in X]
+    Q = [W.right_factor(wl, i, dev) for i in range(nb)]
+    ws = opt.alloc_workspace(dev)
+    status = opt.alloc_status(dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        xchg = opt.step(X, M, G, Q, wl.lr, ws, status, stream)
+    torch.cuda.synchronize(dev)
+    launches = 0
+    with Clocks(local, _pci_bus_id(dev)) as clk:
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            xchg = opt.step(X, M, G, Q, wl.lr, ws, status, stream)
+            launches += opt.last_launch_count
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
+    st = status.cpu()
+    flops, bytes_alg, _ = algorithmic(wl)
+    peaks = measured_peaks()
+    roof_t = max(flops / (peaks["bf16_tflops"] * 1e12),
+                 bytes_alg / (peaks["hbm_gbs"] * 1e9)) / world
+    result = {
+        "metric": METRIC, "value": wl.params / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "bf16" if wl.precision == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "params": wl.params,
+                   "buckets": [[b.count, b.m, b.n, b.r] for b in wl.buckets],
+                   "parallelism": f"row-sharded x{world} (every matrix split by rows)",
+                   "l2": "inputs far larger than L2; no flush"},
+        "exchanges_per_step": [k for k, _ in xchg],
+        "allreduce_floats_per_step": sum(c for _, c in xchg) if world > 1 else 0,
+        "step_roofline": {"t_roofline_ms": roof_t * 1e3, "frac": roof_t * 1e3 / ms},
+        "gpu_launches": launches,
+        "status_bits": int(np.bitwise_or.reduce(st.numpy())) if st.numel() else 0,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    opt.close()
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
 # ------------------------------------------------------------ vector (1-D) parameters
 L2_BYTES = 126 << 20                    # B200 L2
 VEC_BYTES = {"adamw": 28, "lion": 20}   # per element: AdamW reads x, g, m, v and writes
@@ -590,6 +670,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-vector", action="store_true",
                     help="skip the AdamW / Lion step of the vector parameters")
+    ap.add_argument("--rowshard", action="store_true",
+                    help="split every matrix by rows over the ranks (all-reduce of the Grams "
+                         "and R over NCCL) instead of giving each rank its own matrices")
     ap.add_argument("--vector-only", default=None, choices=sorted(W.VECTOR_WORKLOADS),
                     help="time only the vector-parameter step on this workload (for profiling "
                          "its kernel with little else on the device)")
@@ -600,6 +683,8 @@ def main(argv=None):
         run_reference(args)
     elif args.vector_only:
         run_vector_only(args)
+    elif args.rowshard:
+        run_rowshard(args)
     else:
         run_ours(args)
 

@@ -71,7 +71,10 @@ enum {
   DION_MAT_NONFINITE = 4,     /* a Gram matrix held Inf/NaN (inputs were not finite)     */
   DION_MAT_TIMEOUT = 8,       /* a bounded device wait ran out; this matrix's outputs
                                  are not valid and X, M, Q may be partly updated         */
-  DION_MAT_ZERO_COLUMN = 16   /* some column of R had zero norm; its Q column is zero    */
+  DION_MAT_ZERO_COLUMN = 16,  /* some column of R had zero norm; its Q column is zero    */
+  DION_MAT_HIGH_RMMC = 32     /* the momentum changed faster than rmmc_threshold: RMMC =
+                                 max|M' - M| / max|M| > rmmc_threshold (CurvaDion's gate:
+                                 this matrix needs synchronising; see DION_VIEW_RMMC)     */
 };
 
 /* Arithmetic of the four rank-r contractions (B Q, B^T P, P R^T, P Q^T). */
@@ -123,6 +126,8 @@ typedef struct dion_options {
   int32_t kernel_path;     /* dion_kernel_path (default DION_PATH_TENSOR)                  */
   int64_t max_wait_spins;  /* bound on every device-side wait; when it runs out the
                               kernel sets DION_MAT_TIMEOUT and returns (default 1<<26)     */
+  float rmmc_threshold;    /* DION_MAT_HIGH_RMMC where RMMC exceeds it (default 0: every
+                              matrix whose momentum moved; not NaN)                        */
 } dion_options;
 
 /* Device buffers of one bucket, all contiguous, row-major, 16-byte aligned:
@@ -229,6 +234,79 @@ dion_status dion_step_batched_noalloc(dion_handle h, const dion_bucket_ptrs* ptr
                                       int32_t nbuckets, float lr, int32_t* d_status,
                                       void* stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * Row-sharded step.  The article says Dion cuts the data synchronised between
+ * nodes (paragraph 3) and works under data, tensor and fully sharded data
+ * parallelism, FSDP2 included (paragraph 5), without saying how.  Here the rows of
+ * every matrix are split among the ranks: a rank holds rows [row0, row0 + m) of X,
+ * M and G of each matrix and the whole Q (n x r), the same on every rank.  The step
+ * is the whole-matrix step; only sums over ranks of r-sized quantities cross
+ * between ranks, each an all-reduce (sum) of fp32 values that the CALLER performs
+ * (NCCL, or anything else) on a buffer inside the workspace:
+ *
+ *   DION_XCHG_GRAM    the Grams W = P0^T P0 of every bucket (count r^2 floats each)
+ *   DION_XCHG_GRAM2   the second Cholesky-QR pass's Grams, followed by one float per
+ *                     bucket: the number of its matrices Cholesky-QR rejected
+ *   DION_XCHG_GATHER  only for a bucket with rejected matrices: its P0 as
+ *                     [count, m_full, r] with this rank's rows filled and zeros
+ *                     elsewhere (summing gathers it); Householder QR of the whole P0
+ *                     then runs on every rank, which keeps its rows
+ *   DION_XCHG_R       R = B^T P of every bucket (count n r floats each)
+ *
+ * The Cholesky factors, the decisions taken from them and Q = colnorm(R) are
+ * computed from the summed values by the same deterministic kernels on every rank,
+ * so every rank reaches the same P, Q and status.  Usage (every rank):
+ *
+ *   dion_exchange x;
+ *   dion_step_sharded_begin(h, ptrs, nb, lr, ws, ws_bytes, d_status, stream, &x);
+ *   while (x.count > 0) {
+ *     allreduce_sum_fp32(x.d_buf, x.count, stream);   // e.g. ncclAllReduce
+ *     dion_step_sharded_continue(h, &x);
+ *   }
+ *
+ * Every call enqueues work on `stream` and returns; the continue that follows the
+ * DION_XCHG_GRAM2 exchange synchronises `stream` once (it reads the per-bucket
+ * counts to decide which buckets need the gather).  An error abandons the step
+ * (X, M and Q are written only by its last call); all ranks must then abandon it.
+ * Runs on the tensor path only; the rank-sharded fallback is Householder QR of the
+ * gathered P0, never the shifted Cholesky-QR iteration.
+ */
+typedef struct dion_shard_desc {
+  int64_t m_full;  /* rows of every whole matrix of the bucket                          */
+  int64_t row0;    /* first row this rank holds; it holds dion_bucket_desc.m rows      */
+} dion_shard_desc;
+
+enum { DION_XCHG_NONE = 0, DION_XCHG_GRAM = 1, DION_XCHG_GRAM2 = 2, DION_XCHG_GATHER = 3,
+       DION_XCHG_R = 4 };
+
+typedef struct dion_exchange {
+  float* d_buf;    /* device buffer to sum over ranks in place (inside the workspace)  */
+  int64_t count;   /* fp32 elements; 0 when the step is complete                       */
+  int32_t what;    /* DION_XCHG_*                                                      */
+} dion_exchange;
+
+/*
+ * Plan a row-sharded step: buckets[b] gives this rank's rows (m), the columns, the
+ * rank and the count; shards[b] the rows of the whole matrices and this rank's first
+ * row (row0 + m <= m_full).  r <= min(m_full, n); s defaults to sqrt(m_full / n).
+ * Otherwise as dion_init; the plan may only be stepped by dion_step_sharded_begin.
+ */
+dion_status dion_init_sharded(const dion_bucket_desc* buckets, const dion_shard_desc* shards,
+                              int32_t nbuckets, const dion_options* opt, dion_handle* out,
+                              size_t* workspace_bytes);
+
+/* Start a row-sharded step (arguments as dion_step_batched); *next receives the first
+ * exchange.  DION_ERR_INVALID_ARG when a step is already in progress on the handle. */
+dion_status dion_step_sharded_begin(dion_handle h, const dion_bucket_ptrs* ptrs,
+                                    int32_t nbuckets, float lr, void* d_workspace,
+                                    size_t workspace_bytes, int32_t* d_status, void* stream,
+                                    dion_exchange* next);
+
+/* Continue the step after *next's buffer has been summed over all ranks; *next
+ * receives the following exchange, or count 0 when the step is complete. */
+dion_status dion_step_sharded_continue(dion_handle h, dion_exchange* next);
+
 /* Release the handle (host memory only).  NULL is accepted. */
 dion_status dion_free(dion_handle h);
 
@@ -246,8 +324,18 @@ int32_t dion_last_launch_count(dion_handle h);
 
 /* Intermediates of the most recent step, for inspection after the stream has
  * been synchronised: which = DION_VIEW_P gives P (fp32 [count, m, r]),
- * DION_VIEW_R gives R (fp32 [count, n, r]).  *d_ptr points into d_workspace. */
-enum { DION_VIEW_P = 0, DION_VIEW_R = 1 };
+ * DION_VIEW_R gives R (fp32 [count, n, r]), DION_VIEW_RMMC gives each matrix's
+ * relative maximum momentum change (fp32 [count]).  *d_ptr points into d_workspace.
+ *
+ * RMMC is the statistic by which "CurvaDion: Curvature-Adaptive Distributed
+ * Orthonormalization" (mlsanity.com, Abstract) decides which layers need
+ * synchronising: built from the momentum the optimizer already keeps, O(d) per
+ * layer.  The page does not write it down; here, per matrix, with M before the step
+ * and M' after it, RMMC = max_ij |M'_ij - M_ij| / max_ij |M_ij| (+inf for a zero M
+ * that changed, 0 for one that did not).  The fused update computes both maxima from
+ * the values it streams anyway.  In a row-sharded step each rank's value covers its
+ * own rows (the maximum over ranks of each maximum gives the whole matrix's). */
+enum { DION_VIEW_P = 0, DION_VIEW_R = 1, DION_VIEW_RMMC = 2 };
 dion_status dion_workspace_view(dion_handle h, int32_t bucket, int32_t which,
                                 void* d_workspace, void** d_ptr, size_t* bytes);
 

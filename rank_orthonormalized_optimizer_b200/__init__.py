@@ -33,11 +33,12 @@ c_int32, c_int64, c_float, c_void_p, c_size_t = (ctypes.c_int32, ctypes.c_int64,
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_WORKSPACE_TOO_SMALL, ERR_CUDA, \
     ERR_NOT_INITIALIZED, ERR_DEVICE, ERR_MISALIGNED, ERR_HOST = range(9)
 MAT_OK, MAT_FALLBACK, MAT_CHOLQR2, MAT_NONFINITE, MAT_TIMEOUT, MAT_ZERO_COLUMN = 0, 1, 2, 4, 8, 16
+MAT_HIGH_RMMC = 32
 PRECISIONS = {"fp32": 0, "bf16": 1}
 ORTH_MODES = {"auto": 0, "cholqr": 1, "cholqr2": 2, "householder": 3}
 KERNEL_PATHS = {"tensor": 0, "simt": 1}
 KERNEL_CLASSES = ["form_b", "prep_q", "gemm_bq", "orth", "gemm_btp", "colnorm", "update"]
-VIEW_P, VIEW_R = 0, 1
+VIEW_P, VIEW_R, VIEW_RMMC = 0, 1, 2
 STATIC_SCRATCH_BYTES = 16 << 20   # DION_STATIC_SCRATCH_BYTES of include/dion.h
 
 
@@ -49,11 +50,24 @@ class BucketDesc(ctypes.Structure):
 class Options(ctypes.Structure):
     _fields_ = [("mu", c_float), ("precision", c_int32), ("orth_mode", c_int32),
                 ("fallback_cond", c_float), ("orth_tol", c_float), ("kernel_path", c_int32),
-                ("max_wait_spins", c_int64)]
+                ("max_wait_spins", c_int64), ("rmmc_threshold", c_float)]
 
 
 class BucketPtrs(ctypes.Structure):
     _fields_ = [("X", c_void_p), ("M", c_void_p), ("G", c_void_p), ("Q", c_void_p)]
+
+
+class ShardDesc(ctypes.Structure):
+    _fields_ = [("m_full", c_int64), ("row0", c_int64)]
+
+
+class Exchange(ctypes.Structure):
+    _fields_ = [("d_buf", c_void_p), ("count", c_int64), ("what", c_int32)]
+
+
+XCHG_NONE, XCHG_GRAM, XCHG_GRAM2, XCHG_GATHER, XCHG_R = range(5)
+XCHG_NAMES = {XCHG_NONE: "none", XCHG_GRAM: "gram", XCHG_GRAM2: "gram2",
+              XCHG_GATHER: "gather", XCHG_R: "r"}
 
 
 VEC_RULES = {"adamw": 0, "lion": 1}
@@ -87,6 +101,14 @@ dion_step_batched_from_host = _sig("dion_step_batched_from_host", c_int32, c_voi
 dion_step_batched_noalloc = _sig("dion_step_batched_noalloc", c_int32, c_void_p,
                                  ctypes.POINTER(BucketPtrs), c_int32, c_float, c_void_p, c_void_p)
 dion_free = _sig("dion_free", c_int32, c_void_p)
+dion_init_sharded = _sig("dion_init_sharded", c_int32, ctypes.POINTER(BucketDesc),
+                         ctypes.POINTER(ShardDesc), c_int32, ctypes.POINTER(Options),
+                         ctypes.POINTER(c_void_p), ctypes.POINTER(c_size_t))
+dion_step_sharded_begin = _sig("dion_step_sharded_begin", c_int32, c_void_p,
+                               ctypes.POINTER(BucketPtrs), c_int32, c_float, c_void_p, c_size_t,
+                               c_void_p, c_void_p, ctypes.POINTER(Exchange))
+dion_step_sharded_continue = _sig("dion_step_sharded_continue", c_int32, c_void_p,
+                                  ctypes.POINTER(Exchange))
 dion_vec_default_options = _sig("dion_vec_default_options", c_int32, c_int32,
                                 ctypes.POINTER(VecOptions))
 dion_vec_step = _sig("dion_vec_step", c_int32, ctypes.POINTER(VecTensor), c_int32,
@@ -104,7 +126,9 @@ dion_profile_read = _sig("dion_profile_read", c_int32, c_void_p, ctypes.POINTER(
 
 #: every entry point include/dion.h declares
 EXPORTED = ["dion_default_options", "dion_init", "dion_step_batched",
-            "dion_step_batched_from_host", "dion_step_batched_noalloc", "dion_free", "dion_status_string", "dion_last_error",
+            "dion_step_batched_from_host", "dion_step_batched_noalloc", "dion_free",
+            "dion_init_sharded", "dion_step_sharded_begin", "dion_step_sharded_continue",
+            "dion_status_string", "dion_last_error",
             "dion_num_matrices", "dion_last_launch_count", "dion_workspace_view",
             "dion_profile_enable", "dion_profile_read", "dion_vec_default_options",
             "dion_vec_step", "dion_vec_last_launch_count"]
@@ -137,6 +161,28 @@ class Shape:
     r: int
 
 
+def _make_options(mu, precision, orth_mode, kernel_path, fallback_cond, orth_tol,
+                  max_wait_spins, rmmc_threshold=0.0) -> Options:
+    o = default_options()
+    o.rmmc_threshold = rmmc_threshold
+    o.mu = mu
+    o.precision = PRECISIONS[precision]
+    o.orth_mode = ORTH_MODES[orth_mode]
+    o.kernel_path = KERNEL_PATHS[kernel_path]
+    o.fallback_cond = fallback_cond
+    o.orth_tol = orth_tol
+    o.max_wait_spins = max_wait_spins
+    return o
+
+
+def _descs(shapes, scales=None):
+    descs = (BucketDesc * max(len(shapes), 1))()
+    for i, s in enumerate(shapes):
+        descs[i].m, descs[i].n, descs[i].r, descs[i].count = s.m, s.n, s.r, s.count
+        descs[i].scale = float(scales[i]) if scales is not None else 0.0
+    return descs
+
+
 class DionB200:
     """Handle of one planned step over a fixed list of shape buckets.
 
@@ -147,25 +193,14 @@ class DionB200:
 
     def __init__(self, buckets, *, mu=0.95, precision="bf16", orth_mode="auto",
                  kernel_path="tensor", fallback_cond=1e3, orth_tol=2e-5,
-                 max_wait_spins=1 << 26, scales=None):
+                 max_wait_spins=1 << 26, scales=None, rmmc_threshold=0.0):
         self.shapes = [Shape(*map(int, b)) for b in buckets]
-        n = len(self.shapes)
-        descs = (BucketDesc * max(n, 1))()
-        for i, s in enumerate(self.shapes):
-            descs[i].m, descs[i].n, descs[i].r, descs[i].count = s.m, s.n, s.r, s.count
-            descs[i].scale = float(scales[i]) if scales is not None else 0.0
-        o = default_options()
-        o.mu = mu
-        o.precision = PRECISIONS[precision]
-        o.orth_mode = ORTH_MODES[orth_mode]
-        o.kernel_path = KERNEL_PATHS[kernel_path]
-        o.fallback_cond = fallback_cond
-        o.orth_tol = orth_tol
-        o.max_wait_spins = max_wait_spins
-        self.options = o
+        self.options = _make_options(mu, precision, orth_mode, kernel_path, fallback_cond,
+                                     orth_tol, max_wait_spins, rmmc_threshold)
         h = c_void_p()
         ws = c_size_t()
-        _check(dion_init(descs, n, ctypes.byref(o), ctypes.byref(h), ctypes.byref(ws)),
+        _check(dion_init(_descs(self.shapes, scales), len(self.shapes),
+                         ctypes.byref(self.options), ctypes.byref(h), ctypes.byref(ws)),
                "dion_init")
         self._h = h
         self.workspace_bytes = ws.value
@@ -236,14 +271,16 @@ class DionB200:
         return host_status
 
     def view(self, bucket: int, which: int, workspace):
-        """P ([count, m, r]) or R ([count, n, r]) of the last step, as a view of the workspace."""
+        """P ([count, m, r]), R ([count, n, r]) or the momentum-change statistic RMMC
+        ([count]) of the last step, as a view of the workspace."""
         import torch
         ptr, nbytes = c_void_p(), c_size_t()
         _check(dion_workspace_view(self._h, bucket, which, c_void_p(workspace.data_ptr()),
                                    ctypes.byref(ptr), ctypes.byref(nbytes)), "dion_workspace_view")
         off = ptr.value - workspace.data_ptr()
         s = self.shapes[bucket]
-        shape = (s.count, s.m, s.r) if which == VIEW_P else (s.count, s.n, s.r)
+        shape = {VIEW_P: (s.count, s.m, s.r), VIEW_R: (s.count, s.n, s.r),
+                 VIEW_RMMC: (s.count,)}[which]
         return workspace[off:off + nbytes.value].view(torch.float32).view(*shape)
 
     @property
@@ -271,6 +308,92 @@ class DionB200:
             self.close()
         except Exception:
             pass
+
+
+# ---------------------------------------------------------------- row-sharded step
+def row_range(m: int, world: int, rank: int):
+    """Rows [row0, row0 + m_k) of rank ``rank`` when m rows are split as evenly as
+    possible among ``world`` ranks (the first m % world ranks take one row more)."""
+    base, extra = divmod(m, world)
+    return rank * base + min(rank, extra), base + (1 if rank < extra else 0)
+
+
+def _default_allreduce(buf):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(buf)
+
+
+class DionB200RowSharded(DionB200):
+    """This rank's rows of every matrix of a row-sharded step (include/dion.h,
+    dion_init_sharded).  ``buckets`` are the WHOLE shapes (count, m, n, r); rank
+    ``rank`` of ``world`` holds rows ``row_range(m, world, rank)`` of each, so the
+    tensors handed to ``step`` are X, M, G fp32 [count, m_k, n] and the whole Q
+    [count, n, r] (the same on every rank)."""
+
+    def __init__(self, buckets, rank: int, world: int, *, mu=0.95, precision="bf16",
+                 orth_mode="auto", fallback_cond=1e3, orth_tol=2e-5, max_wait_spins=1 << 26,
+                 scales=None, rmmc_threshold=0.0):
+        self.full_shapes = [Shape(*map(int, b)) for b in buckets]
+        self.rank, self.world = int(rank), int(world)
+        rows = [row_range(s.m, self.world, self.rank) for s in self.full_shapes]
+        self.row_ranges = rows
+        self.shapes = [Shape(s.count, mk, s.n, s.r) for s, (_, mk) in zip(self.full_shapes, rows)]
+        shards = (ShardDesc * max(len(self.shapes), 1))()
+        for i, (s, (row0, _)) in enumerate(zip(self.full_shapes, rows)):
+            shards[i].m_full, shards[i].row0 = s.m, row0
+        self.options = _make_options(mu, precision, orth_mode, "tensor", fallback_cond,
+                                     orth_tol, max_wait_spins, rmmc_threshold)
+        h = c_void_p()
+        ws = c_size_t()
+        _check(dion_init_sharded(_descs(self.shapes, scales), shards, len(self.shapes),
+                                 ctypes.byref(self.options), ctypes.byref(h), ctypes.byref(ws)),
+               "dion_init_sharded")
+        self._h = h
+        self.workspace_bytes = ws.value
+        self.num_matrices = dion_num_matrices(h)
+        self._x = Exchange()
+        self._ws = None
+
+    def _buffer(self):
+        """The current exchange's buffer as a float32 view of the workspace."""
+        import torch
+        off = self._x.d_buf - self._ws.data_ptr()
+        return self._ws[off:off + 4 * self._x.count].view(torch.float32)
+
+    def begin(self, X, M, G, Q, lr: float, workspace, status=None, stream=None):
+        """Start a step; returns (kind, buffer) of the first exchange."""
+        arr = self._ptrs(X, M, G, Q)
+        self._ws = workspace
+        _check(dion_step_sharded_begin(self._h, arr, len(self.shapes), float(lr),
+                                       c_void_p(workspace.data_ptr()), workspace.numel(),
+                                       c_void_p(status.data_ptr()) if status is not None else None,
+                                       self._stream(stream), ctypes.byref(self._x)),
+               "dion_step_sharded_begin")
+        return XCHG_NAMES[self._x.what], self._buffer()
+
+    def advance(self):
+        """After the current buffer was summed over the ranks; returns the next
+        (kind, buffer), or ("none", None) when the step is complete."""
+        _check(dion_step_sharded_continue(self._h, ctypes.byref(self._x)),
+               "dion_step_sharded_continue")
+        if self._x.count == 0:
+            return "none", None
+        return XCHG_NAMES[self._x.what], self._buffer()
+
+    def step(self, X, M, G, Q, lr: float, workspace, status=None, stream=None, allreduce=None):
+        """One row-sharded step.  ``allreduce(buf)`` sums a float32 CUDA tensor over the
+        ranks in place on the current stream (default: torch.distributed.all_reduce when a
+        process group of more than one rank exists, else nothing).  Returns the exchanges
+        as (kind, floats) pairs."""
+        reduce = allreduce or _default_allreduce
+        done = []
+        kind, buf = self.begin(X, M, G, Q, lr, workspace, status, stream)
+        while buf is not None:
+            done.append((kind, buf.numel()))
+            reduce(buf)
+            kind, buf = self.advance()
+        return done
 
 
 # ---------------------------------------------------------------- vector parameters

@@ -59,8 +59,12 @@ struct Plan {
   float scale;
   int64_t mat0;
   int nsplit;
+  // row-sharded plans: this rank holds rows [row0, row0 + m) of m_full-row matrices
+  // (m_full == m, row0 == 0 otherwise)
+  int64_t m_full, row0;
   size_t off_Bg, off_Qg, off_P0, off_P, off_P2, off_Pg, off_W, off_Linv, off_dinv, off_R, off_Rg,
-      off_Qng, off_part, off_flags, off_stats, off_P0s, off_Ps, off_Linvs, off_sched, off_Ws, off_Ts;
+      off_Qng, off_part, off_flags, off_stats, off_P0s, off_Ps, off_Linvs, off_sched, off_Ws, off_Ts,
+      off_gather, off_rmmc;
 };
 
 struct EventPair {
@@ -106,6 +110,23 @@ struct dion_ctx {
   cudaStream_t up;
   cudaEvent_t up_start;
   std::vector<cudaEvent_t> up_done;
+  // row-sharded plans: every bucket's Gram (W) and the per-bucket fallback counts lie
+  // in one block, every bucket's R in another, so each exchange is one all-reduce
+  bool sharded;
+  size_t off_wblk, wblk_floats, off_ctrl, off_rblk, rblk_floats;
+  // the sharded step in progress between dion_step_sharded_begin and its last
+  // dion_step_sharded_continue
+  struct ShardStep {
+    int stage;
+    std::vector<dion_bucket_ptrs> ptrs;
+    float lr;
+    char* ws;
+    int32_t* d_status;
+    cudaStream_t s;
+    std::vector<float> ctrl;   // per bucket: matrices needing the gathered fallback
+    int32_t gather_at;         // bucket whose gather is being exchanged
+    int launches;
+  } sh;
 };
 
 namespace {
@@ -125,6 +146,8 @@ dion_status check_options(const dion_options& o) {
   if (o.kernel_path != DION_PATH_TENSOR && o.kernel_path != DION_PATH_SIMT)
     return fail(DION_ERR_INVALID_ARG, "unknown kernel_path %d", o.kernel_path);
   if (o.max_wait_spins < 1) return fail(DION_ERR_INVALID_ARG, "max_wait_spins must be >= 1");
+  if (std::isnan(o.rmmc_threshold))
+    return fail(DION_ERR_INVALID_ARG, "rmmc_threshold is NaN");
   return DION_OK;
 }
 
@@ -137,6 +160,7 @@ struct StepCtx {
   EventPair* open;
   int open_at;
   std::vector<int> p0s_ready;  // per bucket: P0's split was written by B Q
+  bool sharded = false;        // R is a partial sum: column-norm partials from R itself
 };
 
 void begin_cls(StepCtx& c, int cls) {
@@ -338,6 +362,7 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
   int32_t* flags = reinterpret_cast<int32_t*>(ws + p.off_flags);
   float* stats = reinterpret_cast<float*>(ws + p.off_stats);
   int* sched = reinterpret_cast<int*>(ws + p.off_sched);
+  float* rmmc = reinterpret_cast<float*>(ws + p.off_rmmc);
   __nv_bfloat16* P0s = reinterpret_cast<__nv_bfloat16*>(ws + p.off_P0s);
   __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ps);
   __nv_bfloat16* Linvs = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Linvs);
@@ -350,7 +375,7 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
 
   if (phase == PH_INIT) {
     p0s_ready = 0;
-    DION_LAUNCH(c, 1, dion::launch_init_flags(flags, stats, sched, cnt,
+    DION_LAUNCH(c, 1, dion::launch_init_flags(flags, stats, sched, rmmc, cnt,
                                               o.orth_mode == DION_ORTH_HOUSEHOLDER ? DION_MAT_FALLBACK : 0,
                                               s));
     return DION_OK;
@@ -587,7 +612,7 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
   begin_cls(c, DION_KCLASS_COLNORM);
   DION_LAUNCH(c, 2,
               dion::launch_colnorm(R, bp.Q, Rg, Qng, bf ? 1 : (split ? 2 : 0), part, p.nsplit,
-                                   tensor, flags, cnt, n, r, s));
+                                   tensor && !c.sharded, flags, cnt, n, r, s));
   end_cls(c);
   return DION_OK;
   }
@@ -601,7 +626,7 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     if (tensor) {
       int nl = 0;
       cudaError_t e = dion::tc_update(Pg, Rg, Qng, split, bp.G, bp.M, bp.X, cnt, m, n, r, o.mu,
-                                      lrs, o.max_wait_spins, flags, sched, s, &nl, &done);
+                                      lrs, o.max_wait_spins, flags, sched, rmmc, s, &nl, &done);
       c.launches += nl;
       if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_update: %s", cudaGetErrorString(e));
       if (!done) return fail(DION_ERR_CUDA, "tc_update: %s", dion::tc_map_error());
@@ -609,14 +634,16 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     if (!done)
       DION_LAUNCH(c, (cnt + 65534) / 65535,
                   dion::launch_update_simt(Pg, Rg, Qng, bf, bp.G, bp.M, bp.X, cnt, m, n, r, o.mu,
-                                           lrs, s));
+                                           lrs, rmmc, s));
   }
   end_cls(c);
   return DION_OK;
   }
 
-  if (phase == PH_STATUS && d_status)
-    DION_LAUNCH(c, 1, dion::launch_write_status(flags, d_status + p.mat0, cnt, s));
+  // the per-matrix status and CurvaDion's momentum-change statistic (always computed)
+  if (phase == PH_STATUS)
+    DION_LAUNCH(c, 1, dion::launch_write_status(flags, rmmc, o.rmmc_threshold,
+                                                d_status ? d_status + p.mat0 : nullptr, cnt, s));
   return DION_OK;
 }
 
@@ -753,11 +780,13 @@ dion_status dion_default_options(dion_options* opt) {
   opt->orth_tol = 2e-5f;
   opt->kernel_path = DION_PATH_TENSOR;
   opt->max_wait_spins = int64_t(1) << 26;
+  opt->rmmc_threshold = 0.f;
   return DION_OK;
 }
 
-static dion_status dion_init_impl(const dion_bucket_desc* buckets, int32_t nbuckets, const dion_options* opt,
-                      dion_handle* out, size_t* workspace_bytes) {
+static dion_status dion_init_impl(const dion_bucket_desc* buckets, const dion_shard_desc* shards,
+                                  int32_t nbuckets, const dion_options* opt, dion_handle* out,
+                                  size_t* workspace_bytes) {
   if (!out || !workspace_bytes) return fail(DION_ERR_INVALID_ARG, "out or workspace_bytes is NULL");
   *out = nullptr;
   *workspace_bytes = 0;
@@ -766,6 +795,9 @@ static dion_status dion_init_impl(const dion_bucket_desc* buckets, int32_t nbuck
   if (opt) o = *opt; else dion_default_options(&o);
   dion_status st = check_options(o);
   if (st != DION_OK) return st;
+  const bool sharded = shards != nullptr;
+  if (sharded && o.kernel_path != DION_PATH_TENSOR)
+    return fail(DION_ERR_INVALID_ARG, "a row-sharded plan runs on the tensor path only");
   const bool bf = o.precision == DION_PREC_BF16;
   // fp32 precision on the tensor path keeps B, Q, P, R as three bf16 parts
   const bool split = !bf && o.kernel_path == DION_PATH_TENSOR;
@@ -780,61 +812,93 @@ static dion_status dion_init_impl(const dion_bucket_desc* buckets, int32_t nbuck
   };
   for (int32_t b = 0; b < nbuckets; ++b) {
     const dion_bucket_desc& d = buckets[b];
+    const int64_t m_full = sharded ? shards[b].m_full : d.m;
+    const int64_t row0 = sharded ? shards[b].row0 : 0;
     if (d.count < 1) return fail(DION_ERR_INVALID_ARG, "bucket %d: count %d < 1", b, d.count);
     if (d.count > 65535)
       return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: count %d exceeds 65535 (split the bucket)",
                   b, d.count);
     if (d.m < 1 || d.n < 1 || d.r < 1)
       return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: m, n, r must be positive", b);
-    if (d.r > d.m || d.r > d.n)
+    if (sharded && (row0 < 0 || m_full < d.m || row0 > m_full - d.m))
+      return fail(DION_ERR_INVALID_ARG,
+                  "bucket %d: rows [%lld, %lld) are not inside the %lld rows of the matrix", b,
+                  (long long)row0, (long long)(row0 + d.m), (long long)m_full);
+    if (d.r > m_full || d.r > d.n)
       return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: r=%lld exceeds min(m, n)", b, (long long)d.r);
     if (d.r % 16 != 0)
       return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: r=%lld is not a multiple of 16", b, (long long)d.r);
     if (d.n % 8 != 0)
       return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: n=%lld is not a multiple of 8", b, (long long)d.n);
-    if (d.m > (int64_t(1) << 30) || d.n > (int64_t(1) << 30) ||
-        (int64_t)d.count * d.m > kMaxElems / d.n || (int64_t)d.count * d.n > kMaxElems / d.r ||
-        (int64_t)d.count * d.m > kMaxElems / d.r)
+    if (m_full > (int64_t(1) << 30) || d.n > (int64_t(1) << 30) ||
+        (int64_t)d.count * m_full > kMaxElems / d.n || (int64_t)d.count * d.n > kMaxElems / d.r ||
+        (int64_t)d.count * m_full > kMaxElems / d.r)
       return fail(DION_ERR_UNSUPPORTED_SHAPE, "bucket %d: too large", b);
     if (!(std::isfinite(d.scale)))
       return fail(DION_ERR_INVALID_ARG, "bucket %d: scale is not finite", b);
     Plan p{};
     p.m = d.m; p.n = d.n; p.r = d.r; p.count = d.count;
-    p.scale = d.scale > 0.f ? d.scale : (float)std::sqrt((double)d.m / (double)d.n);
+    p.m_full = m_full; p.row0 = row0;
+    // s = sqrt(m / n) of the whole matrix, whatever rows this rank holds
+    p.scale = d.scale > 0.f ? d.scale : (float)std::sqrt((double)m_full / (double)d.n);
     p.mat0 = mats;
     mats += d.count;
     // column-norm partials: on the tensor path B^T P writes them, one per block of
     // R's rows (256 rows with bf16 operands, 32 rows from splits)
     p.nsplit = o.kernel_path != DION_PATH_TENSOR ? dion::colnorm_splits(d.count, d.n)
                : (bf ? dion::tc_btp_col_splits(d.n) : (int)(4 * ((d.n + 127) / 128)));
-    const size_t c = (size_t)d.count;
-    p.off_Bg = take(c * d.m * d.n * ge);
-    p.off_Qg = take(c * d.n * d.r * ge);
-    p.off_P0 = take(c * d.m * d.r * 4);
-    p.off_P = take(c * d.m * d.r * 4);
-    p.off_P2 = take(c * d.m * d.r * 4);
+    plans.push_back(p);
+  }
+  // A sharded plan places every bucket's Gram back to back, then one float per bucket
+  // (the fallback counts), then every bucket's R back to back: each exchange of the
+  // step is then a single all-reduce.  r % 16 == 0 and n % 8 == 0 keep every Gram a
+  // multiple of 1 KB and every R a multiple of 512 bytes.
+  size_t off_wblk = 0, wblk = 0, off_ctrl = 0, off_rblk = 0, rblk = 0;
+  if (sharded) {
+    for (Plan& p : plans) {
+      p.off_W = off_wblk + wblk * 4;
+      wblk += (size_t)p.count * p.r * p.r;
+    }
+    off_ctrl = off_wblk + wblk * 4;
+    off_rblk = align_up(off_ctrl + (size_t)nbuckets * 4, 1024);
+    for (Plan& p : plans) {
+      p.off_R = off_rblk + rblk * 4;
+      rblk += (size_t)p.count * p.n * p.r;
+    }
+    off = align_up(off_rblk + rblk * 4, 1024);
+  }
+  for (Plan& p : plans) {
+    const size_t c = (size_t)p.count;
+    p.off_Bg = take(c * p.m * p.n * ge);
+    p.off_Qg = take(c * p.n * p.r * ge);
+    p.off_P0 = take(c * p.m * p.r * 4);
+    p.off_P = take(c * p.m * p.r * 4);
+    p.off_P2 = take(c * p.m * p.r * 4);
     p.off_Pg = (bf || split) && !(bf && o.kernel_path == DION_PATH_TENSOR)
-                   ? take(c * d.m * d.r * ge) : 0;
-    p.off_W = take(c * d.r * d.r * 4);
-    p.off_Linv = take(c * d.r * d.r * 4);
-    p.off_dinv = take(dion::chol_dinv_floats(d.count, d.r) * 4);
-    p.off_R = take(c * d.n * d.r * 4);
-    p.off_Rg = (bf || split) ? take(c * d.n * d.r * ge) : 0;
-    p.off_Qng = (bf || split) ? take(c * d.n * d.r * ge) : 0;
-    p.off_part = take(c * p.nsplit * d.r * 4);
+                   ? take(c * p.m * p.r * ge) : 0;
+    if (!sharded) p.off_W = take(c * p.r * p.r * 4);
+    p.off_Linv = take(c * p.r * p.r * 4);
+    p.off_dinv = take(dion::chol_dinv_floats(p.count, p.r) * 4);
+    if (!sharded) p.off_R = take(c * p.n * p.r * 4);
+    p.off_Rg = (bf || split) ? take(c * p.n * p.r * ge) : 0;
+    p.off_Qng = (bf || split) ? take(c * p.n * p.r * ge) : 0;
+    p.off_part = take(c * p.nsplit * p.r * 4);
     p.off_flags = take(c * 4);
     p.off_stats = take(c * 4 * 4);
+    p.off_rmmc = take(c * 3 * 4);  // max |M' - M|, max |M|, their ratio: [3][count]
     // three-way bf16 splits for the tensor-core orthonormalisation
-    p.off_P0s = take(c * d.m * d.r * 6);
-    p.off_Ps = take(c * d.m * d.r * 6);
-    p.off_Linvs = take(c * d.r * d.r * 6);
+    p.off_P0s = take(c * p.m * p.r * 6);
+    p.off_Ps = take(c * p.m * p.r * 6);
+    p.off_Linvs = take(c * p.r * p.r * 6);
     p.off_sched = take(64);  // tile counters of the dynamically scheduled kernels
-    if (o.kernel_path == DION_PATH_TENSOR && d.r > 256) {
+    if (o.kernel_path == DION_PATH_TENSOR && p.r > 256) {
       // splits of the Gram / its updates and of L21 for the recursive factorisation
-      p.off_Ws = take(c * d.r * d.r * 6);
-      p.off_Ts = take(c * d.r * d.r * 6);
+      p.off_Ws = take(c * p.r * p.r * 6);
+      p.off_Ts = take(c * p.r * p.r * 6);
     }
-    plans.push_back(p);
+    // row-sharded fallback: the gathered P0 (its QR written in place) and the two
+    // column-major work arrays of Householder QR, each [count, m_full, r] fp32
+    if (sharded) p.off_gather = take(3 * c * p.m_full * p.r * 4);
   }
   dion_ctx* h = new (std::nothrow) dion_ctx();
   if (!h) return fail(DION_ERR_INVALID_ARG, "out of host memory");
@@ -855,6 +919,13 @@ static dion_status dion_init_impl(const dion_bucket_desc* buckets, int32_t nbuck
   h->up_device = -1;
   h->up = nullptr;
   h->up_start = nullptr;
+  h->sharded = sharded;
+  h->off_wblk = off_wblk;
+  h->wblk_floats = wblk;
+  h->off_ctrl = off_ctrl;
+  h->off_rblk = off_rblk;
+  h->rblk_floats = rblk;
+  h->sh.stage = 0;
   *out = h;
   *workspace_bytes = off;
   return DION_OK;
@@ -865,6 +936,8 @@ static dion_status dion_step_batched_impl(dion_handle h, const dion_bucket_ptrs*
                               int32_t* d_status, void* stream) {
   dion_status st = check_step_args(h, ptrs, nbuckets, d_workspace, workspace_bytes, d_status);
   if (st != DION_OK) return st;
+  if (h->sharded)
+    return fail(DION_ERR_INVALID_ARG, "a row-sharded plan steps through dion_step_sharded_begin");
   if (!std::isfinite(lr)) return fail(DION_ERR_INVALID_ARG, "lr is not finite");
   cudaStream_t main = reinterpret_cast<cudaStream_t>(stream);
   StepCtx c{h, main, 0, -1, nullptr, 0, std::vector<int>(nbuckets, 0)};
@@ -980,6 +1053,8 @@ static dion_status dion_step_batched_from_host_impl(dion_handle h, const dion_bu
                                         int32_t* d_status, int32_t* host_status, void* stream) {
   dion_status st = check_step_args(h, ptrs, nbuckets, d_workspace, workspace_bytes, d_status);
   if (st != DION_OK) return st;
+  if (h->sharded)
+    return fail(DION_ERR_INVALID_ARG, "a row-sharded plan steps through dion_step_sharded_begin");
   if (!host_grads || !host_status || !d_status)
     return fail(DION_ERR_INVALID_ARG, "host_grads, host_status and d_status are required");
   if (!std::isfinite(lr)) return fail(DION_ERR_INVALID_ARG, "lr is not finite");
@@ -1010,6 +1085,291 @@ static dion_status dion_step_batched_from_host_impl(dion_handle h, const dion_bu
   e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return fail(DION_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
   return DION_OK;
+}
+
+// ------------------------------------------------------------ row-sharded step
+// Rank k holds rows [row0, row0 + m) of every matrix; Q is replicated.  The step runs
+// as the whole-matrix step, except that four quantities are summed over the ranks by
+// the caller between the calls (an all-reduce of fp32 values):
+//   the Gram W = P0^T P0 of every bucket (before the Cholesky factorisation),
+//   the second pass's Gram and the per-bucket counts of matrices Cholesky-QR rejected,
+//   for a bucket with such matrices, its P0 gathered as zero-padded m_full x r blocks,
+//   R = B^T P of every bucket (before the column norms).
+// Every rank factorises the same summed Gram with the same deterministic kernels, so
+// every rank reaches the same decisions (second pass, fallback) and the same Q.
+enum ShardStage { SH_IDLE = 0, SH_GRAM1, SH_GRAM2, SH_GATHER, SH_R };
+
+struct ShardBufs {
+  float *W, *Linv, *dinv, *P, *P2, *stats, *gather;
+  int32_t* flags;
+  __nv_bfloat16 *P0s, *Ps, *Linvs, *Ws, *Ts;
+  void* Pg;
+};
+
+ShardBufs shard_bufs(const dion_options& o, const Plan& p, char* ws) {
+  const bool bf = o.precision == DION_PREC_BF16;
+  ShardBufs b{};
+  b.W = reinterpret_cast<float*>(ws + p.off_W);
+  b.Linv = reinterpret_cast<float*>(ws + p.off_Linv);
+  b.dinv = reinterpret_cast<float*>(ws + p.off_dinv);
+  b.P = reinterpret_cast<float*>(ws + p.off_P);
+  b.P2 = reinterpret_cast<float*>(ws + p.off_P2);
+  b.stats = reinterpret_cast<float*>(ws + p.off_stats);
+  b.gather = reinterpret_cast<float*>(ws + p.off_gather);
+  b.flags = reinterpret_cast<int32_t*>(ws + p.off_flags);
+  b.P0s = reinterpret_cast<__nv_bfloat16*>(ws + p.off_P0s);
+  b.Ps = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ps);
+  b.Linvs = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Linvs);
+  b.Ws = p.off_Ws ? reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ws) : nullptr;
+  b.Ts = p.off_Ts ? reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ts) : nullptr;
+  // the GEMM copy of P (as in run_bucket): bf16 is the leading plane of P's split
+  b.Pg = bf ? (void*)b.Ps : (void*)(ws + p.off_Pg);
+  return b;
+}
+
+#define DION_TC(ctx, call, what)                                                          \
+  do {                                                                                    \
+    int nl_ = 0;                                                                          \
+    bool done_ = false;                                                                   \
+    cudaError_t e_ = dion::call;                                                          \
+    (ctx).launches += nl_;                                                                \
+    if (e_ != cudaSuccess) return fail(DION_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e_)); \
+    if (!done_) return fail(DION_ERR_CUDA, "%s: %s", what, dion::tc_map_error());          \
+  } while (0)
+
+// Cholesky factorisation (pass 1 or 2) of the summed Gram of one bucket.
+dion_status shard_chol(StepCtx& c, const Plan& p, const ShardBufs& b, int pass) {
+  const dion_options& o = c.h->opt;
+  dion::CholArgs ca{};
+  ca.W = b.W; ca.Linv = b.Linv; ca.Linvs = b.Linvs; ca.dinv = b.dinv; ca.flags = b.flags;
+  ca.stats = b.stats; ca.count = p.count; ca.r = p.r; ca.m = p.m_full;
+  ca.fallback_cond = o.fallback_cond; ca.pass = pass;
+  ca.orth_tol = (pass == 2 && o.orth_mode == DION_ORTH_CHOLQR2) ? -1.f : o.orth_tol;
+  ca.dev_ready = 0;  // the summed Gram is read for max|W - I|: no epilogue measured it
+  if (p.r <= 256) {
+    DION_LAUNCH(c, 1, dion::launch_chol_inv(ca, c.s));
+    return DION_OK;
+  }
+  // the recursion reads the split of W's lower tiles: taken from the summed W
+  const int64_t rr = (int64_t)p.count * p.r * p.r;
+  DION_LAUNCH(c, 1, dion::launch_split3(b.W, b.Ws, rr, rr, c.s));
+  int nl = 0;
+  bool done = false;
+  const char* what = "";
+  cudaError_t e = dion::launch_chol_inv_rec(ca, b.Ws, b.Ts, o.max_wait_spins, c.s, &nl, &done,
+                                            &what);
+  c.launches += nl;
+  if (e != cudaSuccess)
+    return fail(DION_ERR_CUDA, "recursive factorisation (%s): %s", what, cudaGetErrorString(e));
+  if (!done) return fail(DION_ERR_CUDA, "recursive factorisation (%s): %s", what, dion::tc_map_error());
+  return DION_OK;
+}
+
+void shard_next(dion_exchange* x, float* buf, size_t count, int32_t what) {
+  x->d_buf = buf;
+  x->count = (int64_t)count;
+  x->what = what;
+}
+
+// After the gathers (or with none): the fallback's QR, the final P, and R = B^T P.
+dion_status shard_to_r(dion_handle h, StepCtx& c, dion_exchange* x) {
+  auto& sh = h->sh;
+  const dion_options& o = h->opt;
+  const bool bf = o.precision == DION_PREC_BF16;
+  for (size_t bi = 0; bi < h->plans.size(); ++bi) {
+    const Plan& p = h->plans[bi];
+    const ShardBufs b = shard_bufs(o, p, sh.ws);
+    begin_cls(c, DION_KCLASS_ORTH);
+    if (sh.ctrl[bi] > 0.5f) {
+      // Householder QR of the whole gathered P0, in place; this rank keeps its rows
+      const size_t full = (size_t)p.count * p.m_full * p.r;
+      DION_LAUNCH(c, 1, dion::launch_householder(b.gather, nullptr, b.gather + full,
+                                                 b.gather + 2 * full, b.gather, b.flags, p.count,
+                                                 p.m_full, p.r, c.s));
+      DION_LAUNCH(c, 1, dion::launch_rows_from_full(b.gather, b.P, b.flags, p.count, p.m,
+                                                    p.m_full, p.row0, p.r, c.s));
+    }
+    DION_LAUNCH(c, 1, dion::launch_finalize_p(b.P2, b.Pg, bf ? 1 : 2, b.flags, p.count, p.m, p.r,
+                                              b.P, o.orth_mode != DION_ORTH_HOUSEHOLDER, c.s));
+    end_cls(c);
+    dion_status st = run_bucket(c, (int)bi, PH_BTP, p, sh.ptrs[bi], sh.lr, sh.ws, sh.d_status);
+    if (st != DION_OK) return st;
+  }
+  sh.stage = SH_R;
+  shard_next(x, reinterpret_cast<float*>(sh.ws + h->off_rblk), h->rblk_floats, DION_XCHG_R);
+  return DION_OK;
+}
+
+dion_status shard_continue(dion_handle h, dion_exchange* x) {
+  auto& sh = h->sh;
+  const dion_options& o = h->opt;
+  const int32_t nb = (int32_t)h->plans.size();
+  StepCtx c{h, sh.s, 0, -1, nullptr, 0, std::vector<int>(nb, 1)};
+  c.sharded = true;
+  dion_status st = DION_OK;
+  auto done = [&](dion_status result) {
+    end_cls(c);
+    sh.launches += c.launches;
+    h->last_launches = sh.launches;
+    if (result != DION_OK) sh.stage = SH_IDLE;
+    return result;
+  };
+  if (sh.stage == SH_GRAM1) {
+    // pass 1 from the summed Gram, then this rank's part of the second pass's Gram and
+    // the number of matrices Cholesky-QR rejected
+    for (int32_t bi = 0; bi < nb; ++bi) {
+      const Plan& p = h->plans[bi];
+      const ShardBufs b = shard_bufs(o, p, sh.ws);
+      begin_cls(c, DION_KCLASS_ORTH);
+      if (o.orth_mode != DION_ORTH_HOUSEHOLDER) {
+        if ((st = shard_chol(c, p, b, 1)) != DION_OK) return done(st);
+        __nv_bfloat16* P1s = o.precision == DION_PREC_BF16 ? b.Ps
+                                                          : reinterpret_cast<__nv_bfloat16*>(b.Pg);
+        auto ap = [&]() -> dion_status {
+          DION_TC(c, tc_apply(b.P0s, b.Linvs, b.P, P1s, nullptr, p.count, p.m, p.r, b.flags, 0,
+                              DION_MAT_FALLBACK, o.max_wait_spins, c.s, &nl_, &done_),
+                  "tc_apply");
+          if (o.orth_mode != DION_ORTH_CHOLQR)
+            DION_TC(c, tc_gram(P1s, b.W, nullptr, nullptr, 0, p.count, p.m, p.r, b.flags, 0,
+                               DION_MAT_FALLBACK, o.max_wait_spins, c.s, &nl_, &done_),
+                    "tc_gram (second pass)");
+          return DION_OK;
+        };
+        if ((st = ap()) != DION_OK) return done(st);
+      }
+      float* ctrl = reinterpret_cast<float*>(sh.ws + h->off_ctrl) + bi;
+      DION_LAUNCH(c, 1, dion::launch_count_flags(b.flags, p.count, DION_MAT_FALLBACK, ctrl, c.s));
+      end_cls(c);
+    }
+    sh.stage = SH_GRAM2;
+    shard_next(x, reinterpret_cast<float*>(sh.ws + h->off_wblk), h->wblk_floats + nb,
+               DION_XCHG_GRAM2);
+    return done(DION_OK);
+  }
+  if (sh.stage == SH_GRAM2) {
+    // the summed counts decide, identically on every rank, which buckets gather P0
+    cudaError_t e = cudaMemcpyAsync(sh.ctrl.data(), sh.ws + h->off_ctrl, (size_t)nb * 4,
+                                    cudaMemcpyDeviceToHost, sh.s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(sh.s);
+    if (e != cudaSuccess)
+      return done(fail(DION_ERR_CUDA, "fallback counts: %s", cudaGetErrorString(e)));
+    int32_t first = -1;
+    for (int32_t bi = 0; bi < nb; ++bi) {
+      const Plan& p = h->plans[bi];
+      const ShardBufs b = shard_bufs(o, p, sh.ws);
+      begin_cls(c, DION_KCLASS_ORTH);
+      if (o.orth_mode != DION_ORTH_HOUSEHOLDER && o.orth_mode != DION_ORTH_CHOLQR) {
+        if ((st = shard_chol(c, p, b, 2)) != DION_OK) return done(st);
+        __nv_bfloat16* P1s = o.precision == DION_PREC_BF16 ? b.Ps
+                                                          : reinterpret_cast<__nv_bfloat16*>(b.Pg);
+        auto ap = [&]() -> dion_status {
+          DION_TC(c, tc_apply(P1s, b.Linvs, b.P2, nullptr, nullptr, p.count, p.m, p.r, b.flags,
+                              DION_MAT_CHOLQR2, DION_MAT_FALLBACK, o.max_wait_spins, c.s, &nl_,
+                              &done_),
+                  "tc_apply (second pass)");
+          return DION_OK;
+        };
+        if ((st = ap()) != DION_OK) return done(st);
+      }
+      if (sh.ctrl[bi] > 0.5f) {
+        const size_t full = (size_t)p.count * p.m_full * p.r;
+        cudaError_t e2 = cudaMemsetAsync(b.gather, 0, full * 4, sh.s);
+        if (e2 != cudaSuccess) return done(fail(DION_ERR_CUDA, "gather: %s", cudaGetErrorString(e2)));
+        DION_LAUNCH(c, 1, dion::launch_rows_to_full(nullptr, b.P0s, b.gather, p.count, p.m,
+                                                    p.m_full, p.row0, p.r, sh.s));
+        if (first < 0) first = bi;
+      }
+      end_cls(c);
+    }
+    if (first >= 0) {
+      const Plan& p = h->plans[first];
+      sh.stage = SH_GATHER;
+      sh.gather_at = first;
+      shard_next(x, reinterpret_cast<float*>(sh.ws + p.off_gather),
+                 (size_t)p.count * p.m_full * p.r, DION_XCHG_GATHER);
+      return done(DION_OK);
+    }
+    return done(shard_to_r(h, c, x));
+  }
+  if (sh.stage == SH_GATHER) {
+    for (int32_t bi = sh.gather_at + 1; bi < nb; ++bi)
+      if (sh.ctrl[bi] > 0.5f) {
+        const Plan& p = h->plans[bi];
+        sh.gather_at = bi;
+        shard_next(x, reinterpret_cast<float*>(sh.ws + p.off_gather),
+                   (size_t)p.count * p.m_full * p.r, DION_XCHG_GATHER);
+        return done(DION_OK);
+      }
+    return done(shard_to_r(h, c, x));
+  }
+  if (sh.stage == SH_R) {
+    // Q from the summed R on every rank, then this rank's rows of M and X
+    for (int32_t bi = 0; bi < nb; ++bi)
+      for (int phase : {PH_COLNORM, PH_UPDATE, PH_STATUS})
+        if ((st = run_bucket(c, bi, phase, h->plans[bi], sh.ptrs[bi], sh.lr, sh.ws,
+                             sh.d_status)) != DION_OK)
+          return done(st);
+    sh.stage = SH_IDLE;
+    shard_next(x, nullptr, 0, DION_XCHG_NONE);
+    return done(DION_OK);
+  }
+  return done(fail(DION_ERR_INVALID_ARG, "no row-sharded step in progress"));
+}
+
+static dion_status dion_step_sharded_begin_impl(dion_handle h, const dion_bucket_ptrs* ptrs,
+                                                int32_t nbuckets, float lr, void* d_workspace,
+                                                size_t workspace_bytes, int32_t* d_status,
+                                                void* stream, dion_exchange* next) {
+  if (!next) return fail(DION_ERR_INVALID_ARG, "next is NULL");
+  shard_next(next, nullptr, 0, DION_XCHG_NONE);
+  dion_status st = check_step_args(h, ptrs, nbuckets, d_workspace, workspace_bytes, d_status);
+  if (st != DION_OK) return st;
+  if (!h->sharded) return fail(DION_ERR_INVALID_ARG, "the plan is not row-sharded (dion_init_sharded)");
+  if (h->sh.stage != SH_IDLE)
+    return fail(DION_ERR_INVALID_ARG, "a row-sharded step is already in progress on this handle");
+  if (!std::isfinite(lr)) return fail(DION_ERR_INVALID_ARG, "lr is not finite");
+  auto& sh = h->sh;
+  sh.ptrs.assign(ptrs, ptrs + nbuckets);
+  sh.lr = lr;
+  sh.ws = static_cast<char*>(d_workspace);
+  sh.d_status = d_status;
+  sh.s = reinterpret_cast<cudaStream_t>(stream);
+  sh.ctrl.assign((size_t)nbuckets, 0.f);
+  sh.gather_at = -1;
+  sh.launches = 0;
+  StepCtx c{h, sh.s, 0, -1, nullptr, 0, std::vector<int>(nbuckets, 0)};
+  c.sharded = true;
+  auto finish = [&](dion_status result) {
+    end_cls(c);
+    sh.launches += c.launches;
+    h->last_launches = sh.launches;
+    return result;
+  };
+  for (int phase : {PH_INIT, PH_PREPQ})
+    for (int32_t b = 0; b < nbuckets; ++b)
+      if ((st = run_bucket(c, b, phase, h->plans[b], ptrs[b], lr, sh.ws, d_status)) != DION_OK)
+        return finish(st);
+  // B = M + G and P0 = B Q on this rank's rows, then its part of each Gram
+  for (int32_t b = 0; b < nbuckets; ++b) {
+    for (int phase : {PH_FORMB, PH_BQ})
+      if ((st = run_bucket(c, b, phase, h->plans[b], ptrs[b], lr, sh.ws, d_status)) != DION_OK)
+        return finish(st);
+    const Plan& p = h->plans[b];
+    const ShardBufs sb = shard_bufs(h->opt, p, sh.ws);
+    begin_cls(c, DION_KCLASS_ORTH);
+    auto gram = [&]() -> dion_status {
+      DION_TC(c, tc_gram(sb.P0s, sb.W, nullptr, nullptr, 0, p.count, p.m, p.r, sb.flags, 0,
+                         DION_MAT_FALLBACK, h->opt.max_wait_spins, sh.s, &nl_, &done_),
+              "tc_gram");
+      return DION_OK;
+    };
+    if (h->opt.orth_mode != DION_ORTH_HOUSEHOLDER && (st = gram()) != DION_OK) return finish(st);
+    end_cls(c);
+  }
+  sh.stage = SH_GRAM1;
+  shard_next(next, reinterpret_cast<float*>(sh.ws + h->off_wblk), h->wblk_floats,
+             DION_XCHG_GRAM);
+  return finish(DION_OK);
 }
 
 static dion_status dion_free_impl(dion_handle h) {
@@ -1066,6 +1426,9 @@ static dion_status dion_workspace_view_impl(dion_handle h, int32_t bucket, int32
   } else if (which == DION_VIEW_R) {
     *d_ptr = ws + p.off_R;
     *bytes = (size_t)p.count * p.n * p.r * 4;
+  } else if (which == DION_VIEW_RMMC) {
+    *d_ptr = ws + p.off_rmmc + (size_t)2 * p.count * 4;
+    *bytes = (size_t)p.count * 4;
   } else {
     return fail(DION_ERR_INVALID_ARG, "unknown view %d", which);
   }
@@ -1104,8 +1467,9 @@ static dion_status dion_profile_read_impl(dion_handle h, double* ms, int64_t* la
 
 dion_status dion_init(const dion_bucket_desc* buckets, int32_t nbuckets, const dion_options* opt,
                       dion_handle* out, size_t* workspace_bytes) {
-  return guarded("dion_init",
-                 [&] { return dion_init_impl(buckets, nbuckets, opt, out, workspace_bytes); });
+  return guarded("dion_init", [&] {
+    return dion_init_impl(buckets, nullptr, nbuckets, opt, out, workspace_bytes);
+  });
 }
 
 dion_status dion_step_batched(dion_handle h, const dion_bucket_ptrs* ptrs, int32_t nbuckets,
@@ -1129,6 +1493,37 @@ dion_status dion_step_batched_from_host(dion_handle h, const dion_bucket_ptrs* p
 
 dion_status dion_free(dion_handle h) {
   return guarded("dion_free", [&] { return dion_free_impl(h); });
+}
+
+dion_status dion_init_sharded(const dion_bucket_desc* buckets, const dion_shard_desc* shards,
+                              int32_t nbuckets, const dion_options* opt, dion_handle* out,
+                              size_t* workspace_bytes) {
+  return guarded("dion_init_sharded", [&] {
+    if (!shards) return fail(DION_ERR_INVALID_ARG, "shards is NULL");
+    return dion_init_impl(buckets, shards, nbuckets, opt, out, workspace_bytes);
+  });
+}
+
+dion_status dion_step_sharded_begin(dion_handle h, const dion_bucket_ptrs* ptrs,
+                                    int32_t nbuckets, float lr, void* d_workspace,
+                                    size_t workspace_bytes, int32_t* d_status, void* stream,
+                                    dion_exchange* next) {
+  // the step's state is recorded only once every launch of this call succeeded
+  return guarded("dion_step_sharded_begin", [&] {
+    return dion_step_sharded_begin_impl(h, ptrs, nbuckets, lr, d_workspace, workspace_bytes,
+                                        d_status, stream, next);
+  });
+}
+
+dion_status dion_step_sharded_continue(dion_handle h, dion_exchange* next) {
+  return guarded("dion_step_sharded_continue", [&] {
+    if (!valid(h)) return fail(DION_ERR_NOT_INITIALIZED, "invalid or freed handle");
+    if (!next) return fail(DION_ERR_INVALID_ARG, "next is NULL");
+    shard_next(next, nullptr, 0, DION_XCHG_NONE);
+    if (!h->sharded || h->sh.stage == SH_IDLE)
+      return fail(DION_ERR_INVALID_ARG, "no row-sharded step in progress");
+    return shard_continue(h, next);
+  });
 }
 
 dion_status dion_workspace_view(dion_handle h, int32_t bucket, int32_t which, void* d_workspace,

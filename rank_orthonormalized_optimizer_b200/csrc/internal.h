@@ -47,7 +47,7 @@ cudaError_t launch_prep_q_split(const float* Q, void* Qs, int count, int64_t n, 
                                 cudaStream_t s);
 // Zero the per-matrix flags (or set init_bits), the Cholesky statistics and the 16
 // tile counters of the bucket's dynamically scheduled kernels.
-cudaError_t launch_init_flags(int32_t* flags, float* stats, int* sched, int count,
+cudaError_t launch_init_flags(int32_t* flags, float* stats, int* sched, float* rmmc, int count,
                               int32_t init_bits, cudaStream_t s);
 // mode 0: fp32 P only; 1: + bf16 copy Pg; 2: + three-way bf16 split Pg.  pg_ready: Pg
 // already holds the first pass's P; only second-pass and fallback matrices are written.
@@ -63,14 +63,30 @@ cudaError_t launch_colnorm(const float* R, float* Q, void* Rg, void* Qg, int mod
                            int64_t n, int64_t r, cudaStream_t s);
 cudaError_t launch_split3(const float* src, void* dst, int64_t n, int64_t dst_stride,
                           cudaStream_t s);
-cudaError_t launch_write_status(const int32_t* flags, int32_t* d_status, int count,
+// RMMC = max |M' - M| / max |M| per matrix (rmmc: [3][count], the third plane written;
+// +inf for a zero M that changed, 0 for one that did not) and, when d_status is not
+// null, the public flag bits with DION_MAT_HIGH_RMMC where RMMC > rmmc_threshold.
+cudaError_t launch_write_status(const int32_t* flags, float* rmmc, float rmmc_threshold,
+                                int32_t* d_status, int count, cudaStream_t s);
+// Row-sharded step: this rank's rows [row0, row0 + m) of P0 (fp32, or its three-way
+// split when P0s is not null) into the zeroed m_full x r buffers `full`; the flagged
+// matrices' rows back from `full` into P; the number of matrices with (flags & mask).
+cudaError_t launch_rows_to_full(const float* P0, const void* P0s, float* full, int count,
+                                int64_t m, int64_t m_full, int64_t row0, int64_t r,
                                 cudaStream_t s);
+cudaError_t launch_rows_from_full(const float* full, float* P, const int32_t* flags, int count,
+                                  int64_t m, int64_t m_full, int64_t row0, int64_t r,
+                                  cudaStream_t s);
+cudaError_t launch_count_flags(const int32_t* flags, int count, int32_t mask, float* out,
+                               cudaStream_t s);
 
 // ---- SIMT contractions (k_gemm_simt.cu)
 cudaError_t launch_gemm_simt(const GemmDesc& d, bool bf16_operands, cudaStream_t s);
+// rmmc: [2][count], max |M' - M| and max |M| of each matrix max-ed into them
 cudaError_t launch_update_simt(const void* Pg, const void* Rg, const void* Qg, bool use_bf16,
                                const float* G, float* M, float* X, int count, int64_t m,
-                               int64_t n, int64_t r, float mu, float lr_scale, cudaStream_t s);
+                               int64_t n, int64_t r, float mu, float lr_scale, float* rmmc,
+                               cudaStream_t s);
 
 // ---- orthonormalisation (k_orth.cu)
 // pass 1: Cholesky of W = P0^T P0; pass 2: checks W = P1^T P1 first.

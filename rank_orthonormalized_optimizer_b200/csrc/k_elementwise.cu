@@ -200,7 +200,7 @@ cudaError_t launch_split3(const float* src, void* dst, int64_t n, int64_t dst_st
 }
 
 // ---------------------------------------------------------- flags and status
-__global__ void k_init_flags(int32_t* flags, float* stats, int* sched, int count,
+__global__ void k_init_flags(int32_t* flags, float* stats, int* sched, float* rmmc, int count,
                              int32_t init_bits) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < 16) sched[b] = 0;
@@ -210,24 +210,105 @@ __global__ void k_init_flags(int32_t* flags, float* stats, int* sched, int count
     stats[ST * b + 1] = 0.f;     // running max of diag(L)
     stats[ST * b + 2] = 0.f;
     stats[ST * b + 3] = 0.f;
+    rmmc[b] = 0.f;               // max |M' - M|, max-ed into by the update
+    rmmc[count + b] = 0.f;       // max |M|
   }
 }
 
-cudaError_t launch_init_flags(int32_t* flags, float* stats, int* sched, int count,
+cudaError_t launch_init_flags(int32_t* flags, float* stats, int* sched, float* rmmc, int count,
                               int32_t init_bits, cudaStream_t s) {
   const int n = count > 16 ? count : 16;
-  k_init_flags<<<(n + 255) / 256, 256, 0, s>>>(flags, stats, sched, count, init_bits);
+  k_init_flags<<<(n + 255) / 256, 256, 0, s>>>(flags, stats, sched, rmmc, count, init_bits);
   return cudaGetLastError();
 }
 
-__global__ void k_write_status(const int32_t* flags, int32_t* st, int count) {
+// CurvaDion's statistic from the update's maxima (the relative maximum momentum change):
+// RMMC = max |M' - M| / max |M|, and the gate bit where it exceeds the threshold.
+__global__ void k_write_status(const int32_t* flags, float* rmmc, float tau, int32_t* st,
+                               int count) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < count) st[b] = flags[b] & F_PUBLIC;
+  if (b >= count) return;
+  const float num = rmmc[b], den = rmmc[count + b];
+  const float v = den > 0.f ? num / den : (num > 0.f ? INFINITY : 0.f);
+  rmmc[2 * count + b] = v;
+  if (st) st[b] = (flags[b] & F_PUBLIC) | (v > tau ? DION_MAT_HIGH_RMMC : 0);
 }
 
-cudaError_t launch_write_status(const int32_t* flags, int32_t* d_status, int count,
+cudaError_t launch_write_status(const int32_t* flags, float* rmmc, float rmmc_threshold,
+                                int32_t* d_status, int count, cudaStream_t s) {
+  k_write_status<<<(count + 255) / 256, 256, 0, s>>>(flags, rmmc, rmmc_threshold, d_status,
+                                                     count);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------ row-sharded step: P0 gather
+// In a row-sharded step every rank holds rows [row0, row0 + m) of each matrix's P0.
+// When a matrix needs the Householder fallback the whole P0 is assembled by summing,
+// over ranks, m_full x r buffers that hold only the rank's own rows (zero elsewhere).
+// Its rows go into `full` (zeroed beforehand); P0 is read in fp32, or as the sum of its
+// three bf16 parts when P0s is not null (planes `plane` elements apart).
+__global__ void k_rows_to_full(const float* __restrict__ P0, const bf16* __restrict__ P0s,
+                               int64_t plane, float* __restrict__ full, int64_t m,
+                               int64_t m_full, int64_t row0, int64_t r) {
+  const int64_t b = blockIdx.y;
+  const int64_t mr = m * r;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < mr;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t src = b * mr + e;
+    const float v = P0s ? (__bfloat162float(P0s[src]) + __bfloat162float(P0s[src + plane])) +
+                              __bfloat162float(P0s[src + 2 * plane])
+                        : P0[src];
+    full[b * m_full * r + row0 * r + e] = v;
+  }
+}
+
+cudaError_t launch_rows_to_full(const float* P0, const void* P0s, float* full, int count,
+                                int64_t m, int64_t m_full, int64_t row0, int64_t r,
                                 cudaStream_t s) {
-  k_write_status<<<(count + 255) / 256, 256, 0, s>>>(flags, d_status, count);
+  int64_t gx = (m * r + 255) / 256;
+  if (gx > 64) gx = 64;
+  k_rows_to_full<<<dim3((unsigned)gx, (unsigned)count), 256, 0, s>>>(
+      P0, (const bf16*)P0s, (int64_t)count * m * r, full, m, m_full, row0, r);
+  return cudaGetLastError();
+}
+
+// P[b] (m x r) = rows [row0, row0 + m) of full[b] (m_full x r), for the matrices
+// flagged F_FALLBACK only (the others keep their Cholesky-QR result).
+__global__ void k_rows_from_full(const float* __restrict__ full, float* __restrict__ P,
+                                 const int32_t* __restrict__ flags, int64_t m,
+                                 int64_t m_full, int64_t row0, int64_t r) {
+  const int64_t b = blockIdx.y;
+  if (!(flags[b] & F_FALLBACK)) return;
+  const int64_t mr = m * r;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < mr;
+       e += (int64_t)gridDim.x * blockDim.x)
+    P[b * mr + e] = full[b * m_full * r + row0 * r + e];
+}
+
+cudaError_t launch_rows_from_full(const float* full, float* P, const int32_t* flags, int count,
+                                  int64_t m, int64_t m_full, int64_t row0, int64_t r,
+                                  cudaStream_t s) {
+  int64_t gx = (m * r + 255) / 256;
+  if (gx > 64) gx = 64;
+  k_rows_from_full<<<dim3((unsigned)gx, (unsigned)count), 256, 0, s>>>(full, P, flags, m,
+                                                                        m_full, row0, r);
+  return cudaGetLastError();
+}
+
+// *out = the number of matrices with (flags & mask) != 0, as a float (one block; the
+// count is exact far beyond 65535 matrices).
+__global__ void __launch_bounds__(256) k_count_flags(const int32_t* flags, int count,
+                                                     int32_t mask, float* out) {
+  __shared__ float red[32];
+  float c = 0.f;
+  for (int b = threadIdx.x; b < count; b += 256) c += (flags[b] & mask) ? 1.f : 0.f;
+  c = block_sum<256>(c, red);
+  if (threadIdx.x == 0) *out = c;
+}
+
+cudaError_t launch_count_flags(const int32_t* flags, int count, int32_t mask, float* out,
+                               cudaStream_t s) {
+  k_count_flags<<<1, 256, 0, s>>>(flags, count, mask, out);
   return cudaGetLastError();
 }
 

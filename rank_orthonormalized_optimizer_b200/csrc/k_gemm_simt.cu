@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(NT) k_update_simt(const T* __restrict__ Pg,
                                                      const float* __restrict__ G,
                                                      float* __restrict__ M, float* __restrict__ X,
                                                      int64_t m, int64_t n, int64_t r,
-                                                     float one_minus_mu, float lr_scale) {
+                                                     float one_minus_mu, float lr_scale,
+                                                     float* __restrict__ rmmc, int batch) {
   __shared__ __align__(16) float Ps[BK][BM + 4];
   __shared__ __align__(16) float Rs[BK][BN + 4];
   __shared__ __align__(16) float Qs[BK][BN + 4];
@@ -183,32 +184,47 @@ __global__ void __launch_bounds__(NT) k_update_simt(const T* __restrict__ Pg,
     __syncthreads();
   }
   const int64_t j = j0 + tx * 4;
-  if (j >= n) return;
+  // momentum-change statistics: max |M' - M| and max |M| over this thread's elements
+  float dmax = 0.f, mmax = 0.f;
+  if (j < n) {
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int64_t i = i0 + ty * 4 + a;
-    if (i >= m) continue;
-    const int64_t e = b * m * n + i * n + j;
-    const float4 mv = *reinterpret_cast<const float4*>(M + e);
-    const float4 gv = __ldcs(reinterpret_cast<const float4*>(G + e));
-    const float4 xv = *reinterpret_cast<const float4*>(X + e);
-    float4 mo, xo;
-    mo.x = (mv.x + gv.x) - one_minus_mu * a1[a][0];
-    mo.y = (mv.y + gv.y) - one_minus_mu * a1[a][1];
-    mo.z = (mv.z + gv.z) - one_minus_mu * a1[a][2];
-    mo.w = (mv.w + gv.w) - one_minus_mu * a1[a][3];
-    xo.x = xv.x - lr_scale * a2[a][0];
-    xo.y = xv.y - lr_scale * a2[a][1];
-    xo.z = xv.z - lr_scale * a2[a][2];
-    xo.w = xv.w - lr_scale * a2[a][3];
-    *reinterpret_cast<float4*>(M + e) = mo;
-    *reinterpret_cast<float4*>(X + e) = xo;
+    for (int a = 0; a < 4; ++a) {
+      const int64_t i = i0 + ty * 4 + a;
+      if (i >= m) continue;
+      const int64_t e = b * m * n + i * n + j;
+      const float4 mv = *reinterpret_cast<const float4*>(M + e);
+      const float4 gv = __ldcs(reinterpret_cast<const float4*>(G + e));
+      const float4 xv = *reinterpret_cast<const float4*>(X + e);
+      float4 mo, xo;
+      mo.x = (mv.x + gv.x) - one_minus_mu * a1[a][0];
+      mo.y = (mv.y + gv.y) - one_minus_mu * a1[a][1];
+      mo.z = (mv.z + gv.z) - one_minus_mu * a1[a][2];
+      mo.w = (mv.w + gv.w) - one_minus_mu * a1[a][3];
+      xo.x = xv.x - lr_scale * a2[a][0];
+      xo.y = xv.y - lr_scale * a2[a][1];
+      xo.z = xv.z - lr_scale * a2[a][2];
+      xo.w = xv.w - lr_scale * a2[a][3];
+      dmax = fmaxf(dmax, fmaxf(fmaxf(fabsf(mo.x - mv.x), fabsf(mo.y - mv.y)),
+                               fmaxf(fabsf(mo.z - mv.z), fabsf(mo.w - mv.w))));
+      mmax = fmaxf(mmax, fmaxf(fmaxf(fabsf(mv.x), fabsf(mv.y)), fmaxf(fabsf(mv.z), fabsf(mv.w))));
+      *reinterpret_cast<float4*>(M + e) = mo;
+      *reinterpret_cast<float4*>(X + e) = xo;
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+    mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+  }
+  if ((threadIdx.x & 31) == 0) {
+    atomic_max_pos(rmmc + b, dmax);
+    atomic_max_pos(rmmc + batch + b, mmax);
   }
 }
 
 cudaError_t launch_update_simt(const void* Pg, const void* Rg, const void* Qg, bool use_bf16,
                                const float* G, float* M, float* X, int count, int64_t m,
-                               int64_t n, int64_t r, float mu, float lr_scale, cudaStream_t s) {
+                               int64_t n, int64_t r, float mu, float lr_scale, float* rmmc,
+                               cudaStream_t s) {
   for (int b0 = 0; b0 < count; b0 += 65535) {
     const int nb = (count - b0) < 65535 ? (count - b0) : 65535;
     dim3 grid((unsigned)((n + BN - 1) / BN), (unsigned)((m + BM - 1) / BM), (unsigned)nb);
@@ -217,12 +233,12 @@ cudaError_t launch_update_simt(const void* Pg, const void* Rg, const void* Qg, b
       k_update_simt<bf16><<<grid, NT, 0, s>>>(
           (const bf16*)Pg + (size_t)b0 * m * r, (const bf16*)Rg + (size_t)b0 * n * r,
           (const bf16*)Qg + (size_t)b0 * n * r, G + mn, M + mn, X + mn, m, n, r, 1.f - mu,
-          lr_scale);
+          lr_scale, rmmc + b0, count);
     else
       k_update_simt<float><<<grid, NT, 0, s>>>(
           (const float*)Pg + (size_t)b0 * m * r, (const float*)Rg + (size_t)b0 * n * r,
           (const float*)Qg + (size_t)b0 * n * r, G + mn, M + mn, X + mn, m, n, r, 1.f - mu,
-          lr_scale);
+          lr_scale, rmmc + b0, count);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

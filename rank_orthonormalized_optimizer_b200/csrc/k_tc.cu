@@ -1148,6 +1148,7 @@ struct UpdP {
   int npairs;         // 1: bf16 operands; 3: split operands, products (1,0) (0,1) (0,0)
   int pa[3], pb[3];   // part of P and of R, Q in each product
   int64_t max_spins;
+  float* rmmc;        // [2][batch]: max |M' - M| and max |M| per matrix (max-ed into)
 };
 
 // Tiles are handed out in order from a global counter rather than dealt round-robin:
@@ -1361,6 +1362,9 @@ __global__ void __launch_bounds__(NT, 1)
       const int m0 = (rem / p.tiles_n) * BM;
       const int n0 = (rem % p.tiles_n) * UPD_BN;
       const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * 256;
+      // momentum-change statistics of the tile (out-of-range rows and columns load as
+      // zeros and change by zero, so they do not count)
+      float dmax = 0.f, mmax = 0.f;
       for (int sl = 0; sl < NSLAB; ++sl) {
         float ar[32], aq[32];
         tmem_ld32(tbase + sl * SLAB, ar);
@@ -1382,10 +1386,15 @@ __global__ void __launch_bounds__(NT, 1)
           float4 mv = *reinterpret_cast<const float4*>(rm + off);
           const float4 gv = *reinterpret_cast<const float4*>(rg + off);
           float4 xv = *reinterpret_cast<const float4*>(rx + off);
+          const float4 m_old = mv;
           mv.x = (mv.x + gv.x) - p.omm * ar[4 * c + 0];
           mv.y = (mv.y + gv.y) - p.omm * ar[4 * c + 1];
           mv.z = (mv.z + gv.z) - p.omm * ar[4 * c + 2];
           mv.w = (mv.w + gv.w) - p.omm * ar[4 * c + 3];
+          dmax = fmaxf(dmax, fmaxf(fmaxf(fabsf(mv.x - m_old.x), fabsf(mv.y - m_old.y)),
+                                   fmaxf(fabsf(mv.z - m_old.z), fabsf(mv.w - m_old.w))));
+          mmax = fmaxf(mmax, fmaxf(fmaxf(fabsf(m_old.x), fabsf(m_old.y)),
+                                   fmaxf(fabsf(m_old.z), fabsf(m_old.w))));
           xv.x = xv.x - p.lrs * aq[4 * c + 0];
           xv.y = xv.y - p.lrs * aq[4 * c + 1];
           xv.z = xv.z - p.lrs * aq[4 * c + 2];
@@ -1406,6 +1415,14 @@ __global__ void __launch_bounds__(NT, 1)
         if (++stage == SLAB_STAGES) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;  // t stays on the unfinished tile
+      for (int o = 16; o > 0; o >>= 1) {
+        dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+        mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+      }
+      if (lane == 0) {
+        atomic_max_pos(p.rmmc + b, dmax);
+        atomic_max_pos(p.rmmc + p.batch + b, mmax);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + acc);
@@ -1427,7 +1444,7 @@ __global__ void __launch_bounds__(NT, 1)
 cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, bool split, const float* G,
                       float* M, float* X, int count, int64_t m, int64_t n, int64_t r, float mu,
                       float lr_scale, int64_t max_spins, int32_t* flags, int* tile_counter,
-                      cudaStream_t s, int* nlaunch, bool* done) {
+                      float* rmmc, cudaStream_t s, int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
@@ -1455,6 +1472,7 @@ cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, bool split
   p.pa[1] = 0; p.pb[1] = split ? 1 : 0;
   p.pa[2] = 0; p.pb[2] = 0;
   p.max_spins = max_spins;
+  p.rmmc = rmmc;
   cudaError_t e = cudaFuncSetAttribute(k_tc_update, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)UPD_SMEM);
   if (e != cudaSuccess) return e;

@@ -36,10 +36,12 @@ int tc_btp_col_splits(int64_t n);
 // M <- (M + G) - (1 - mu) Pg Rg^T and X <- X - lr_scale Pg Qg^T (Pg: m x r, Rg, Qg: n x r, bf16).
 // tile_counter: one int in device memory, zero before the call (tiles are taken from it).
 // split: Pg, Rg, Qg are three-way bf16 splits ([3][count][...]) of fp32 operands.
+// rmmc: [2][count] floats, max |M' - M| and max |M| of each matrix max-ed into them
+// (non-negative before the call).
 cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, bool split, const float* G,
                       float* M, float* X, int count, int64_t m, int64_t n, int64_t r, float mu,
                       float lr_scale, int64_t max_spins, int32_t* flags, int* tile_counter,
-                      cudaStream_t s, int* nlaunch, bool* done);
+                      float* rmmc, cudaStream_t s, int* nlaunch, bool* done);
 // fp32 contractions from three-way bf16 splits: P0s = split(Bs Qs^T), R = Bs^T Ps.
 cudaError_t tc_gemm_bq_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Qs,
                              __nv_bfloat16* P0s, int count, int64_t m, int64_t n, int64_t r,
