@@ -420,8 +420,9 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
   } else if (split) {
     int nl = 0;
     bool done = false;
-    cudaError_t e = dion::tc_gemm_bq_split((const __nv_bfloat16*)Bg, (const __nv_bfloat16*)Qg, P0s,
-                                           cnt, m, n, r, o.max_wait_spins, flags, s, &nl, &done);
+    cudaError_t e = dion::tc_gemm_bq_split((const __nv_bfloat16*)Bg, (const __nv_bfloat16*)Qg, P0,
+                                           P0s, cnt, m, n, r, o.max_wait_spins, flags, s, &nl,
+                                           &done);
     c.launches += nl;
     if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_gemm_bq_split: %s", cudaGetErrorString(e));
     if (!done) return fail(DION_ERR_CUDA, "tc_gemm_bq_split: %s", dion::tc_map_error());
@@ -529,9 +530,12 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
         // the second pass's Gram also measures max|W - I| per matrix (statistics slot 2,
         // zero since the step began), so that its factorisation can skip matrices the
         // first pass left orthonormal without reading W
+        // P1 is orthonormal to about cond(P0)^2 u already: its Gram needs only the two
+        // leading parts of its split (three products, about 2^-17 relative, far below
+        // orth_tol and below what the second factorisation needs)
         e = dion::tc_gram(P1s, W, Ws, r <= 256 ? stats + 2 : nullptr, dion::ST, cnt, m, r, flags,
                           0, DION_MAT_FALLBACK, o.max_wait_spins, s,
-                          &nl, &done);
+                          &nl, &done, 2);
         if ((st = tc_check(e, "tc_gram")) != DION_OK) return st;
         ca.pass = 2;
         ca.orth_tol = o.orth_mode == DION_ORTH_CHOLQR2 ? -1.f : o.orth_tol;
@@ -1231,7 +1235,7 @@ dion_status shard_continue(dion_handle h, dion_exchange* x) {
                   "tc_apply");
           if (o.orth_mode != DION_ORTH_CHOLQR)
             DION_TC(c, tc_gram(P1s, b.W, nullptr, nullptr, 0, p.count, p.m, p.r, b.flags, 0,
-                               DION_MAT_FALLBACK, o.max_wait_spins, c.s, &nl_, &done_),
+                               DION_MAT_FALLBACK, o.max_wait_spins, c.s, &nl_, &done_, 2),
                     "tc_gram (second pass)");
           return DION_OK;
         };

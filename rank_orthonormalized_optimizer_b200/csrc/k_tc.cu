@@ -334,8 +334,10 @@ __global__ void __launch_bounds__(NT, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    // split products, smallest terms first: (2,0) (0,2) (1,1) (1,0) (0,1) (0,0)
-    constexpr int NPROD = SPLIT == 3 ? 6 : 1;
+    // split products, smallest terms first: (2,0) (0,2) (1,1) (1,0) (0,1) (0,0); with
+    // two parts loaded (SPLIT = 2) only (1,0) (0,1) (0,0), about 2^-17 relative
+    constexpr int NPROD = SPLIT == 3 ? 6 : (SPLIT == 2 ? 3 : 1);
+    constexpr int P0 = SPLIT == 3 ? 0 : 3;  // first product of the table used
     const int pa[6] = {2, 0, 1, 1, 0, 0};
     const int pb[6] = {0, 2, 1, 0, 1, 0};
     int stage = 0;
@@ -365,8 +367,8 @@ __global__ void __launch_bounds__(NT, 1)
         for (int k = 0; k < BK / 16; ++k) {
 #pragma unroll
           for (int q = 0; q < NPROD; ++q) {
-            const uint32_t ab = a_base + (SPLIT == 3 ? pa[q] : 0) * p.a_bytes;
-            const uint32_t bb = b_base + (SPLIT == 3 ? pb[q] : 0) * p.b_bytes;
+            const uint32_t ab = a_base + (SPLIT > 1 ? pa[P0 + q] : 0) * p.a_bytes;
+            const uint32_t bb = b_base + (SPLIT > 1 ? pb[P0 + q] : 0) * p.b_bytes;
             const uint64_t ad = A_MN ? sw128_desc(ab + k * 2048, 8192, 1024)
                                      : sw128_desc(ab + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? sw128_desc(bb + k * 2048, 8192, 1024)
@@ -638,8 +640,8 @@ cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, float* colsq, 
 }
 
 // fp32 contractions on bf16 tensor cores: operands as three bf16 parts.
-cudaError_t tc_gemm_bq_split(const bf16* Bs, const bf16* Qs, bf16* P0s, int count, int64_t m,
-                             int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
+cudaError_t tc_gemm_bq_split(const bf16* Bs, const bf16* Qs, float* P0, bf16* P0s, int count,
+                             int64_t m, int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
                              cudaStream_t s, int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
@@ -656,8 +658,12 @@ cudaError_t tc_gemm_bq_split(const bf16* Bs, const bf16* Qs, bf16* P0s, int coun
   p.tiles_n = (int)((r + bn - 1) / bn);
   p.num_kb = (int)((n + BK - 1) / BK);
   p.idesc = idesc_bf16(BM, bn, false, false);
-  p.C = nullptr; p.ldc = r; p.c_bs = m * r;
+  // K in chunks summed in fp32 registers: the tensor cores' biased accumulation would
+  // otherwise cost about K / 16 * 6 * 2^-24 relative (1.8e-4 at K = 8192), far above the
+  // split's 2^-24; the chunks' partial sums pass through the fp32 P0
+  p.C = P0; p.ldc = r; p.c_bs = m * r;
   p.Cs = P0s; p.cs_stride = (int64_t)count * m * r;
+  p.kchunk = KCHUNK_SUMSQ;
   p.flags = flags;
   p.max_spins = max_spins;
   cudaError_t e = launch_gemm<false, false, 3>(ma, mb, p, s);
@@ -685,6 +691,7 @@ cudaError_t tc_gemm_btp_split(const bf16* Bs, const bf16* Ps, float* R, float* c
   p.idesc = idesc_bf16(BM, bn, true, true);
   p.C = R; p.ldc = r; p.c_bs = n * r;
   p.colsq = colsq;
+  p.kchunk = KCHUNK_SUMSQ;  // unbiased accumulation over long K, as in B Q
   p.flags = flags;
   p.max_spins = max_spins;
   cudaError_t e = launch_gemm<true, true, 3>(ma, mb, p, s);
@@ -694,7 +701,7 @@ cudaError_t tc_gemm_btp_split(const bf16* Bs, const bf16* Ps, float* R, float* c
 
 cudaError_t tc_gram(const bf16* Xs, float* W, bf16* Ws, float* devmax, int dev_stride, int count,
                     int64_t m, int64_t r, int32_t* flags, int32_t need, int32_t skip,
-                    int64_t max_spins, cudaStream_t s, int* nlaunch, bool* done) {
+                    int64_t max_spins, cudaStream_t s, int* nlaunch, bool* done, int parts) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
@@ -718,7 +725,8 @@ cudaError_t tc_gram(const bf16* Xs, float* W, bf16* Ws, float* devmax, int dev_s
   p.kchunk = KCHUNK_SUMSQ;  // the diagonal sums squares: keep the accumulation unbiased
   p.devmax = devmax; p.dev_stride = dev_stride;
   p.max_spins = max_spins;
-  cudaError_t e = launch_gemm<true, true, 3>(ma, mb, p, s);
+  cudaError_t e = parts == 2 ? launch_gemm<true, true, 2>(ma, mb, p, s)
+                             : launch_gemm<true, true, 3>(ma, mb, p, s);
   if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
   return e;
 }

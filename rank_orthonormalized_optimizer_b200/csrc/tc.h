@@ -42,8 +42,9 @@ cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, bool split
                       float* M, float* X, int count, int64_t m, int64_t n, int64_t r, float mu,
                       float lr_scale, int64_t max_spins, int32_t* flags, int* tile_counter,
                       float* rmmc, cudaStream_t s, int* nlaunch, bool* done);
-// fp32 contractions from three-way bf16 splits: P0s = split(Bs Qs^T), R = Bs^T Ps.
-cudaError_t tc_gemm_bq_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Qs,
+// fp32 contractions from three-way bf16 splits: P0 (fp32) and P0s = split(Bs Qs^T),
+// R = Bs^T Ps; K is accumulated in 512-wide chunks added in fp32 registers.
+cudaError_t tc_gemm_bq_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Qs, float* P0,
                              __nv_bfloat16* P0s, int count, int64_t m, int64_t n, int64_t r,
                              int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
                              bool* done);
@@ -57,10 +58,13 @@ cudaError_t tc_gemm_btp_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Ps, 
 // Only the 128 x 128 tiles on and below the diagonal are written (r > 64), and, when Ws
 // is not null, their split ([3][count][r][r]) as well.  When devmax is not null,
 // max_{j <= i} |W_ij - I_ij| of matrix b is max-ed into devmax[b * dev_stride] (which must
-// hold a non-negative value before the call; NaN wins).
+// hold a non-negative value before the call; NaN wins).  parts = 2 reads only the two
+// leading parts and sums three products, (1,0) (0,1) (0,0): about 2^-17 relative, enough
+// for the Gram of an already orthonormalised first pass (the second Cholesky-QR pass).
 cudaError_t tc_gram(const __nv_bfloat16* Xs, float* W, __nv_bfloat16* Ws, float* devmax,
                     int dev_stride, int count, int64_t m, int64_t r, int32_t* flags, int32_t need,
-                    int32_t skip, int64_t max_spins, cudaStream_t s, int* nlaunch, bool* done);
+                    int32_t skip, int64_t max_spins, cudaStream_t s, int* nlaunch, bool* done,
+                    int parts = 3);
 // Y[b] (m x r, fp32) = X[b] L[b]^T from the splits Xs ([3][count][m][r]) and Ls
 // ([3][count][r][r], L lower triangular), optionally writing Y's split to Ys and its
 // bf16 rounding to Yb ([count][m][r]).  Column

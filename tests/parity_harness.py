@@ -24,6 +24,7 @@ class Report:
     rel_x: float = 0.0
     rel_m: float = 0.0
     rel_q: float = 0.0
+    rel_q_w: float = 0.0           # Q's error with each column weighted by ||R_j|| (see below)
     rel_dx: float = 0.0
     dx_floor: float = 0.0          # fp32 rounding of the stored X, relative to ||dX||
     orth_gpu: float = 0.0          # max |P^T P - I| over every matrix of the GPU run
@@ -31,7 +32,8 @@ class Report:
     per_slot: list = field(default_factory=list)
 
     def __str__(self):
-        return (f"rel_F X {self.rel_x:.3e}  M {self.rel_m:.3e}  Q {self.rel_q:.3e}  "
+        return (f"rel_F X {self.rel_x:.3e}  M {self.rel_m:.3e}  Q {self.rel_q:.3e} "
+                f"(R-weighted {self.rel_q_w:.3e})  "
                 f"dX {self.rel_dx:.3e} (fp32 floor {self.dx_floor:.1e})  |P^T P - I| {self.orth_gpu:.3e}  status {self.status_or}")
 
 
@@ -92,7 +94,20 @@ def oracle_slot(wl: W.Workload, bi: int, slot: int, steps: int, gen: str):
              for t in range(steps))
     X, M, Q, P, R = oracle.run_steps(X0, M, Q, grads, wl.mu, wl.lr,
                                      reset_momentum=(wl.grad == "fixed_sqrt_spectrum"))
-    return X0, X, M, Q, P
+    return X0, X, M, Q, P, R
+
+
+def rel_q_weighted(q_gpu, Q_ref, R_ref) -> float:
+    """||(Q_gpu - Q_ref) D||_F / ||Q_ref D||_F with D = diag(||R_ref[:, j]||).
+
+    Q = colnorm(R): column j is R_j / ||R_j||.  The operands' rounding perturbs R_j by
+    about eps ||B|| whatever ||R_j|| is, so the direction of a column whose norm is small
+    beside ||B|| (full rank: the last columns) is fixed only to eps ||B|| / ||R_j||.
+    Weighting each column's error by the norm of the R column it normalises measures Q
+    at the accuracy the arithmetic gives it (it is R's relative error, column directions
+    only)."""
+    d = np.sqrt(np.sum(R_ref * R_ref, axis=0))
+    return float(np.linalg.norm((q_gpu - Q_ref) * d) / max(np.linalg.norm(Q_ref * d), 1e-300))
 
 
 def compare(run: GpuRun, steps: int, slots_per_bucket=None) -> Report:
@@ -105,7 +120,7 @@ def compare(run: GpuRun, steps: int, slots_per_bucket=None) -> Report:
         else:
             slots = sorted({s % b.count for s in slots_per_bucket})
         for s in slots:
-            X0, X, M, Q, P = oracle_slot(run.wl, bi, s, steps, run.gen)
+            X0, X, M, Q, P, R = oracle_slot(run.wl, bi, s, steps, run.gen)
             gx = run.X[bi][s].double().cpu().numpy()
             gm = run.M[bi][s].double().cpu().numpy()
             gq = run.Q[bi][s].double().cpu().numpy()
@@ -114,12 +129,13 @@ def compare(run: GpuRun, steps: int, slots_per_bucket=None) -> Report:
             floor = 2.0 ** -24 * np.linalg.norm(X0) * math.sqrt(steps) / max(
                 np.linalg.norm(X - X0), 1e-300)
             one = dict(bucket=bi, slot=s, rel_x=oracle.rel_fro(gx, X), rel_m=oracle.rel_fro(gm, M),
-                       rel_q=oracle.rel_fro(gq, Q), rel_dx=oracle.rel_fro(gx - X0, X - X0),
-                       dx_floor=floor)
+                       rel_q=oracle.rel_fro(gq, Q), rel_q_w=rel_q_weighted(gq, Q, R),
+                       rel_dx=oracle.rel_fro(gx - X0, X - X0), dx_floor=floor)
             rep.per_slot.append(one)
             rep.rel_x = max(rep.rel_x, one["rel_x"])
             rep.rel_m = max(rep.rel_m, one["rel_m"])
             rep.rel_q = max(rep.rel_q, one["rel_q"])
+            rep.rel_q_w = max(rep.rel_q_w, one["rel_q_w"])
             rep.rel_dx = max(rep.rel_dx, one["rel_dx"])
             rep.dx_floor = max(rep.dx_floor, one["dx_floor"])
     rep.orth_gpu = run.orth_error()

@@ -2,7 +2,11 @@
 
 Tolerances (relative Frobenius error per matrix, max over the checked matrices):
   fp32 contractions   X, M and Q <= 1e-4 after the step count of the workload
-  bf16-input GEMMs    X, M and Q <= 2e-2
+  bf16-input GEMMs    X and M <= 2e-2; Q <= 2e-2 with its columns weighted by the norms
+                      of the R columns they normalise (a bf16 operand perturbs R_j by
+                      about 2^-8 ||B||, so the direction of a column of R that is small
+                      beside ||B|| -- the last ones at full rank -- is fixed only to
+                      2^-8 ||B|| / ||R_j||; weighted, Q's error is R's)
   every matrix        max |P^T P - I| <= 1e-4 on the GPU's own P
 The weight change dX = X_T - X_0 is checked too, since X_0 dominates X.  Its bound
 has two parts: the operand rounding (bf16 operands carry a relative error up to 2^-8
@@ -31,7 +35,9 @@ def _check(rep, precision, dx=True):
     print(rep)
     assert rep.rel_x <= TOL[precision], rep
     assert rep.rel_m <= TOL[precision], rep
-    assert rep.rel_q <= TOL[precision], rep
+    assert rep.rel_q_w <= TOL[precision], rep
+    if precision == "fp32":
+        assert rep.rel_q <= TOL[precision], rep
     assert rep.orth_gpu <= ORTH_TOL, rep
     if dx:
         assert rep.rel_dx <= TOL_DX[precision] + 3 * rep.dx_floor, rep
@@ -259,7 +265,7 @@ def test_nonfinite_gradient_is_reported_and_contained():
     st = run.status.cpu().numpy()
     assert st[1] & 4 and not (st[0] & 4) and not (st[2] & 4), st
     for s in (0, 2):
-        X0, X, M, Q, P = oracle_slot(wl, 0, s, 1, "cpu")
+        X0, X, M, Q, P, R = oracle_slot(wl, 0, s, 1, "cpu")
         assert oracle.rel_fro(run.X[0][s].double().cpu().numpy(), X) <= TOL["fp32"]
 
 

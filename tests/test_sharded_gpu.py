@@ -13,7 +13,7 @@ import torch
 
 import oracle
 import workloads as W
-from parity_harness import oracle_slot
+from parity_harness import oracle_slot, rel_q_weighted
 from rank_orthonormalized_optimizer_b200 import VIEW_P, DionB200RowSharded
 
 pytestmark = pytest.mark.gpu
@@ -104,9 +104,13 @@ def test_row_shards_match_the_oracle(precision, world):
         X, M, Q, P = em.whole(i)
         assert _orth_err(P) <= ORTH_TOL
         for s in range(b.count):
-            X0, Xr, Mr, Qr, _ = oracle_slot(wl, i, s, wl.steps, "cpu")
-            rel = [oracle.rel_fro(a[s].double().cpu().numpy(), ref) for a, ref in
-                   ((X, Xr), (M, Mr), (Q, Qr))]
+            X0, Xr, Mr, Qr, _, Rr = oracle_slot(wl, i, s, wl.steps, "cpu")
+            q = Q[s].double().cpu().numpy()
+            rel = [oracle.rel_fro(X[s].double().cpu().numpy(), Xr),
+                   oracle.rel_fro(M[s].double().cpu().numpy(), Mr),
+                   # Q as in the whole-matrix parity tests: plain in fp32, its columns
+                   # weighted by the norms of R's columns with bf16 operands
+                   oracle.rel_fro(q, Qr) if precision == "fp32" else rel_q_weighted(q, Qr, Rr)]
             print(precision, world, i, s, ["%.2e" % v for v in rel])
             assert max(rel) <= TOL[precision], (i, s, rel)
 
@@ -153,7 +157,7 @@ def test_householder_mode_gathers_every_bucket():
     for i, b in enumerate(wl.buckets):
         X, M, Q, P = em.whole(i)
         for s in range(b.count):
-            _, Xr, Mr, Qr, _ = oracle_slot(wl, i, s, wl.steps, "cpu")
+            _, Xr, Mr, Qr, _, _ = oracle_slot(wl, i, s, wl.steps, "cpu")
             for a, ref in ((X, Xr), (M, Mr), (Q, Qr)):
                 assert oracle.rel_fro(a[s].double().cpu().numpy(), ref) <= TOL["fp32"]
 
