@@ -411,19 +411,37 @@ __global__ void __launch_bounds__(NT, 1)
       k_range(p, tile_mi(p, rem) * BM, (int)n0, kb0, kb1);
       float rsq = 0.f;  // transposed store: this lane's row sum of squares over the tile
       const int nch = n_chunks(p, kb0, kb1);
+      // split operands: the chunks are added, in fp32 registers, into a running sum kept
+      // in a third TMEM region (columns [2 block_n, 3 block_n), this thread's lane = its
+      // row), and C is written once from the last chunk; otherwise each later chunk adds
+      // into C in memory
+      const bool tsum = SPLIT > 1 && nch > 1;
+      const uint32_t sbase = tmem + ((uint32_t)(ew * 32) << 16) + 2 * p.acc_stride;
       for (int ch = 0; ch < nch; ++ch) {
         const int acc = lt & 1;
         const uint32_t acc_phase = (lt >> 1) & 1;
         if (!wait_bounded(tfull + acc, acc_phase, p.max_spins, abort)) { ok = false; break; }
         tc_fence_after();
-        const int epi = ch == 0 ? p.epi : 2;
+        const int epi = (ch == 0 || tsum) ? p.epi : 2;
         const float alpha = p.epi == 0 ? 1.f : p.alpha;
         const bool last = ch == nch - 1;
         const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * p.acc_stride;
         for (int c = 0; c < p.block_n; c += 16) {
           float v[16];
           tmem_ld16(tbase + c, v);
-          tmem_wait_ld();
+          if (tsum && ch > 0) {
+            float run[16];
+            tmem_ld16(sbase + c, run);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[q] += run[q];
+          } else {
+            tmem_wait_ld();
+          }
+          if (tsum && !last) {
+            tmem_st16(sbase + c, v);
+            continue;
+          }
           if (n0 + c >= p.N) continue;  // uniform across the warp
           if (p.c_trans) {
             // C[j][i]: for each column j the warp's 32 rows are 32 consecutive floats
@@ -504,6 +522,7 @@ __global__ void __launch_bounds__(NT, 1)
           }
           __syncwarp();
         }
+        if (tsum && !last) tmem_wait_st();  // the running sum is read back next chunk
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(tempty + acc);
@@ -549,7 +568,10 @@ static cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Gem
   if (stages < 1) return cudaErrorInvalidValue;
   p.stages = stages;
   p.acc_stride = (uint32_t)p.block_n;
-  p.tmem_cols = pow2_cols(2 * p.block_n);
+  // two accumulators, and with split operands over K chunks a third region for the
+  // chunks' running sum
+  p.tmem_cols = pow2_cols((SPLIT > 1 && p.kchunk > 0 ? 3 : 2) * p.block_n);
+  if (p.tmem_cols > 512) return cudaErrorInvalidValue;
   const size_t smem = 1024 + stages * stage_bytes + (2 * stages + 5) * 8 + 16 +
                       4 * 32 * EPI_LD * sizeof(float);
   auto kern = k_tc_gemm<A_MN, B_MN, SPLIT>;

@@ -31,12 +31,15 @@ TOL_DX = {"fp32": 1e-3, "bf16": 6e-2}
 ORTH_TOL = 1e-4
 
 
-def _check(rep, precision, dx=True):
+def _check(rep, precision, dx=True, full_rank=False):
     print(rep)
     assert rep.rel_x <= TOL[precision], rep
     assert rep.rel_m <= TOL[precision], rep
     assert rep.rel_q_w <= TOL[precision], rep
-    if precision == "fp32":
+    if precision == "fp32" and not full_rank:
+        # below full rank R's columns are the leading directions, none small beside
+        # ||B||: Q itself must meet the bound (at full rank the last columns of R are
+        # as small as B's smallest singular values, and only the weighted error is due)
         assert rep.rel_q <= TOL[precision], rep
     assert rep.orth_gpu <= ORTH_TOL, rep
     if dx:
@@ -124,7 +127,7 @@ def test_square_8x8192_rank_sweep(r):
     wl = W.WORKLOADS[f"square_8x8192_r{r}"]
     run = GpuRun(wl)
     rep = compare(run, wl.steps, slots_per_bucket=(0,))
-    _check(rep, "fp32")
+    _check(rep, "fp32", full_rank=(r == 8192))
 
 
 # ------------------------------------------------------------------ edge cases

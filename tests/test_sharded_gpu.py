@@ -167,7 +167,7 @@ def test_one_rank_is_the_whole_step():
     dion_step_batched, except that the column norms' partial sums come from R itself
     rather than from B^T P's epilogue.  After one step M (which does not depend on the
     new Q) is bit for bit the same; X and Q differ by the rounding of that sum's order,
-    and so does the second step."""
+    which the second step carries on: they must agree within the parity tolerance."""
     from parity_harness import GpuRun
     wl = W.custom("rowshard_one", [(3, 256, 128, 32), (2, 600, 560, 272)], precision="fp32",
                   steps=2)
@@ -182,4 +182,4 @@ def test_one_rank_is_the_whole_step():
             if t == 0:
                 assert torch.equal(M, ref.M[i])
             for a, b in ((X - ref.X0[i], ref.X[i] - ref.X0[i]), (M, ref.M[i]), (Q, ref.Q[i])):
-                assert ((a - b).norm() / b.norm()).item() <= 1e-5
+                assert ((a - b).norm() / b.norm()).item() <= TOL["fp32"]
