@@ -333,10 +333,6 @@ dion_status fb_launch(dion_handle h, int bi, const Plan& p, const void* ws, cons
   return DION_OK;
 }
 
-// Where the buckets' orthonormalisation chains start: right after each bucket's B Q
-// (beside the later buckets' B Q), or all together once every B Q is done.
-constexpr bool kOrthAfterAllBQ = false;
-
 // Phases of one step; each runs over every bucket before the next starts.
 enum Phase { PH_INIT, PH_PREPQ, PH_FORMB, PH_BQ, PH_ORTH, PH_BTP, PH_COLNORM, PH_UPDATE,
              PH_STATUS, PH_COUNT };
@@ -971,29 +967,20 @@ static dion_status dion_step_batched_impl(dion_handle h, const dion_bucket_ptrs*
   for (int phase : {PH_INIT, PH_PREPQ})
     for (int32_t b = 0; b < nbuckets; ++b)
       if ((st = run(phase, b, main)) != DION_OK) return finish(st);
-  auto fork_orth = [&](int32_t b) -> dion_status {
-    cudaStreamWaitEvent(h->side[b], h->fork_ev, 0);
-    dion_status r = run(PH_ORTH, b, h->side[b]);
-    end_cls(c);
-    cudaEventRecord(h->side_done[b], h->side[b]);
-    forked = b + 1;
-    return r;
-  };
   for (int32_t b = 0; b < nbuckets; ++b) {
     for (int phase : {PH_FORMB, PH_BQ})
       if ((st = run(phase, b, main)) != DION_OK) return finish(st);
-    if (fork && !kOrthAfterAllBQ) {
+    if (fork) {
       cudaEventRecord(h->fork_ev, main);
-      st = fork_orth(b);
-    } else if (!fork) {
+      cudaStreamWaitEvent(h->side[b], h->fork_ev, 0);
+      st = run(PH_ORTH, b, h->side[b]);
+      end_cls(c);
+      cudaEventRecord(h->side_done[b], h->side[b]);
+      forked = b + 1;
+    } else {
       st = run(PH_ORTH, b, main);
     }
     if (st != DION_OK) return finish(st);
-  }
-  if (fork && kOrthAfterAllBQ) {
-    cudaEventRecord(h->fork_ev, main);
-    for (int32_t b = 0; b < nbuckets; ++b)
-      if ((st = fork_orth(b)) != DION_OK) return finish(st);
   }
   for (int32_t b = 0; b < nbuckets; ++b) {
     if (fork) {

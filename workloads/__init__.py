@@ -96,6 +96,21 @@ WORKLOADS = {
             note="16 attention-sized 4096x4096 matrices, rank 256: a 3 GB case for profiling "
                  "(inputs larger than L2)",
             sample_slots=(0, 15)),
+        # the two MLP shapes of the 7B-like workload, 4 matrices each (2.2 GB of fp32
+        # X, M, G, larger than L2): cases small enough for a profiler to capture one
+        # launch of each kernel at the headline's shapes
+        Workload(
+            name="mlp_up_4x4096x11008_r256",
+            buckets=(Bucket(4, 4096, 11008, 256),),
+            precision="bf16", mu=0.95, lr=0.01, steps=3, grad="gaussian_1e-3",
+            note="4 of the 7B-like W_gate/W_up shape (4096x11008), rank 256: for profiling",
+            sample_slots=(0, 3)),
+        Workload(
+            name="mlp_down_4x11008x4096_r256",
+            buckets=(Bucket(4, 11008, 4096, 256),),
+            precision="bf16", mu=0.95, lr=0.01, steps=3, grad="gaussian_1e-3",
+            note="4 of the 7B-like W_down shape (11008x4096), rank 256: for profiling",
+            sample_slots=(0, 3)),
     ] + [_sweep(r) for r in (64, 128, 256, 512, 1024, 2048, 4096, 8192)]
 }
 
