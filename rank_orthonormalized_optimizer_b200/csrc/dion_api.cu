@@ -62,9 +62,21 @@ struct Plan {
   // row-sharded plans: this rank holds rows [row0, row0 + m) of m_full-row matrices
   // (m_full == m, row0 == 0 otherwise)
   int64_t m_full, row0;
+  // the stack the bucket's orthonormalisation runs in: every bucket with the same m and
+  // r shares one (its matrices at positions [stack_off, stack_off + count) of the
+  // stack's `zplane` matrices; split parts of m x r arrays zplane * m * r elements apart)
+  int group, stack_off, zplane;
   size_t off_Bg, off_Qg, off_P0, off_P, off_P2, off_Pg, off_W, off_Linv, off_dinv, off_R, off_Rg,
       off_Qng, off_part, off_flags, off_stats, off_P0s, off_Ps, off_Linvs, off_sched, off_Ws, off_Ts,
       off_gather, off_rmmc;
+};
+
+// A stack of the orthonormalisation: the buckets whose P has the same shape (m x r),
+// whatever their n, stacked into one [count, m, r] batch.  `orth` is a plan of the whole
+// stack (count = the members' counts summed) for the orthonormalisation's kernels.
+struct OrthGroup {
+  std::vector<int32_t> members;  // bucket indices, in bucket order
+  Plan orth;
 };
 
 struct EventPair {
@@ -79,6 +91,7 @@ struct dion_ctx {
   uint64_t magic;
   dion_options opt;
   std::vector<Plan> plans;
+  std::vector<OrthGroup> groups;
   size_t ws_bytes;
   int64_t total_mats;
   int32_t last_launches;
@@ -161,6 +174,7 @@ struct StepCtx {
   int open_at;
   std::vector<int> p0s_ready;  // per bucket: P0's split was written by B Q
   bool sharded = false;        // R is a partial sum: column-norm partials from R itself
+  std::vector<int> g_ready;    // per stack: P0's split was written by every member's B Q
 };
 
 void begin_cls(StepCtx& c, int cls) {
@@ -368,7 +382,9 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
   __nv_bfloat16* Linvs = reinterpret_cast<__nv_bfloat16*>(ws + p.off_Linvs);
   __nv_bfloat16* Ws = p.off_Ws ? reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ws) : nullptr;
   __nv_bfloat16* Ts = p.off_Ts ? reinterpret_cast<__nv_bfloat16*>(ws + p.off_Ts) : nullptr;
-  int& p0s_ready = c.p0s_ready[bi];
+  // PH_ORTH runs once per stack (bi is then the stack's index and p its plan)
+  int& p0s_ready = phase == PH_ORTH ? c.g_ready[bi] : c.p0s_ready[bi];
+  const int64_t plane_mr = (int64_t)p.zplane * p.m * p.r;  // between split parts of m x r
   const int64_t m = p.m, n = p.n, r = p.r;
   const int cnt = p.count;
   cudaStream_t s = c.s;
@@ -378,6 +394,12 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     DION_LAUNCH(c, 1, dion::launch_init_flags(flags, stats, sched, rmmc, cnt,
                                               o.orth_mode == DION_ORTH_HOUSEHOLDER ? DION_MAT_FALLBACK : 0,
                                               s));
+    // a stack of several buckets has counters of its own (the fallback loop's rounds)
+    const OrthGroup& g = c.h->groups[p.group];
+    if (g.members.size() > 1 && g.members[0] == bi)
+      DION_LAUNCH(c, 1, dion::launch_init_flags(nullptr, nullptr,
+                                                reinterpret_cast<int*>(ws + g.orth.off_sched),
+                                                nullptr, 0, 0, s));
     return DION_OK;
   }
 
@@ -411,8 +433,8 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
   if (fused_bq) {
     int nl = 0;
     bool done = false;
-    cudaError_t e = dion::tc_formb_bq(bp.M, bp.G, Qg, Bg, P0s, cnt, m, n, r, o.max_wait_spins,
-                                      flags, sched + 1, s, &nl, &done);
+    cudaError_t e = dion::tc_formb_bq(bp.M, bp.G, Qg, Bg, P0s, plane_mr, cnt, m, n, r,
+                                      o.max_wait_spins, flags, sched + 1, s, &nl, &done);
     c.launches += nl;
     if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_formb_bq: %s", cudaGetErrorString(e));
     if (!done) return fail(DION_ERR_CUDA, "tc_formb_bq: %s", dion::tc_map_error());
@@ -421,8 +443,8 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     int nl = 0;
     bool done = false;
     cudaError_t e = dion::tc_gemm_bq_split((const __nv_bfloat16*)Bg, (const __nv_bfloat16*)Qg, P0,
-                                           P0s, cnt, m, n, r, o.max_wait_spins, flags, s, &nl,
-                                           &done);
+                                           P0s, plane_mr, cnt, m, n, r, o.max_wait_spins, flags,
+                                           s, &nl, &done);
     c.launches += nl;
     if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_gemm_bq_split: %s", cudaGetErrorString(e));
     if (!done) return fail(DION_ERR_CUDA, "tc_gemm_bq_split: %s", dion::tc_map_error());
@@ -432,8 +454,8 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     if (tensor && bf) {
       int nl = 0;
       // only the split of P0 is written: the orthonormalisation reads nothing else
-      cudaError_t e = dion::tc_gemm_bq(Bg, Qg, nullptr, P0s, cnt, m, n, r, o.max_wait_spins, flags,
-                                       s, &nl, &done);
+      cudaError_t e = dion::tc_gemm_bq(Bg, Qg, nullptr, P0s, plane_mr, cnt, m, n, r,
+                                       o.max_wait_spins, flags, s, &nl, &done);
       c.launches += nl;
       if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_gemm_bq: %s", cudaGetErrorString(e));
       if (!done) return fail(DION_ERR_CUDA, "tc_gemm_bq: %s", dion::tc_map_error());
@@ -583,9 +605,9 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     bool done = false;
     if (split) {
       int nl = 0;
-      cudaError_t e = dion::tc_gemm_btp_split((const __nv_bfloat16*)Bg, (const __nv_bfloat16*)Pg, R,
-                                              part, cnt, m, n, r, o.max_wait_spins, flags, s, &nl,
-                                              &done);
+      cudaError_t e = dion::tc_gemm_btp_split((const __nv_bfloat16*)Bg, (const __nv_bfloat16*)Pg,
+                                              p.zplane, R, part, cnt, m, n, r, o.max_wait_spins,
+                                              flags, s, &nl, &done);
       c.launches += nl;
       if (e != cudaSuccess)
         return fail(DION_ERR_CUDA, "tc_gemm_btp_split: %s", cudaGetErrorString(e));
@@ -629,8 +651,9 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
     const float lrs = lr * p.scale;
     if (tensor) {
       int nl = 0;
-      cudaError_t e = dion::tc_update(Pg, Rg, Qng, split, bp.G, bp.M, bp.X, cnt, m, n, r, o.mu,
-                                      lrs, o.max_wait_spins, flags, sched, rmmc, s, &nl, &done);
+      cudaError_t e = dion::tc_update(Pg, p.zplane, Rg, Qng, split, bp.G, bp.M, bp.X, cnt, m, n,
+                                      r, o.mu, lrs, o.max_wait_spins, flags, sched, rmmc, s, &nl,
+                                      &done);
       c.launches += nl;
       if (e != cudaSuccess) return fail(DION_ERR_CUDA, "tc_update: %s", cudaGetErrorString(e));
       if (!done) return fail(DION_ERR_CUDA, "tc_update: %s", dion::tc_map_error());
@@ -871,44 +894,105 @@ static dion_status dion_init_impl(const dion_bucket_desc* buckets, const dion_sh
     }
     off = align_up(off_rblk + rblk * 4, 1024);
   }
+  // Stacks of the orthonormalisation: the buckets whose P has the same shape (m, r)
+  // share one [count, m, r] stack of every per-matrix array the orthonormalisation uses
+  // (P0, P and their splits, the Gram and the factor, flags, statistics), so that it runs
+  // once over all of them, as DASH stacks equal-sized blocks of different layers.  Each
+  // bucket's arrays are slices of its stack.  A row-sharded plan keeps one stack per
+  // bucket (its exchanges are laid out per bucket).
+  std::vector<OrthGroup> groups;
+  for (int32_t b = 0; b < nbuckets; ++b) {
+    Plan& p = plans[b];
+    int gi = -1;
+    if (!sharded)
+      for (size_t g = 0; g < groups.size(); ++g) {
+        const Plan& q = plans[groups[g].members[0]];
+        if (q.m == p.m && q.r == p.r) gi = (int)g;
+      }
+    if (gi < 0) {
+      gi = (int)groups.size();
+      groups.push_back(OrthGroup{});
+    }
+    p.group = gi;
+    groups[gi].members.push_back(b);
+  }
+  for (OrthGroup& g : groups) {
+    Plan go = plans[g.members[0]];
+    go.count = 0;
+    for (int32_t b : g.members) go.count += plans[b].count;
+    const size_t c = (size_t)go.count;
+    const int64_t m = go.m, r = go.r;
+    go.zplane = go.count;
+    go.stack_off = 0;
+    go.off_P0 = take(c * m * r * 4);
+    go.off_P = take(c * m * r * 4);
+    go.off_P2 = take(c * m * r * 4);
+    go.off_Pg = (bf || split) && !(bf && o.kernel_path == DION_PATH_TENSOR) ? take(c * m * r * ge)
+                                                                             : 0;
+    if (!sharded) go.off_W = take(c * r * r * 4);
+    go.off_Linv = take(c * r * r * 4);
+    go.off_dinv = take(dion::chol_dinv_floats(go.count, r) * 4);
+    go.off_flags = take(c * 4);
+    go.off_stats = take(c * 4 * 4);
+    // three-way bf16 splits for the tensor-core orthonormalisation
+    go.off_P0s = take(c * m * r * 6);
+    go.off_Ps = take(c * m * r * 6);
+    go.off_Linvs = take(c * r * r * 6);
+    go.off_sched = take(64);  // the fallback loop's counters
+    go.off_Ws = go.off_Ts = 0;
+    if (o.kernel_path == DION_PATH_TENSOR && r > 256) {
+      // splits of the Gram / its updates and of L21 for the recursive factorisation
+      go.off_Ws = take(c * r * r * 6);
+      go.off_Ts = take(c * r * r * 6);
+    }
+    size_t at = 0;  // matrices of the stack before this bucket
+    for (int32_t b : g.members) {
+      Plan& p = plans[b];
+      p.stack_off = (int)at;
+      p.zplane = go.count;
+      p.off_P0 = go.off_P0 + at * m * r * 4;
+      p.off_P = go.off_P + at * m * r * 4;
+      p.off_P2 = go.off_P2 + at * m * r * 4;
+      // (the bf16 copy, or the leading part of the split: 2 bytes an element either way)
+      p.off_Pg = go.off_Pg ? go.off_Pg + at * m * r * 2 : 0;
+      if (!sharded) p.off_W = go.off_W + at * r * r * 4;
+      p.off_Linv = go.off_Linv + at * r * r * 4;
+      p.off_dinv = go.off_dinv + dion::chol_dinv_floats((int)at, r) * 4;
+      p.off_flags = go.off_flags + at * 4;
+      p.off_stats = go.off_stats + at * 4 * 4;
+      p.off_P0s = go.off_P0s + at * m * r * 2;
+      p.off_Ps = go.off_Ps + at * m * r * 2;
+      p.off_Linvs = go.off_Linvs + at * r * r * 2;
+      p.off_Ws = go.off_Ws ? go.off_Ws + at * r * r * 2 : 0;
+      p.off_Ts = go.off_Ts ? go.off_Ts + at * r * r * 2 : 0;
+      at += (size_t)p.count;
+    }
+    if (sharded) go.off_W = plans[g.members[0]].off_W;
+    g.orth = go;
+  }
   for (Plan& p : plans) {
     const size_t c = (size_t)p.count;
     p.off_Bg = take(c * p.m * p.n * ge);
     p.off_Qg = take(c * p.n * p.r * ge);
-    p.off_P0 = take(c * p.m * p.r * 4);
-    p.off_P = take(c * p.m * p.r * 4);
-    p.off_P2 = take(c * p.m * p.r * 4);
-    p.off_Pg = (bf || split) && !(bf && o.kernel_path == DION_PATH_TENSOR)
-                   ? take(c * p.m * p.r * ge) : 0;
-    if (!sharded) p.off_W = take(c * p.r * p.r * 4);
-    p.off_Linv = take(c * p.r * p.r * 4);
-    p.off_dinv = take(dion::chol_dinv_floats(p.count, p.r) * 4);
     if (!sharded) p.off_R = take(c * p.n * p.r * 4);
     p.off_Rg = (bf || split) ? take(c * p.n * p.r * ge) : 0;
     p.off_Qng = (bf || split) ? take(c * p.n * p.r * ge) : 0;
     p.off_part = take(c * p.nsplit * p.r * 4);
-    p.off_flags = take(c * 4);
-    p.off_stats = take(c * 4 * 4);
     p.off_rmmc = take(c * 3 * 4);  // max |M' - M|, max |M|, their ratio: [3][count]
-    // three-way bf16 splits for the tensor-core orthonormalisation
-    p.off_P0s = take(c * p.m * p.r * 6);
-    p.off_Ps = take(c * p.m * p.r * 6);
-    p.off_Linvs = take(c * p.r * p.r * 6);
     p.off_sched = take(64);  // tile counters of the dynamically scheduled kernels
-    if (o.kernel_path == DION_PATH_TENSOR && p.r > 256) {
-      // splits of the Gram / its updates and of L21 for the recursive factorisation
-      p.off_Ws = take(c * p.r * p.r * 6);
-      p.off_Ts = take(c * p.r * p.r * 6);
-    }
     // row-sharded fallback: the gathered P0 (its QR written in place) and the two
     // column-major work arrays of Householder QR, each [count, m_full, r] fp32
     if (sharded) p.off_gather = take(3 * c * p.m_full * p.r * 4);
   }
+  // a stack of one bucket is that bucket: its counters are the bucket's
+  for (OrthGroup& g : groups)
+    if (g.members.size() == 1) g.orth.off_sched = plans[g.members[0]].off_sched;
   dion_ctx* h = new (std::nothrow) dion_ctx();
   if (!h) return fail(DION_ERR_INVALID_ARG, "out of host memory");
   h->magic = kMagic;
   h->opt = o;
   h->plans = std::move(plans);
+  h->groups = std::move(groups);
   h->ws_bytes = off;
   h->total_mats = mats;
   h->last_launches = 0;
@@ -946,13 +1030,15 @@ static dion_status dion_step_batched_impl(dion_handle h, const dion_bucket_ptrs*
   cudaStream_t main = reinterpret_cast<cudaStream_t>(stream);
   StepCtx c{h, main, 0, -1, nullptr, 0, std::vector<int>(nbuckets, 0)};
   char* ws = static_cast<char*>(d_workspace);
-  // Each bucket's orthonormalisation is a chain of short, latency-bound kernels that
-  // needs only that bucket's P0.  It is forked onto the bucket's own stream as soon
-  // as B Q has written P0, so it runs beside the B Q of the later buckets and the
-  // B^T P, column norms and update of the earlier ones; the main stream joins it
-  // just before that bucket's B^T P.
-  const bool fork = nbuckets > 1 && ensure_side_streams(h, (size_t)nbuckets);
-  int32_t forked = 0, joined = 0;  // side streams [joined, forked) still to be joined
+  // Each stack's orthonormalisation is a chain of short, latency-bound kernels that
+  // needs only its buckets' P0.  It is forked onto the stack's own stream as soon as the
+  // last of them has run B Q, so it runs beside the B Q of the later buckets and the
+  // B^T P, column norms and update of the earlier ones; the main stream joins it just
+  // before the B^T P of its first bucket.
+  const int32_t ng = (int32_t)h->groups.size();
+  const bool fork = (ng > 1 || nbuckets > 1) && ensure_side_streams(h, (size_t)ng);
+  c.g_ready.assign((size_t)ng, 0);
+  std::vector<char> forked((size_t)ng, 0), joined((size_t)ng, 0);
   auto run = [&](int phase, int32_t b, cudaStream_t s) -> dion_status {
     c.s = s;
     return run_bucket(c, b, phase, h->plans[b], ptrs[b], lr, ws, d_status);
@@ -960,7 +1046,8 @@ static dion_status dion_step_batched_impl(dion_handle h, const dion_bucket_ptrs*
   auto finish = [&](dion_status result) -> dion_status {
     end_cls(c);
     // a failed step still leaves `main` ordered after every forked chain
-    for (; joined < forked; ++joined) cudaStreamWaitEvent(main, h->side_done[joined], 0);
+    for (int32_t g = 0; g < ng; ++g)
+      if (forked[g] && !joined[g]) cudaStreamWaitEvent(main, h->side_done[g], 0);
     h->last_launches = c.launches;
     return result;
   };
@@ -970,22 +1057,28 @@ static dion_status dion_step_batched_impl(dion_handle h, const dion_bucket_ptrs*
   for (int32_t b = 0; b < nbuckets; ++b) {
     for (int phase : {PH_FORMB, PH_BQ})
       if ((st = run(phase, b, main)) != DION_OK) return finish(st);
+    const int32_t g = h->plans[b].group;
+    const OrthGroup& og = h->groups[g];
+    c.g_ready[g] = c.p0s_ready[b];
+    if (og.members.back() != b) continue;  // the stack is complete after its last bucket
+    c.s = fork ? h->side[g] : main;
     if (fork) {
       cudaEventRecord(h->fork_ev, main);
-      cudaStreamWaitEvent(h->side[b], h->fork_ev, 0);
-      st = run(PH_ORTH, b, h->side[b]);
+      cudaStreamWaitEvent(h->side[g], h->fork_ev, 0);
+    }
+    st = run_bucket(c, g, PH_ORTH, og.orth, ptrs[og.members[0]], lr, ws, d_status);
+    if (fork) {
       end_cls(c);
-      cudaEventRecord(h->side_done[b], h->side[b]);
-      forked = b + 1;
-    } else {
-      st = run(PH_ORTH, b, main);
+      cudaEventRecord(h->side_done[g], h->side[g]);
+      forked[g] = 1;
     }
     if (st != DION_OK) return finish(st);
   }
   for (int32_t b = 0; b < nbuckets; ++b) {
-    if (fork) {
-      cudaStreamWaitEvent(main, h->side_done[b], 0);
-      joined = b + 1;
+    const int32_t g = h->plans[b].group;
+    if (fork && !joined[g]) {
+      cudaStreamWaitEvent(main, h->side_done[g], 0);
+      joined[g] = 1;
     }
     for (int phase : {PH_BTP, PH_COLNORM, PH_UPDATE, PH_STATUS})
       if ((st = run(phase, b, main)) != DION_OK) return finish(st);
@@ -993,21 +1086,36 @@ static dion_status dion_step_batched_impl(dion_handle h, const dion_bucket_ptrs*
   return finish(DION_OK);
 }
 
-// The step with the gradients uploaded bucket by bucket on a copy stream: each bucket's
-// whole step (B Q to update) starts as soon as its own gradients have arrived, so it runs
-// while the later buckets' gradients cross the host link.  Buckets are uploaded largest
-// first, so what is left after the last copy is the step of the smallest bucket.
+// The step with the gradients uploaded bucket by bucket on a copy stream: each
+// orthonormalisation stack's whole step (B Q to update of its buckets) starts as soon as
+// its buckets' gradients have arrived, so it runs while the later stacks' gradients cross
+// the host link.  Stacks are uploaded largest first, so what is left after the last copy
+// is the step of the smallest one.
 static dion_status step_overlapped(dion_handle h, const dion_bucket_ptrs* ptrs,
                                    const float* const* host_grads, int32_t nbuckets, float lr,
                                    char* ws, int32_t* d_status, cudaStream_t main) {
-  std::vector<int32_t> order((size_t)nbuckets);
-  std::iota(order.begin(), order.end(), 0);
   auto grad_bytes = [&](int32_t b) {
     const Plan& p = h->plans[b];
     return (size_t)p.count * p.m * p.n * sizeof(float);
   };
-  std::stable_sort(order.begin(), order.end(),
-                   [&](int32_t a, int32_t b) { return grad_bytes(a) > grad_bytes(b); });
+  // stacks of the orthonormalisation in order of their gradients' size, largest first;
+  // a stack's step starts once all of its buckets' gradients are on the device
+  const int32_t ng = (int32_t)h->groups.size();
+  std::vector<int32_t> gorder((size_t)ng);
+  std::iota(gorder.begin(), gorder.end(), 0);
+  auto group_bytes = [&](int32_t g) {
+    size_t t = 0;
+    for (int32_t b : h->groups[g].members) t += grad_bytes(b);
+    return t;
+  };
+  std::stable_sort(gorder.begin(), gorder.end(),
+                   [&](int32_t a, int32_t b) { return group_bytes(a) > group_bytes(b); });
+  std::vector<int32_t> order;            // upload order of the buckets
+  std::vector<int32_t> last_upload((size_t)ng);
+  for (int32_t g : gorder) {
+    for (int32_t b : h->groups[g].members) order.push_back(b);
+    last_upload[g] = (int32_t)order.size() - 1;
+  }
   // the previous work on the caller's stream (an earlier step) may still read G
   cudaError_t e = cudaEventRecord(h->up_start, main);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(h->up, h->up_start, 0);
@@ -1025,28 +1133,39 @@ static dion_status step_overlapped(dion_handle h, const dion_bucket_ptrs* ptrs,
     }
   }
   StepCtx c{h, main, 0, -1, nullptr, 0, std::vector<int>(nbuckets, 0)};
-  int32_t waited = 0;  // uploads [0, waited) the caller's stream is ordered after
+  c.g_ready.assign((size_t)ng, 0);
+  int32_t waited = -1;  // the caller's stream is ordered after uploads [0, waited]
   auto finish = [&](dion_status result) -> dion_status {
     end_cls(c);
-    if (waited < nbuckets) cudaStreamWaitEvent(main, h->up_done[nbuckets - 1], 0);
+    if (waited < nbuckets - 1) cudaStreamWaitEvent(main, h->up_done[nbuckets - 1], 0);
     h->last_launches = c.launches;
     return result;
+  };
+  auto run = [&](int phase, int32_t b) {
+    c.s = main;
+    return run_bucket(c, b, phase, h->plans[b], ptrs[b], lr, ws, d_status);
   };
   dion_status st;
   for (int phase : {PH_INIT, PH_PREPQ})
     for (int32_t b = 0; b < nbuckets; ++b)
-      if ((st = run_bucket(c, b, phase, h->plans[b], ptrs[b], lr, ws, d_status)) != DION_OK)
-        return finish(st);
-  for (int32_t k = 0; k < nbuckets; ++k) {
-    const int32_t b = order[k];
-    if ((e = cudaStreamWaitEvent(main, h->up_done[k], 0)) != cudaSuccess)
+      if ((st = run(phase, b)) != DION_OK) return finish(st);
+  for (int32_t g : gorder) {
+    const OrthGroup& og = h->groups[g];
+    if ((e = cudaStreamWaitEvent(main, h->up_done[last_upload[g]], 0)) != cudaSuccess)
       return finish(fail(DION_ERR_CUDA, "upload wait: %s", cudaGetErrorString(e)));
-    waited = k + 1;
-    for (int phase : {PH_FORMB, PH_BQ, PH_ORTH, PH_BTP, PH_COLNORM, PH_UPDATE, PH_STATUS}) {
-      c.s = main;
-      if ((st = run_bucket(c, b, phase, h->plans[b], ptrs[b], lr, ws, d_status)) != DION_OK)
-        return finish(st);
+    waited = last_upload[g];
+    for (int32_t b : og.members) {
+      for (int phase : {PH_FORMB, PH_BQ})
+        if ((st = run(phase, b)) != DION_OK) return finish(st);
+      c.g_ready[g] = c.p0s_ready[b];
     }
+    c.s = main;
+    if ((st = run_bucket(c, g, PH_ORTH, og.orth, ptrs[og.members[0]], lr, ws, d_status)) !=
+        DION_OK)
+      return finish(st);
+    for (int32_t b : og.members)
+      for (int phase : {PH_BTP, PH_COLNORM, PH_UPDATE, PH_STATUS})
+        if ((st = run(phase, b)) != DION_OK) return finish(st);
   }
   return finish(DION_OK);
 }

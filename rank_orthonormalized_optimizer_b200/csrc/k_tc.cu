@@ -175,6 +175,7 @@ struct GemmP {
   int64_t ldc, c_bs;
   bf16* Cs;                          // three-way bf16 split of the result (may be null)
   int64_t cs_stride;                 // elements between the split parts
+  int zplane_a, zplane_b;            // split operands: matrices between parts (0: batch)
   bf16* Cb;                          // bf16 copy of the result (may be null)
   float* colsq;                      // per-warp column sums of squares (may be null):
                                      // [batch][tiles_m * 4][N], row block tm*4 + warp
@@ -305,18 +306,18 @@ __global__ void __launch_bounds__(NT, 1)
         for (int part = 0; part < SPLIT; ++part) {
           uint8_t* a_dst = sA + (size_t)stage * stage_a + part * p.a_bytes;
           uint8_t* b_dst = sB + (size_t)stage * stage_b + part * p.b_bytes;
-          const int z = part * p.batch + b;
+          const int za = part * p.zplane_a + b, zb = part * p.zplane_b + b;
           if (A_MN) {  // A^T stored [K][M]: boxes of 64 (M) x 64 (K)
-            tma_load_3d(a_dst, &tmA, full + stage, m0, k0, z);
-            tma_load_3d(a_dst + 8192, &tmA, full + stage, m0 + 64, k0, z);
+            tma_load_3d(a_dst, &tmA, full + stage, m0, k0, za);
+            tma_load_3d(a_dst + 8192, &tmA, full + stage, m0 + 64, k0, za);
           } else {     // A stored [M][K]: 128 rows of 64 K elements
-            tma_load_3d(a_dst, &tmA, full + stage, k0, m0, z);
+            tma_load_3d(a_dst, &tmA, full + stage, k0, m0, za);
           }
           if (B_MN) {  // B stored [K][N]: boxes of 64 (N) x 64 (K)
             for (int j = 0; j < p.block_n / 64; ++j)
-              tma_load_3d(b_dst + j * 8192, &tmB, full + stage, n0 + 64 * j, k0, z);
+              tma_load_3d(b_dst + j * 8192, &tmB, full + stage, n0 + 64 * j, k0, zb);
           } else {     // B stored [N][K]: block_n rows of 64 K elements
-            tma_load_3d(b_dst, &tmB, full + stage, k0, n0, z);
+            tma_load_3d(b_dst, &tmB, full + stage, k0, n0, zb);
           }
         }
         if (used < p.stages) ++used;
@@ -562,6 +563,8 @@ static cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Gem
                                cudaStream_t s) {
   p.a_bytes = BM * BK * 2;
   p.b_bytes = (uint32_t)p.block_n * BK * 2;
+  if (p.zplane_a == 0) p.zplane_a = p.batch;
+  if (p.zplane_b == 0) p.zplane_b = p.batch;
   const size_t stage_bytes = (size_t)SPLIT * (p.a_bytes + p.b_bytes);
   int stages = (int)((200 * 1024) / stage_bytes);
   if (stages > 8) stages = 8;
@@ -597,9 +600,9 @@ static int pick_block_n(int64_t r, int mult) {
 
 }  // namespace tc
 
-cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, bf16* P0s, int count, int64_t m,
-                       int64_t n, int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s,
-                       int* nlaunch, bool* done) {
+cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, bf16* P0s, int64_t plane,
+                       int count, int64_t m, int64_t n, int64_t r, int64_t max_spins,
+                       int32_t* flags, cudaStream_t s, int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
@@ -616,7 +619,7 @@ cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, bf16* P0s, int
   p.num_kb = (int)((n + BK - 1) / BK);
   p.idesc = idesc_bf16(BM, bn, false, false);
   p.C = P0; p.ldc = r; p.c_bs = m * r;
-  p.Cs = P0s; p.cs_stride = (int64_t)count * m * r;
+  p.Cs = P0s; p.cs_stride = plane > 0 ? plane : (int64_t)count * m * r;
   p.flags = flags;
   p.max_spins = max_spins;
   cudaError_t e = launch_gemm<false, false, 1>(ma, mb, p, s);
@@ -662,9 +665,10 @@ cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, float* colsq, 
 }
 
 // fp32 contractions on bf16 tensor cores: operands as three bf16 parts.
-cudaError_t tc_gemm_bq_split(const bf16* Bs, const bf16* Qs, float* P0, bf16* P0s, int count,
-                             int64_t m, int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
-                             cudaStream_t s, int* nlaunch, bool* done) {
+cudaError_t tc_gemm_bq_split(const bf16* Bs, const bf16* Qs, float* P0, bf16* P0s,
+                             int64_t plane, int count, int64_t m, int64_t n, int64_t r,
+                             int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
+                             bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
@@ -684,7 +688,7 @@ cudaError_t tc_gemm_bq_split(const bf16* Bs, const bf16* Qs, float* P0, bf16* P0
   // otherwise cost about K / 16 * 6 * 2^-24 relative (1.8e-4 at K = 8192), far above the
   // split's 2^-24; the chunks' partial sums pass through the fp32 P0
   p.C = P0; p.ldc = r; p.c_bs = m * r;
-  p.Cs = P0s; p.cs_stride = (int64_t)count * m * r;
+  p.Cs = P0s; p.cs_stride = plane > 0 ? plane : (int64_t)count * m * r;
   p.kchunk = KCHUNK_SUMSQ;
   p.flags = flags;
   p.max_spins = max_spins;
@@ -693,16 +697,20 @@ cudaError_t tc_gemm_bq_split(const bf16* Bs, const bf16* Qs, float* P0, bf16* P0
   return e;
 }
 
-cudaError_t tc_gemm_btp_split(const bf16* Bs, const bf16* Ps, float* R, float* colsq, int count,
-                              int64_t m, int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
-                              cudaStream_t s, int* nlaunch, bool* done) {
+cudaError_t tc_gemm_btp_split(const bf16* Bs, const bf16* Ps, int zplane_p, float* R,
+                              float* colsq, int count, int64_t m, int64_t n, int64_t r,
+                              int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
+                              bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
   const int bn = r <= 64 ? 64 : 128;        // MN-major B: whole 64-wide atoms
   CUtensorMap ma, mb;
+  // P's parts may lie further apart than count matrices (a stack shared with other
+  // buckets): part i of matrix b is matrix i * zplane_p + b
+  const int zp = zplane_p > 0 ? zplane_p : count;
   if (!map3d(&ma, Bs, true, n, m, 3 * (uint64_t)count, 64, BK)) return cudaSuccess;
-  if (!map3d(&mb, Ps, true, r, m, 3 * (uint64_t)count, 64, BK)) return cudaSuccess;
+  if (!map3d(&mb, Ps, true, r, m, 2 * (uint64_t)zp + count, 64, BK)) return cudaSuccess;
   GemmP p{};
   p.M = n; p.N = r; p.K = m;
   p.batch = count;
@@ -713,6 +721,7 @@ cudaError_t tc_gemm_btp_split(const bf16* Bs, const bf16* Ps, float* R, float* c
   p.idesc = idesc_bf16(BM, bn, true, true);
   p.C = R; p.ldc = r; p.c_bs = n * r;
   p.colsq = colsq;
+  p.zplane_b = zp;
   p.kchunk = KCHUNK_SUMSQ;  // unbiased accumulation over long K, as in B Q
   p.flags = flags;
   p.max_spins = max_spins;
@@ -1126,9 +1135,9 @@ __global__ void __launch_bounds__(FB_NT, 1)
 }  // namespace tc
 
 cudaError_t tc_formb_bq(const float* M, const float* G, const void* Qg, void* Bg, bf16* P0s,
-                        int count, int64_t m, int64_t n, int64_t r, int64_t max_spins,
-                        int32_t* flags, int* tile_counter, cudaStream_t s, int* nlaunch,
-                        bool* done) {
+                        int64_t plane, int count, int64_t m, int64_t n, int64_t r,
+                        int64_t max_spins, int32_t* flags, int* tile_counter, cudaStream_t s,
+                        int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
@@ -1149,7 +1158,7 @@ cudaError_t tc_formb_bq(const float* M, const float* G, const void* Qg, void* Bg
   p.b_bytes = (uint32_t)bn * BK * 2;
   p.tmem_cols = pow2_cols(2 * bn);
   p.P0s = P0s;
-  p.cs_stride = (int64_t)count * m * r;
+  p.cs_stride = plane > 0 ? plane : (int64_t)count * m * r;
   p.flags = flags;
   p.tile_counter = tile_counter;
   p.max_spins = max_spins;
@@ -1177,6 +1186,7 @@ struct UpdP {
   int* tile_counter;  // zero before the launch; tiles are taken from it in order
   int npairs;         // 1: bf16 operands; 3: split operands, products (1,0) (0,1) (0,0)
   int pa[3], pb[3];   // part of P and of R, Q in each product
+  int zplane_p;       // matrices between P's split parts
   int64_t max_spins;
   float* rmmc;        // [2][batch]: max |M' - M| and max |M| per matrix (max-ed into)
 };
@@ -1279,7 +1289,7 @@ __global__ void __launch_bounds__(NT, 1)
       bool ok = true;
       for (int it = 0; it < p.num_kb * p.npairs; ++it) {
         const int kb = it / p.npairs, pi = it % p.npairs;
-        const int za = p.pa[pi] * p.batch + b, zb = p.pb[pi] * p.batch + b;
+        const int za = p.pa[pi] * p.zplane_p + b, zb = p.pb[pi] * p.batch + b;
         if (!wait_bounded(empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
         mbar_expect_tx(full + stage, UPD_A_BYTES + UPD_B_BYTES);
         uint8_t* a_dst = sA + stage * UPD_A_BYTES;
@@ -1471,16 +1481,18 @@ __global__ void __launch_bounds__(NT, 1)
 
 }  // namespace tc
 
-cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, bool split, const float* G,
-                      float* M, float* X, int count, int64_t m, int64_t n, int64_t r, float mu,
-                      float lr_scale, int64_t max_spins, int32_t* flags, int* tile_counter,
-                      float* rmmc, cudaStream_t s, int* nlaunch, bool* done) {
+cudaError_t tc_update(const void* Pg, int zplane_p, const void* Rg, const void* Qg, bool split,
+                      const float* G, float* M, float* X, int count, int64_t m, int64_t n,
+                      int64_t r, float mu, float lr_scale, int64_t max_spins, int32_t* flags,
+                      int* tile_counter, float* rmmc, cudaStream_t s, int* nlaunch, bool* done) {
   using namespace tc;
   *nlaunch = 0;
   *done = false;
   CUtensorMap mP, mR, mQ, mM, mG, mX, mMs, mXs;
   const uint64_t zc = (split ? 3 : 1) * (uint64_t)count;
-  bool ok = map3d(&mP, Pg, true, r, m, zc, BK, BM) && map3d(&mR, Rg, true, r, n, zc, BK, UPD_BN) &&
+  const int zp = zplane_p > 0 ? zplane_p : count;  // matrices between P's split parts
+  const uint64_t zcp = split ? 2 * (uint64_t)zp + count : (uint64_t)count;
+  bool ok = map3d(&mP, Pg, true, r, m, zcp, BK, BM) && map3d(&mR, Rg, true, r, n, zc, BK, UPD_BN) &&
             map3d(&mQ, Qg, true, r, n, zc, BK, UPD_BN) &&
             map3d(&mM, M, false, n, m, count, SLAB, BM) && map3d(&mG, G, false, n, m, count, SLAB, BM) &&
             map3d(&mX, X, false, n, m, count, SLAB, BM) &&
@@ -1501,6 +1513,7 @@ cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, bool split
   p.pa[0] = split ? 1 : 0; p.pb[0] = 0;
   p.pa[1] = 0; p.pb[1] = split ? 1 : 0;
   p.pa[2] = 0; p.pb[2] = 0;
+  p.zplane_p = zp;
   p.max_spins = max_spins;
   p.rmmc = rmmc;
   cudaError_t e = cudaFuncSetAttribute(k_tc_update, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -14,17 +14,21 @@ namespace dion {
 const char* tc_map_error();
 
 // P0[b] (m x r, fp32) = Bg[b] (m x n, bf16) * Qg[b]^T (Qg: r x n, bf16); when P0s is
-// not null its three-way bf16 split ([3][count][m][r]) is written as well.
-cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, __nv_bfloat16* P0s, int count,
-                       int64_t m, int64_t n, int64_t r, int64_t max_spins, int32_t* flags,
-                       cudaStream_t s, int* nlaunch, bool* done);
+// not null its three-way bf16 split is written as well, its parts `plane` elements
+// apart (0: count * m * r, [3][count][m][r]; more when the bucket's P0 lies in a stack
+// shared with other buckets of the same m and r).
+cudaError_t tc_gemm_bq(const void* Bg, const void* Qg, float* P0, __nv_bfloat16* P0s,
+                       int64_t plane, int count, int64_t m, int64_t n, int64_t r,
+                       int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
+                       bool* done);
 // Steps 1 and 2 fused: Bg[b] = bf16(M[b] + G[b]) (written for B^T P) and the
 // three-way bf16 split of P0[b] = Bg[b] Qg[b]^T into P0s ([3][count][m][r]).
 // tile_counter: one int in device memory, zero before the call (tiles are taken from it).
+// P0s's parts lie `plane` elements apart (0: count * m * r).
 cudaError_t tc_formb_bq(const float* M, const float* G, const void* Qg, void* Bg,
-                        __nv_bfloat16* P0s, int count, int64_t m, int64_t n, int64_t r,
-                        int64_t max_spins, int32_t* flags, int* tile_counter, cudaStream_t s,
-                        int* nlaunch, bool* done);
+                        __nv_bfloat16* P0s, int64_t plane, int count, int64_t m, int64_t n,
+                        int64_t r, int64_t max_spins, int32_t* flags, int* tile_counter,
+                        cudaStream_t s, int* nlaunch, bool* done);
 // R[b] (n x r, fp32) = Bg[b]^T (n x m) * Pg[b] (m x r, bf16).  When colsq is not null it
 // receives the sums of squares of R's columns over blocks of R's rows, fixed order:
 // colsq[b][i][j] for row block i < tc_btp_col_splits(n) (the partials of Q = colnorm(R)).
@@ -38,18 +42,20 @@ int tc_btp_col_splits(int64_t n);
 // split: Pg, Rg, Qg are three-way bf16 splits ([3][count][...]) of fp32 operands.
 // rmmc: [2][count] floats, max |M' - M| and max |M| of each matrix max-ed into them
 // (non-negative before the call).
-cudaError_t tc_update(const void* Pg, const void* Rg, const void* Qg, bool split, const float* G,
-                      float* M, float* X, int count, int64_t m, int64_t n, int64_t r, float mu,
-                      float lr_scale, int64_t max_spins, int32_t* flags, int* tile_counter,
-                      float* rmmc, cudaStream_t s, int* nlaunch, bool* done);
+// zplane_p: matrices between Pg's split parts (0: count).
+cudaError_t tc_update(const void* Pg, int zplane_p, const void* Rg, const void* Qg, bool split,
+                      const float* G, float* M, float* X, int count, int64_t m, int64_t n,
+                      int64_t r, float mu, float lr_scale, int64_t max_spins, int32_t* flags,
+                      int* tile_counter, float* rmmc, cudaStream_t s, int* nlaunch, bool* done);
 // fp32 contractions from three-way bf16 splits: P0 (fp32) and P0s = split(Bs Qs^T),
 // R = Bs^T Ps; K is accumulated in 512-wide chunks added in fp32 registers.
+// (P0s's parts `plane` elements apart, Ps's `zplane_p` matrices apart; 0: count.)
 cudaError_t tc_gemm_bq_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Qs, float* P0,
-                             __nv_bfloat16* P0s, int count, int64_t m, int64_t n, int64_t r,
-                             int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
-                             bool* done);
-cudaError_t tc_gemm_btp_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Ps, float* R,
-                              float* colsq, int count, int64_t m, int64_t n, int64_t r,
+                             __nv_bfloat16* P0s, int64_t plane, int count, int64_t m, int64_t n,
+                             int64_t r, int64_t max_spins, int32_t* flags, cudaStream_t s,
+                             int* nlaunch, bool* done);
+cudaError_t tc_gemm_btp_split(const __nv_bfloat16* Bs, const __nv_bfloat16* Ps, int zplane_p,
+                              float* R, float* colsq, int count, int64_t m, int64_t n, int64_t r,
                               int64_t max_spins, int32_t* flags, cudaStream_t s, int* nlaunch,
                               bool* done);
 

@@ -144,6 +144,11 @@ EDGE = [
     # r <= 256 with m over 512 rows: the Gram adds 512-row K chunks in fp32 (3 chunks,
     # the last ragged; 5 chunks over a 2 x 2 tile grid with r = 144)
     ("chunked_gram", [(3, 1300, 96, 64), (2, 2100, 256, 144)]),
+    # buckets of equal m and r share one orthonormalisation stack: the first and third
+    # here (the stack completes after the third bucket's B Q), the second alone
+    ("stacked_orth", [(3, 256, 128, 32), (2, 300, 64, 48), (2, 256, 384, 32)]),
+    # a stack on the recursive factorisation (r = 272 > 256)
+    ("stacked_recursive", [(2, 600, 560, 272), (1, 600, 320, 272)]),
 ]
 
 
@@ -302,7 +307,8 @@ def test_step_from_host_equals_device_step(precision):
     that the previous step's update read, it gives bitwise the device step's state and
     status.  The buckets are listed smallest first, so the upload order is not theirs;
     r = 272 takes the recursive factorisation and the fallback graph."""
-    wl = W.custom("from_host", [(2, 256, 128, 32), (3, 600, 560, 272), (4, 1024, 512, 64)],
+    wl = W.custom("from_host", [(2, 256, 128, 32), (3, 600, 560, 272), (4, 1024, 512, 64),
+                                (1, 256, 64, 32)],
                   precision=precision, steps=3)
     a = GpuRun(wl)
     b = GpuRun(wl)
@@ -320,6 +326,29 @@ def test_step_from_host_equals_device_step(precision):
             assert torch.equal(b.G[i].cpu(), grads[i])
         assert torch.equal(host_status, a.status.cpu()), t
         assert torch.equal(b.status.cpu(), a.status.cpu()), t
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_stacked_orthonormalisation_is_bucket_by_bucket_bitwise(precision):
+    """Buckets of equal m and r share one orthonormalisation stack; every matrix is still
+    orthonormalised on its own (its own Gram tiles, its own Cholesky), so a bucket's X, M,
+    Q and status are bit for bit those of the same bucket planned alone."""
+    shapes = [(3, 256, 128, 32), (2, 256, 384, 32), (2, 600, 560, 272), (1, 600, 320, 272)]
+    wl = W.custom(f"stacked_{precision}", shapes, precision=precision, steps=3)
+    together = GpuRun(wl)
+    together.step(3)
+    for i, b in enumerate(shapes):
+        alone_wl = W.custom(f"stacked_{precision}", [b], precision=precision, steps=3)
+        alone = GpuRun(alone_wl)
+        # the same inputs: bucket i's seeds under the stacked workload's name and index
+        alone.X[0].copy_(W.weights(wl, i, alone.gen).cuda())
+        alone.Q[0].copy_(W.right_factor(wl, i, alone.gen).cuda())
+        for t in range(3):
+            alone.step(1, G_override=[W.gradient(wl, i, t, alone.gen).cuda()])
+        assert torch.equal(alone.X[0], together.X[i]), i
+        assert torch.equal(alone.M[0], together.M[i]) and torch.equal(alone.Q[0], together.Q[i]), i
+        lo = sum(s[0] for s in shapes[:i])
+        assert torch.equal(alone.status.cpu(), together.status.cpu()[lo:lo + b[0]]), i
 
 
 def test_tensor_and_simt_paths_agree():
