@@ -71,6 +71,9 @@ struct Plan {
       off_gather, off_rmmc;
 };
 
+// Whether buckets of equal m and r share one orthonormalisation stack.
+constexpr bool kStackOrth = true;
+
 // A stack of the orthonormalisation: the buckets whose P has the same shape (m x r),
 // whatever their n, stacked into one [count, m, r] batch.  `orth` is a plan of the whole
 // stack (count = the members' counts summed) for the orthonormalisation's kernels.
@@ -904,7 +907,7 @@ static dion_status dion_init_impl(const dion_bucket_desc* buckets, const dion_sh
   for (int32_t b = 0; b < nbuckets; ++b) {
     Plan& p = plans[b];
     int gi = -1;
-    if (!sharded)
+    if (!sharded && kStackOrth)
       for (size_t g = 0; g < groups.size(); ++g) {
         const Plan& q = plans[groups[g].members[0]];
         if (q.m == p.m && q.r == p.r) gi = (int)g;

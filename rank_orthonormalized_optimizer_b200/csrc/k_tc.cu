@@ -844,9 +844,12 @@ namespace tc {
 // 128-byte-swizzled A operand of the MMA; the same shared-memory bytes are stored by
 // TMA as bf16 B for the later B^T P.  B is read from HBM once (8 bytes per element)
 // and written once (2 bytes); nothing re-reads it for B Q.
-//   warp 0       TMA: M, G (fp32, 2 boxes of 32 columns each) and the Q^T tile
+//   warp 0       TMA: M, G (fp32, 2 boxes of 32 columns each)
 //   warp 1       MMA issuer
 //   warp 2       TMEM allocator
+//   warp 3       TMA: the Q^T tile (apart from M and G, so that a stage's fp32 staging
+//                is refilled as soon as the converters are done with it, without
+//                waiting for the MMA to release the stage's Q^T)
 //   warps 4..7   epilogue: P0's three-way bf16 split
 //   warps 8..11  converters
 // Tiles of the fused kernel come in order from a global counter through a ring of
@@ -868,9 +871,9 @@ struct FusedP {
   int* tile_counter;  // zero before the launch; tiles are taken from it in order
   int64_t max_spins;
 };
-// consumers of the fused kernel's tile ring: MMA issuer, four converter warps, four
-// epilogue warps (the TMA producer fills it)
-constexpr int FB_RING_CONSUMERS = 9;
+// consumers of the fused kernel's tile ring: the Q^T producer, the MMA issuer, four
+// converter warps, four epilogue warps (the M, G producer fills it)
+constexpr int FB_RING_CONSUMERS = 10;
 
 __global__ void __launch_bounds__(FB_NT, 1)
     k_tc_formb_bq(const __grid_constant__ CUtensorMap tmM, const __grid_constant__ CUtensorMap tmG,
@@ -946,10 +949,9 @@ __global__ void __launch_bounds__(FB_NT, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer of M and G
     prefetch_map(&tmM);
     prefetch_map(&tmG);
-    prefetch_map(&tmQ);
     int stage = 0, used = 0, slot = 0;
     uint32_t phase = 0, rphase = 0;
     while (true) {
@@ -964,11 +966,9 @@ __global__ void __launch_bounds__(FB_NT, 1)
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
       const int m0 = (rem / p.tiles_n) * BM;
-      const int n0 = (rem % p.tiles_n) * p.block_n;
       bool ok = true;
       for (int kb = 0; kb < p.num_kb; ++kb) {
-        if (!wait_bounded(f_empty + stage, phase ^ 1, p.max_spins, abort) ||
-            !wait_bounded(b_empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
+        if (!wait_bounded(f_empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
         const int k0 = kb * BK;
         uint8_t* f = sF + stage * FB_F32_BYTES;
         mbar_expect_tx(f_full + stage, FB_F32_BYTES);
@@ -976,8 +976,6 @@ __global__ void __launch_bounds__(FB_NT, 1)
         tma_load_3d(f + 16384, &tmM, f_full + stage, k0 + 32, m0, b);
         tma_load_3d(f + 32768, &tmG, f_full + stage, k0, m0, b);
         tma_load_3d(f + 49152, &tmG, f_full + stage, k0 + 32, m0, b);
-        mbar_expect_tx(b_full + stage, p.b_bytes);
-        tma_load_3d(sB + stage * p.b_bytes, &tmQ, b_full + stage, k0, n0, b);
         if (used < FB_STAGES) ++used;
         if (++stage == FB_STAGES) { stage = 0; phase ^= 1; }
       }
@@ -988,6 +986,29 @@ __global__ void __launch_bounds__(FB_NT, 1)
         stage = (stage + FB_STAGES - 1) % FB_STAGES;
         if (stage == FB_STAGES - 1) phase ^= 1;
         wait_drain(f_full + stage, phase);
+      }
+  } else if (warp == 3 && lane == 0) {
+    // ---------------- TMA producer of the Q^T tiles
+    prefetch_map(&tmQ);
+    int stage = 0, used = 0;
+    uint32_t phase = 0;
+    for (int t = next_tile(false); t >= 0; t = next_tile(false)) {
+      const int b = t / tiles_per_mat;
+      const int n0 = (t % tiles_per_mat % p.tiles_n) * p.block_n;
+      bool ok = true;
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!wait_bounded(b_empty + stage, phase ^ 1, p.max_spins, abort)) { ok = false; break; }
+        mbar_expect_tx(b_full + stage, p.b_bytes);
+        tma_load_3d(sB + stage * p.b_bytes, &tmQ, b_full + stage, kb * BK, n0, b);
+        if (used < FB_STAGES) ++used;
+        if (++stage == FB_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+    if (*abort)
+      for (int i = 0; i < used; ++i) {
+        stage = (stage + FB_STAGES - 1) % FB_STAGES;
+        if (stage == FB_STAGES - 1) phase ^= 1;
         wait_drain(b_full + stage, phase);
       }
   } else if (warp == 1 && lane == 0) {
