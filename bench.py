@@ -234,16 +234,32 @@ def measured_peaks():
             "source": "fallback"}
 
 
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_tc_update_traffic_stack16x4096_r256.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_tc_update_traffic_r256_shapes.json")
 
 
 def update_traffic():
-    """DRAM bytes per weight element of the fused update, from the committed ncu capture,
-    and the hash of the kernel source it was taken on."""
+    """DRAM bytes per weight element of the fused update by matrix shape ("MxN"), from the
+    committed ncu captures, and the hash of the kernel source they were taken on."""
     if os.path.exists(TRAFFIC_FILE):
         d = json.load(open(TRAFFIC_FILE))
         return d.get("dram_bytes_per_element"), d.get("kernel_source_hash")
     return None, None
+
+
+def update_traffic_per_launch(wl: W.Workload, launches: float):
+    """The update's DRAM bytes per launch on this workload from the per-shape captures
+    (bytes per element of each bucket's shape times its elements, over the launches);
+    None when a bucket's shape was not captured or the kernel changed since."""
+    per, h = update_traffic()
+    if not per or h != update_kernel_hash() or launches <= 0:
+        return None
+    total = 0.0
+    for b in wl.buckets:
+        key = f"{b.m}x{b.n}"
+        if key not in per:
+            return None
+        total += per[key] * b.params
+    return total / launches
 
 
 def update_kernel_hash():
@@ -360,10 +376,7 @@ def run_ours(args):
     upd_ms = prof["update"][0] / args.steps
     upd_launches = prof["update"][1] / args.steps
     achieved = upd_bytes / (upd_ms / 1e3) / 1e9
-    traffic_per_elem, traffic_hash = update_traffic()
-    traffic = None
-    if traffic_per_elem is not None and traffic_hash == update_kernel_hash():
-        traffic = traffic_per_elem * sum(b.params for b in wl.buckets) / max(upd_launches, 1)
+    traffic = update_traffic_per_launch(wl, upd_launches)
     roof_t = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_alg / (peaks["hbm_gbs"] * 1e9))
     comp_bytes = sum(b.count * (20 * b.m * b.n + 8 * b.n * b.r) for b in wl.buckets)
     comp_t = comp_bytes / (peaks["hbm_gbs"] * 1e9)

@@ -128,6 +128,15 @@ typedef struct dion_options {
                               kernel sets DION_MAT_TIMEOUT and returns (default 1<<26)     */
   float rmmc_threshold;    /* DION_MAT_HIGH_RMMC where RMMC exceeds it (default 0: every
                               matrix whose momentum moved; not NaN)                        */
+  int32_t stack_orth;      /* 1: buckets of equal m and r share one orthonormalisation
+                              stack -- one Gram, Cholesky and apply launch over all their
+                              matrices, as "DASH: Faster Shampoo via Batched Block
+                              Preconditioning and Efficient Inverse-Root Solvers"
+                              (Methodologie, section 1) stacks equal-sized blocks of
+                              different layers; results are bit for bit those of 0.  It
+                              pays where many small buckets leave each launch latency-
+                              bound; the stack can only start after its last bucket's
+                              B Q, which costs overlap on large buckets (default 0)      */
 } dion_options;
 
 /* Device buffers of one bucket, all contiguous, row-major, 16-byte aligned:

@@ -50,7 +50,8 @@ class BucketDesc(ctypes.Structure):
 class Options(ctypes.Structure):
     _fields_ = [("mu", c_float), ("precision", c_int32), ("orth_mode", c_int32),
                 ("fallback_cond", c_float), ("orth_tol", c_float), ("kernel_path", c_int32),
-                ("max_wait_spins", c_int64), ("rmmc_threshold", c_float)]
+                ("max_wait_spins", c_int64), ("rmmc_threshold", c_float),
+                ("stack_orth", c_int32)]
 
 
 class BucketPtrs(ctypes.Structure):
@@ -162,9 +163,10 @@ class Shape:
 
 
 def _make_options(mu, precision, orth_mode, kernel_path, fallback_cond, orth_tol,
-                  max_wait_spins, rmmc_threshold=0.0) -> Options:
+                  max_wait_spins, rmmc_threshold=0.0, stack_orth=False) -> Options:
     o = default_options()
     o.rmmc_threshold = rmmc_threshold
+    o.stack_orth = int(bool(stack_orth))
     o.mu = mu
     o.precision = PRECISIONS[precision]
     o.orth_mode = ORTH_MODES[orth_mode]
@@ -193,10 +195,10 @@ class DionB200:
 
     def __init__(self, buckets, *, mu=0.95, precision="bf16", orth_mode="auto",
                  kernel_path="tensor", fallback_cond=1e3, orth_tol=2e-5,
-                 max_wait_spins=1 << 26, scales=None, rmmc_threshold=0.0):
+                 max_wait_spins=1 << 26, scales=None, rmmc_threshold=0.0, stack_orth=False):
         self.shapes = [Shape(*map(int, b)) for b in buckets]
         self.options = _make_options(mu, precision, orth_mode, kernel_path, fallback_cond,
-                                     orth_tol, max_wait_spins, rmmc_threshold)
+                                     orth_tol, max_wait_spins, rmmc_threshold, stack_orth)
         h = c_void_p()
         ws = c_size_t()
         _check(dion_init(_descs(self.shapes, scales), len(self.shapes),

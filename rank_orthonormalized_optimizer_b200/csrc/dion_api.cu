@@ -71,9 +71,6 @@ struct Plan {
       off_gather, off_rmmc;
 };
 
-// Whether buckets of equal m and r share one orthonormalisation stack.
-constexpr bool kStackOrth = true;
-
 // A stack of the orthonormalisation: the buckets whose P has the same shape (m x r),
 // whatever their n, stacked into one [count, m, r] batch.  `orth` is a plan of the whole
 // stack (count = the members' counts summed) for the orthonormalisation's kernels.
@@ -164,6 +161,8 @@ dion_status check_options(const dion_options& o) {
   if (o.max_wait_spins < 1) return fail(DION_ERR_INVALID_ARG, "max_wait_spins must be >= 1");
   if (std::isnan(o.rmmc_threshold))
     return fail(DION_ERR_INVALID_ARG, "rmmc_threshold is NaN");
+  if (o.stack_orth != 0 && o.stack_orth != 1)
+    return fail(DION_ERR_INVALID_ARG, "stack_orth must be 0 or 1");
   return DION_OK;
 }
 
@@ -811,6 +810,7 @@ dion_status dion_default_options(dion_options* opt) {
   opt->kernel_path = DION_PATH_TENSOR;
   opt->max_wait_spins = int64_t(1) << 26;
   opt->rmmc_threshold = 0.f;
+  opt->stack_orth = 0;
   return DION_OK;
 }
 
@@ -897,17 +897,18 @@ static dion_status dion_init_impl(const dion_bucket_desc* buckets, const dion_sh
     }
     off = align_up(off_rblk + rblk * 4, 1024);
   }
-  // Stacks of the orthonormalisation: the buckets whose P has the same shape (m, r)
-  // share one [count, m, r] stack of every per-matrix array the orthonormalisation uses
-  // (P0, P and their splits, the Gram and the factor, flags, statistics), so that it runs
-  // once over all of them, as DASH stacks equal-sized blocks of different layers.  Each
-  // bucket's arrays are slices of its stack.  A row-sharded plan keeps one stack per
-  // bucket (its exchanges are laid out per bucket).
+  // Stacks of the orthonormalisation: with stack_orth, the buckets whose P has the same
+  // shape (m, r) share one [count, m, r] stack of every per-matrix array the
+  // orthonormalisation uses (P0, P and their splits, the Gram and the factor, flags,
+  // statistics), so that it runs once over all of them, as DASH stacks equal-sized
+  // blocks of different layers.  Each bucket's arrays are slices of its stack.  Without
+  // it (and always in a row-sharded plan, whose exchanges are laid out per bucket) every
+  // bucket is a stack of its own.
   std::vector<OrthGroup> groups;
   for (int32_t b = 0; b < nbuckets; ++b) {
     Plan& p = plans[b];
     int gi = -1;
-    if (!sharded && kStackOrth)
+    if (!sharded && o.stack_orth)
       for (size_t g = 0; g < groups.size(); ++g) {
         const Plan& q = plans[groups[g].members[0]];
         if (q.m == p.m && q.r == p.r) gi = (int)g;

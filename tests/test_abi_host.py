@@ -92,10 +92,23 @@ def test_init_shape_checks(bucket, code):
 
 @pytest.mark.parametrize("field,value", [("mu", 1.0), ("mu", -0.1), ("precision", 7),
                                          ("orth_mode", 9), ("fallback_cond", 0.5),
-                                         ("kernel_path", 3), ("max_wait_spins", 0)])
+                                         ("kernel_path", 3), ("max_wait_spins", 0),
+                                         ("rmmc_threshold", float("nan")), ("stack_orth", 2)])
 def test_init_option_checks(field, value):
     c, h, _ = _init([(1, 256, 128, 32)], **{field: value})
     assert c == dion.ERR_INVALID_ARG
+
+
+def test_stacking_shares_the_orthonormalisation_arrays():
+    """Buckets of equal m and r stacked: the same arrays, laid out once per stack, so the
+    workspace is no larger than without stacking (up to alignment)."""
+    shapes = [(3, 256, 128, 32), (2, 256, 384, 32), (2, 200, 136, 16)]
+    c0, h0, ws0 = _init(shapes)
+    c1, h1, ws1 = _init(shapes, stack_orth=1)
+    assert c0 == c1 == dion.OK
+    assert ws1 <= ws0
+    for h in (h0, h1):
+        dion.dion_free(h)
 
 
 def test_workspace_covers_the_layout():

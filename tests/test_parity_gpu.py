@@ -144,8 +144,9 @@ EDGE = [
     # r <= 256 with m over 512 rows: the Gram adds 512-row K chunks in fp32 (3 chunks,
     # the last ragged; 5 chunks over a 2 x 2 tile grid with r = 144)
     ("chunked_gram", [(3, 1300, 96, 64), (2, 2100, 256, 144)]),
-    # buckets of equal m and r share one orthonormalisation stack: the first and third
-    # here (the stack completes after the third bucket's B Q), the second alone
+    # with stack_orth, buckets of equal m and r share one orthonormalisation stack: the
+    # first and third here (the stack completes after the third bucket's B Q), the
+    # second alone
     ("stacked_orth", [(3, 256, 128, 32), (2, 300, 64, 48), (2, 256, 384, 32)]),
     # a stack on the recursive factorisation (r = 272 > 256)
     ("stacked_recursive", [(2, 600, 560, 272), (1, 600, 320, 272)]),
@@ -157,7 +158,7 @@ EDGE = [
 @pytest.mark.parametrize("name,buckets", EDGE, ids=[e[0] for e in EDGE])
 def test_edge_shapes(name, buckets, precision, path):
     wl = W.custom(f"edge_{name}", buckets, precision=precision, steps=4)
-    run = GpuRun(wl, kernel_path=path)
+    run = GpuRun(wl, kernel_path=path, stack_orth=name.startswith("stacked"))
     X_before = [x.clone() for x in run.X]
     rep = compare(run, 4)
     _check(rep, precision, dx=False)
@@ -310,8 +311,9 @@ def test_step_from_host_equals_device_step(precision):
     wl = W.custom("from_host", [(2, 256, 128, 32), (3, 600, 560, 272), (4, 1024, 512, 64),
                                 (1, 256, 64, 32)],
                   precision=precision, steps=3)
-    a = GpuRun(wl)
-    b = GpuRun(wl)
+    # the first and last bucket share an orthonormalisation stack
+    a = GpuRun(wl, stack_orth=True)
+    b = GpuRun(wl, stack_orth=True)
     nb = len(wl.buckets)
     host_status = torch.zeros(b.opt.num_matrices, dtype=torch.int32).pin_memory()
     for t in range(3):
@@ -330,12 +332,12 @@ def test_step_from_host_equals_device_step(precision):
 
 @pytest.mark.parametrize("precision", ["fp32", "bf16"])
 def test_stacked_orthonormalisation_is_bucket_by_bucket_bitwise(precision):
-    """Buckets of equal m and r share one orthonormalisation stack; every matrix is still
-    orthonormalised on its own (its own Gram tiles, its own Cholesky), so a bucket's X, M,
-    Q and status are bit for bit those of the same bucket planned alone."""
+    """With stack_orth, buckets of equal m and r share one orthonormalisation stack; every
+    matrix is still orthonormalised on its own (its own Gram tiles, its own Cholesky), so
+    a bucket's X, M, Q and status are bit for bit those of the same bucket planned alone."""
     shapes = [(3, 256, 128, 32), (2, 256, 384, 32), (2, 600, 560, 272), (1, 600, 320, 272)]
     wl = W.custom(f"stacked_{precision}", shapes, precision=precision, steps=3)
-    together = GpuRun(wl)
+    together = GpuRun(wl, stack_orth=True)
     together.step(3)
     for i, b in enumerate(shapes):
         alone_wl = W.custom(f"stacked_{precision}", [b], precision=precision, steps=3)
