@@ -31,10 +31,6 @@ namespace dion {
 namespace tc {
 
 constexpr int BM = 128;       // tile rows = TMEM lanes
-// B^T P with r > 128: both 128-row halves of a tile of R^T in one CTA (two MMAs per B
-// stage, one accumulator of 512 TMEM columns) rather than on two neighbouring CTAs
-// that each read the B stage from L2 (double-buffered accumulators)
-constexpr bool kBtpPairHalves = true;
 constexpr int KCHUNK_SUMSQ = 8;  // K blocks per accumulation chunk of sums of squares
 constexpr int EPI_LD = 17;       // row stride (floats) of the epilogue's staging blocks
 constexpr int BK = 64;        // bf16 elements per 128-byte swizzle row
@@ -180,9 +176,6 @@ struct GemmP {
   bf16* Cs;                          // three-way bf16 split of the result (may be null)
   int64_t cs_stride;                 // elements between the split parts
   int zplane_a, zplane_b;            // split operands: matrices between parts (0: batch)
-  int m2;                            // both 128-row halves of a 256-row tile in one CTA
-                                     // (A MN-major, one operand part): two MMAs share each
-                                     // B stage; one accumulator of 2 block_n columns
   bf16* Cb;                          // bf16 copy of the result (may be null)
   float* colsq;                      // per-warp column sums of squares (may be null):
                                      // [batch][tiles_m * 4][N], row block tm*4 + warp
@@ -300,7 +293,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (!tile_active(p, t, tiles_per_mat)) continue;
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
-      const int m0 = tile_mi(p, rem) * (p.m2 ? 2 * BM : BM);
+      const int m0 = tile_mi(p, rem) * BM;
       const int n0 = tile_ni(p, rem) * p.block_n;
       int kb0, kb1;
       k_range(p, m0, n0, kb0, kb1);
@@ -315,10 +308,8 @@ __global__ void __launch_bounds__(NT, 1)
           uint8_t* b_dst = sB + (size_t)stage * stage_b + part * p.b_bytes;
           const int za = part * p.zplane_a + b, zb = part * p.zplane_b + b;
           if (A_MN) {  // A^T stored [K][M]: boxes of 64 (M) x 64 (K)
-            for (int h = 0; h < (p.m2 ? 2 : 1); ++h) {  // the 128-row halves, 16 KB apart
-              tma_load_3d(a_dst + h * 16384, &tmA, full + stage, m0 + h * BM, k0, za);
-              tma_load_3d(a_dst + h * 16384 + 8192, &tmA, full + stage, m0 + h * BM + 64, k0, za);
-            }
+            tma_load_3d(a_dst, &tmA, full + stage, m0, k0, za);
+            tma_load_3d(a_dst + 8192, &tmA, full + stage, m0 + 64, k0, za);
           } else {     // A stored [M][K]: 128 rows of 64 K elements
             tma_load_3d(a_dst, &tmA, full + stage, k0, m0, za);
           }
@@ -358,13 +349,11 @@ __global__ void __launch_bounds__(NT, 1)
       if (!tile_active(p, t, tiles_per_mat)) continue;
       const int rem = t % tiles_per_mat;
       int kb0, kb1;
-      k_range(p, tile_mi(p, rem) * (p.m2 ? 2 * BM : BM), tile_ni(p, rem) * p.block_n, kb0, kb1);
+      k_range(p, tile_mi(p, rem) * BM, tile_ni(p, rem) * p.block_n, kb0, kb1);
       const int nch = n_chunks(p, kb0, kb1);
       for (int ch = 0; ch < nch && ok; ++ch) {
-      // two accumulators alternate between tiles; with m2 the one accumulator holds both
-      // halves and every tile waits for the epilogue of the one before
-      const int acc = p.m2 ? 0 : (lt & 1);
-      const uint32_t acc_phase = p.m2 ? (uint32_t)(lt & 1) : (uint32_t)((lt >> 1) & 1);
+      const int acc = lt & 1;
+      const uint32_t acc_phase = (lt >> 1) & 1;
       if (!wait_bounded(tempty + acc, acc_phase ^ 1, p.max_spins, abort)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d = tmem + acc * p.acc_stride;
@@ -386,9 +375,6 @@ __global__ void __launch_bounds__(NT, 1)
             const uint64_t bd = B_MN ? sw128_desc(bb + k * 2048, 8192, 1024)
                                      : sw128_desc(bb + k * 32, 16, 1024);
             mma_bf16(d, ad, bd, p.idesc, ((kb - c0) | k | q) != 0);
-            if (A_MN && SPLIT == 1 && p.m2)  // the second half: A 16 KB further, D block_n
-              mma_bf16(d + p.block_n, sw128_desc(ab + 16384 + k * 2048, 8192, 1024), bd, p.idesc,
-                       ((kb - c0) | k | q) != 0);
           }
         }
         mma_commit(empty + stage);
@@ -420,11 +406,10 @@ __global__ void __launch_bounds__(NT, 1)
       if (!tile_active(p, t, tiles_per_mat)) continue;
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
-      const int nh = p.m2 ? 2 : 1;  // 128-row halves of the tile
-      const int64_t rowb = (int64_t)tile_mi(p, rem) * (nh * BM) + ew * 32;  // this warp's rows
+      const int64_t row0 = (int64_t)tile_mi(p, rem) * BM + ew * 32;  // this warp's rows
       const int64_t n0 = (int64_t)tile_ni(p, rem) * p.block_n;
       int kb0, kb1;
-      k_range(p, tile_mi(p, rem) * (nh * BM), (int)n0, kb0, kb1);
+      k_range(p, tile_mi(p, rem) * BM, (int)n0, kb0, kb1);
       float rsq = 0.f;  // transposed store: this lane's row sum of squares over the tile
       const int nch = n_chunks(p, kb0, kb1);
       // split operands: the chunks are added, in fp32 registers, into a running sum kept
@@ -434,17 +419,14 @@ __global__ void __launch_bounds__(NT, 1)
       const bool tsum = SPLIT > 1 && nch > 1;
       const uint32_t sbase = tmem + ((uint32_t)(ew * 32) << 16) + 2 * p.acc_stride;
       for (int ch = 0; ch < nch; ++ch) {
-        const int acc = p.m2 ? 0 : (lt & 1);
-        const uint32_t acc_phase = p.m2 ? (uint32_t)(lt & 1) : (uint32_t)((lt >> 1) & 1);
+        const int acc = lt & 1;
+        const uint32_t acc_phase = (lt >> 1) & 1;
         if (!wait_bounded(tfull + acc, acc_phase, p.max_spins, abort)) { ok = false; break; }
         tc_fence_after();
         const int epi = (ch == 0 || tsum) ? p.epi : 2;
         const float alpha = p.epi == 0 ? 1.f : p.alpha;
         const bool last = ch == nch - 1;
-        for (int hh = 0; hh < nh; ++hh) {
-        const int64_t row0 = rowb + hh * BM;
-        const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * p.acc_stride +
-                               hh * p.block_n;
+        const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * p.acc_stride;
         for (int c = 0; c < p.block_n; c += 16) {
           float v[16];
           tmem_ld16(tbase + c, v);
@@ -541,11 +523,6 @@ __global__ void __launch_bounds__(NT, 1)
           }
           __syncwarp();
         }
-        // transposed store: this lane's row sum of squares over the tile, per half
-        if (last && p.c_trans && p.colsq && row0 + lane < p.M)
-          p.colsq[((int64_t)b * p.tiles_n + tile_ni(p, rem)) * p.M + row0 + lane] = rsq;
-        rsq = 0.f;
-        }  // halves
         if (tsum && !last) tmem_wait_st();  // the running sum is read back next chunk
         tc_fence_before();
         __syncwarp();
@@ -553,6 +530,8 @@ __global__ void __launch_bounds__(NT, 1)
         ++lt;
       }
       if (!ok) break;
+      if (p.c_trans && p.colsq && row0 + lane < p.M)
+        p.colsq[((int64_t)b * p.tiles_n + tile_ni(p, rem)) * p.M + row0 + lane] = rsq;
       if (p.devmax) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) dev = max_keep_nan(dev, __shfl_xor_sync(0xffffffffu, dev, o));
@@ -582,7 +561,7 @@ static uint32_t pow2_cols(uint32_t c) {
 template <bool A_MN, bool B_MN, int SPLIT>
 static cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, GemmP p,
                                cudaStream_t s) {
-  p.a_bytes = (p.m2 ? 2 : 1) * BM * BK * 2;
+  p.a_bytes = BM * BK * 2;
   p.b_bytes = (uint32_t)p.block_n * BK * 2;
   if (p.zplane_a == 0) p.zplane_a = p.batch;
   if (p.zplane_b == 0) p.zplane_b = p.batch;
@@ -595,7 +574,6 @@ static cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Gem
   // two accumulators, and with split operands over K chunks a third region for the
   // chunks' running sum
   p.tmem_cols = pow2_cols((SPLIT > 1 && p.kchunk > 0 ? 3 : 2) * p.block_n);
-  if (p.m2 && (!A_MN || SPLIT != 1 || p.kchunk > 0)) return cudaErrorInvalidValue;
   if (p.tmem_cols > 512) return cudaErrorInvalidValue;
   const size_t smem = 1024 + stages * stage_bytes + (2 * stages + 5) * 8 + 16 +
                       4 * 32 * EPI_LD * sizeof(float);
@@ -671,9 +649,7 @@ cudaError_t tc_gemm_btp(const void* Bg, const void* Pg, float* R, float* colsq, 
   p.M = r; p.N = n; p.K = m;
   p.batch = count;
   p.block_n = bn;
-  // r > 128: both 128-row halves of R^T in one CTA, each B stage read once for both
-  p.m2 = kBtpPairHalves && r > BM ? 1 : 0;
-  p.tiles_m = (int)((r + (p.m2 ? 2 * BM : BM) - 1) / (p.m2 ? 2 * BM : BM));
+  p.tiles_m = (int)((r + BM - 1) / BM);
   p.tiles_n = (int)((n + bn - 1) / bn);
   p.num_kb = (int)((m + BK - 1) / BK);
   p.idesc = idesc_bf16(BM, bn, true, true);
