@@ -332,7 +332,9 @@ int64_t dion_num_matrices(dion_handle h);
 int32_t dion_last_launch_count(dion_handle h);
 
 /* Intermediates of the most recent step, for inspection after the stream has
- * been synchronised: which = DION_VIEW_P gives P (fp32 [count, m, r]),
+ * been synchronised (DION_VIEW_P on the tensor path first rebuilds the fp32 P from
+ * the bf16 split the step keeps, with a kernel on the legacy default stream that the
+ * call waits for): which = DION_VIEW_P gives P (fp32 [count, m, r]),
  * DION_VIEW_R gives R (fp32 [count, n, r]), DION_VIEW_RMMC gives each matrix's
  * relative maximum momentum change (fp32 [count]).  *d_ptr points into d_workspace.
  *

@@ -546,8 +546,12 @@ dion_status run_bucket(StepCtx& c, int bi, int phase, const Plan& p, const dion_
       // the split's leading plane); the finalize then touches only the matrices that
       // took the second pass or the fallback
       __nv_bfloat16* P1s = split ? reinterpret_cast<__nv_bfloat16*>(Pg) : Ps;
-      e = dion::tc_apply(P0s, Linvs, P, P1s, nullptr, cnt, m, r, flags, 0, DION_MAT_FALLBACK,
-                         o.max_wait_spins, s, &nl, &done);
+      // only the split is written: every later reader of the first pass's P reads the
+      // split, and dion_workspace_view rebuilds the fp32 P from it (exactly: the three
+      // parts sum to the fp32 value); the matrices that take the second pass or the
+      // fallback get their fp32 P from the finalize
+      e = dion::tc_apply(P0s, Linvs, nullptr, P1s, nullptr, cnt, m, r, flags, 0,
+                         DION_MAT_FALLBACK, o.max_wait_spins, s, &nl, &done);
       if ((st = tc_check(e, "tc_apply")) != DION_OK) return st;
       pg_ready = true;
       if (o.orth_mode != DION_ORTH_CHOLQR) {
@@ -1353,7 +1357,7 @@ dion_status shard_continue(dion_handle h, dion_exchange* x) {
         __nv_bfloat16* P1s = o.precision == DION_PREC_BF16 ? b.Ps
                                                           : reinterpret_cast<__nv_bfloat16*>(b.Pg);
         auto ap = [&]() -> dion_status {
-          DION_TC(c, tc_apply(b.P0s, b.Linvs, b.P, P1s, nullptr, p.count, p.m, p.r, b.flags, 0,
+          DION_TC(c, tc_apply(b.P0s, b.Linvs, nullptr, P1s, nullptr, p.count, p.m, p.r, b.flags, 0,
                               DION_MAT_FALLBACK, o.max_wait_spins, c.s, &nl_, &done_),
                   "tc_apply");
           if (o.orth_mode != DION_ORTH_CHOLQR)
@@ -1550,6 +1554,21 @@ static dion_status dion_workspace_view_impl(dion_handle h, int32_t bucket, int32
   if (which == DION_VIEW_P) {
     *d_ptr = ws + p.off_P;
     *bytes = (size_t)p.count * p.m * p.r * 4;
+    // on the tensor path the first Cholesky-QR pass leaves P as its three-way split only:
+    // rebuild the fp32 P of the matrices that kept that pass (on the legacy stream, after
+    // the caller's synchronisation), and wait for it
+    if (h->opt.kernel_path == DION_PATH_TENSOR && h->opt.orth_mode != DION_ORTH_HOUSEHOLDER &&
+        h->last_launches > 0) {
+      const bool bf = h->opt.precision == DION_PREC_BF16;
+      const void* split = ws + (bf ? p.off_Ps : p.off_Pg);
+      cudaError_t e = dion::launch_p_from_split(reinterpret_cast<float*>(ws + p.off_P), split,
+                                                (int64_t)p.zplane * p.m * p.r,
+                                                reinterpret_cast<const int32_t*>(ws + p.off_flags),
+                                                p.count, p.m, p.r, 0);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(0);
+      if (e != cudaSuccess)
+        return fail(DION_ERR_CUDA, "rebuilding P from its split: %s", cudaGetErrorString(e));
+    }
   } else if (which == DION_VIEW_R) {
     *d_ptr = ws + p.off_R;
     *bytes = (size_t)p.count * p.n * p.r * 4;

@@ -79,6 +79,10 @@ cudaError_t launch_rows_from_full(const float* full, float* P, const int32_t* fl
                                   cudaStream_t s);
 cudaError_t launch_count_flags(const int32_t* flags, int count, int32_t mask, float* out,
                                cudaStream_t s);
+// P[b] = the sum of the three bf16 parts of Ps[b] (parts `plane` elements apart), for the
+// matrices that took neither the second pass nor the fallback.
+cudaError_t launch_p_from_split(float* P, const void* Ps, int64_t plane, const int32_t* flags,
+                                int count, int64_t m, int64_t r, cudaStream_t s);
 
 // ---- SIMT contractions (k_gemm_simt.cu)
 cudaError_t launch_gemm_simt(const GemmDesc& d, bool bf16_operands, cudaStream_t s);

@@ -312,6 +312,31 @@ cudaError_t launch_count_flags(const int32_t* flags, int count, int32_t mask, fl
   return cudaGetLastError();
 }
 
+// ------------------------------------------------ fp32 P from its split (inspection)
+// The first Cholesky-QR pass on the tensor path writes P only as its three-way bf16
+// split x0 + x1 + x2; each part is the rounding of what the earlier ones left, so the
+// fp32 sum (x0 + x1) + x2 is the fp32 P exactly.
+__global__ void k_p_from_split(float* __restrict__ P, const bf16* __restrict__ Ps, int64_t plane,
+                               const int32_t* __restrict__ flags, int64_t mr) {
+  const int64_t b = blockIdx.y;
+  if (flags[b] & (F_FALLBACK | F_CHOLQR2)) return;  // their fp32 P is the finalize's
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < mr;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = b * mr + e;
+    P[i] = (__bfloat162float(Ps[i]) + __bfloat162float(Ps[i + plane])) +
+           __bfloat162float(Ps[i + 2 * plane]);
+  }
+}
+
+cudaError_t launch_p_from_split(float* P, const void* Ps, int64_t plane, const int32_t* flags,
+                                int count, int64_t m, int64_t r, cudaStream_t s) {
+  int64_t gx = (m * r + 255) / 256;
+  if (gx > 64) gx = 64;
+  k_p_from_split<<<dim3((unsigned)gx, (unsigned)count), 256, 0, s>>>(P, (const bf16*)Ps, plane,
+                                                                      flags, m * r);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------- final P
 // P holds the first Cholesky-QR pass or the fallback's result; P2 the
 // second pass.  Picks per matrix, then writes the GEMM copy Pg (bf16 mode).
