@@ -230,8 +230,14 @@ dion_status fb_iteration(const Plan& p, const dion_options& o, const FbBufs& f,
   const int32_t skip = dion::F_SDONE | dion::F_SFAIL | DION_MAT_NONFINITE;
   int nl = 0;
   bool done = false;
+  // The iterate is exactly the previous one times R^-1 (an upper-triangular matrix with
+  // a positive diagonal) whatever R is, so the Gram's accuracy decides only how fast the
+  // iteration converges, not its limit: two split parts (three products, about 2^-17,
+  // far below the shift) serve, as they do for the second Cholesky-QR pass.  The test
+  // max|A^T A - I| <= orth_tol is then read to about 1e-5 (orth_tol is 2e-5 against a
+  // bound of 1e-4 on P).
   cudaError_t e = dion::tc_gram(src, f.W, f.Ws, nullptr, 0, p.count, p.m, p.r, f.flags, need, skip,
-                                o.max_wait_spins, s, &nl, &done);
+                                o.max_wait_spins, s, &nl, &done, 2);
   if (e != cudaSuccess || !done)
     return fail(DION_ERR_CUDA, "shifted iteration, Gram: %s",
                 e != cudaSuccess ? cudaGetErrorString(e) : dion::tc_map_error());
