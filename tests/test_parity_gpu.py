@@ -301,19 +301,21 @@ def test_deterministic_and_resumable():
         assert torch.equal(a.X[i], d.X[i]) and torch.equal(a.M[i], d.M[i])
 
 
+@pytest.mark.parametrize("stack_orth", [False, True])
 @pytest.mark.parametrize("precision", ["fp32", "bf16"])
-def test_step_from_host_equals_device_step(precision):
-    """The host-gradient entry point uploads bucket by bucket (largest first) and steps
-    each bucket as soon as its gradients arrive; over several steps, each overwriting G
-    that the previous step's update read, it gives bitwise the device step's state and
-    status.  The buckets are listed smallest first, so the upload order is not theirs;
-    r = 272 takes the recursive factorisation and the fallback graph."""
+def test_step_from_host_equals_device_step(precision, stack_orth):
+    """The host-gradient entry point uploads the buckets of one orthonormalisation stack
+    after another (the largest stack first) and steps a stack as soon as its gradients
+    have arrived; over several steps, each overwriting G that the previous step's update
+    read, it gives bitwise the device step's state and status.  The buckets are listed
+    smallest first, so the upload order is not theirs; r = 272 takes the recursive
+    factorisation and the fallback graph."""
     wl = W.custom("from_host", [(2, 256, 128, 32), (3, 600, 560, 272), (4, 1024, 512, 64),
                                 (1, 256, 64, 32)],
                   precision=precision, steps=3)
-    # the first and last bucket share an orthonormalisation stack
-    a = GpuRun(wl, stack_orth=True)
-    b = GpuRun(wl, stack_orth=True)
+    # with stack_orth the first and last bucket share an orthonormalisation stack
+    a = GpuRun(wl, stack_orth=stack_orth)
+    b = GpuRun(wl, stack_orth=stack_orth)
     nb = len(wl.buckets)
     host_status = torch.zeros(b.opt.num_matrices, dtype=torch.int32).pin_memory()
     for t in range(3):
