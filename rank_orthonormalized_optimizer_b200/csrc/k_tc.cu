@@ -184,6 +184,7 @@ struct GemmP {
   int c_trans;                       // store C transposed: C[j * ldc + i] (no Cs, Cb); colsq
                                      // then holds row sums of squares [batch][tiles_n][M]
   int m_fast;                        // tile order: M tiles of one N tile next to each other
+  int tiles_mat;                     // tiles per matrix as enumerated (set by the launcher)
   int32_t* flags;
   int32_t need_mask, skip_mask;      // matrices whose flags fail this are skipped
   int lower_only;                    // skip tiles above the diagonal (symmetric results)
@@ -220,11 +221,30 @@ __device__ __forceinline__ void k_range(const GemmP& p, int m0, int n0, int& kb0
   if (kb1 <= kb0) kb1 = kb0 + 1;  // never empty: a block past K loads as zeros
 }
 
-// M and N tile of tile rem within a matrix
+// row i of the lower triangle holding entry rem of its row-major enumeration:
+// i (i + 1) / 2 <= rem < (i + 1) (i + 2) / 2
+__device__ __forceinline__ int tri_row(int rem) {
+  int i = (int)((sqrtf(8.f * (float)rem + 1.f) - 1.f) * 0.5f);
+  while (i > 0 && i * (i + 1) / 2 > rem) --i;
+  while ((i + 1) * (i + 2) / 2 <= rem) ++i;
+  return i;
+}
+
+// M and N tile of tile rem within a matrix.  With a static tile schedule (tile t on CTA
+// t mod grid) the enumeration decides what each CTA gets: listing the tiles above the
+// diagonal of a symmetric result and skipping them left whole CTAs idle (grid and tiles
+// per matrix share factors), so with TRI those tiles are not enumerated at all.
+template <bool TRI = false>
 __device__ __forceinline__ int tile_mi(const GemmP& p, int rem) {
+  if constexpr (TRI) return tri_row(rem);
   return p.m_fast ? rem % p.tiles_m : rem / p.tiles_n;
 }
+template <bool TRI = false>
 __device__ __forceinline__ int tile_ni(const GemmP& p, int rem) {
+  if constexpr (TRI) {
+    const int i = tri_row(rem);
+    return rem - i * (i + 1) / 2;
+  }
   return p.m_fast ? rem / p.tiles_m : rem % p.tiles_n;
 }
 
@@ -238,10 +258,17 @@ __device__ __forceinline__ bool tile_active(const GemmP& p, int t, int tiles_per
   return (f & p.need_mask) == p.need_mask && !(f & p.skip_mask);
 }
 
-template <bool A_MN, bool B_MN, int SPLIT>
+// Epilogue and tile-order variants, fixed at compile time so that each instantiation
+// carries only its own code (the latency-bound long-K GEMMs are sensitive to it):
+constexpr int GM_DIRECT = 1;  // rows leave the epilogue straight from registers as
+                              // 16-byte vectors (no c_trans, no colsq; aligned C, Cb, Cs)
+constexpr int GM_TRI = 2;     // tiles enumerated over the lower triangle (square grid)
+
+template <bool A_MN, bool B_MN, int SPLIT, int MODE>
 __global__ void __launch_bounds__(NT, 1)
     k_tc_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const GemmP p) {
+  constexpr bool DIRECT = (MODE & GM_DIRECT) != 0, TRI = (MODE & GM_TRI) != 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t stage_a = SPLIT * p.a_bytes, stage_b = SPLIT * p.b_bytes;
@@ -257,7 +284,7 @@ __global__ void __launch_bounds__(NT, 1)
   float* escr = reinterpret_cast<float*>(tmem_slot + 4);  // 4 warps x [32][EPI_LD]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles_per_mat = p.tiles_m * p.tiles_n;
+  const int tiles_per_mat = TRI ? p.tiles_mat : p.tiles_m * p.tiles_n;
   const int ntiles = p.batch * tiles_per_mat;
 
   if (threadIdx.x == 0) {
@@ -293,8 +320,8 @@ __global__ void __launch_bounds__(NT, 1)
       if (!tile_active(p, t, tiles_per_mat)) continue;
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
-      const int m0 = tile_mi(p, rem) * BM;
-      const int n0 = tile_ni(p, rem) * p.block_n;
+      const int m0 = tile_mi<TRI>(p, rem) * BM;
+      const int n0 = tile_ni<TRI>(p, rem) * p.block_n;
       int kb0, kb1;
       k_range(p, m0, n0, kb0, kb1);
       bool ok = true;
@@ -349,7 +376,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (!tile_active(p, t, tiles_per_mat)) continue;
       const int rem = t % tiles_per_mat;
       int kb0, kb1;
-      k_range(p, tile_mi(p, rem) * BM, tile_ni(p, rem) * p.block_n, kb0, kb1);
+      k_range(p, tile_mi<TRI>(p, rem) * BM, tile_ni<TRI>(p, rem) * p.block_n, kb0, kb1);
       const int nch = n_chunks(p, kb0, kb1);
       for (int ch = 0; ch < nch && ok; ++ch) {
       const int acc = lt & 1;
@@ -406,10 +433,10 @@ __global__ void __launch_bounds__(NT, 1)
       if (!tile_active(p, t, tiles_per_mat)) continue;
       const int b = t / tiles_per_mat;
       const int rem = t % tiles_per_mat;
-      const int64_t row0 = (int64_t)tile_mi(p, rem) * BM + ew * 32;  // this warp's rows
-      const int64_t n0 = (int64_t)tile_ni(p, rem) * p.block_n;
+      const int64_t row0 = (int64_t)tile_mi<TRI>(p, rem) * BM + ew * 32;  // this warp's rows
+      const int64_t n0 = (int64_t)tile_ni<TRI>(p, rem) * p.block_n;
       int kb0, kb1;
-      k_range(p, tile_mi(p, rem) * BM, (int)n0, kb0, kb1);
+      k_range(p, tile_mi<TRI>(p, rem) * BM, (int)n0, kb0, kb1);
       float rsq = 0.f;  // transposed store: this lane's row sum of squares over the tile
       const int nch = n_chunks(p, kb0, kb1);
       // split operands: the chunks are added, in fp32 registers, into a running sum kept
@@ -444,6 +471,61 @@ __global__ void __launch_bounds__(NT, 1)
             continue;
           }
           if (n0 + c >= p.N) continue;  // uniform across the warp
+          if constexpr (DIRECT) {
+            // lane = row: its 16 consecutive columns go out as 16-byte vectors, with no
+            // pass through shared memory (a short-K GEMM such as the triangular apply is
+            // bound by this epilogue, not by its MMAs)
+            const int64_t row = row0 + lane;
+            if (row < p.M) {
+              const int64_t at = (int64_t)b * p.c_bs + row * p.ldc + n0 + c;
+              if (epi != 0) {
+                float o[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                  if (epi == 2) o4 = reinterpret_cast<const float4*>(p.C + at)[j];
+                  o[4 * j] = o4.x; o[4 * j + 1] = o4.y; o[4 * j + 2] = o4.z; o[4 * j + 3] = o4.w;
+                }
+#pragma unroll
+                for (int q = 0; q < 16; ++q) v[q] = epi == 2 ? fmaf(alpha, v[q], o[q]) : alpha * v[q];
+              }
+              if (p.C) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  reinterpret_cast<float4*>(p.C + at)[j] =
+                      make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+              }
+              if (last && p.Cb) {
+                __align__(16) bf16 h[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) h[q] = __float2bfloat16_rn(v[q]);
+                reinterpret_cast<uint4*>(p.Cb + at)[0] = reinterpret_cast<const uint4*>(h)[0];
+                reinterpret_cast<uint4*>(p.Cb + at)[1] = reinterpret_cast<const uint4*>(h)[1];
+              }
+              if (last && p.Cs) {
+                __align__(16) bf16 h[16], mi[16], lo[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) split3_bf16(v[q], h[q], mi[q], lo[q]);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                  reinterpret_cast<uint4*>(p.Cs + at)[j] = reinterpret_cast<const uint4*>(h)[j];
+                  reinterpret_cast<uint4*>(p.Cs + at + p.cs_stride)[j] =
+                      reinterpret_cast<const uint4*>(mi)[j];
+                  reinterpret_cast<uint4*>(p.Cs + at + 2 * p.cs_stride)[j] =
+                      reinterpret_cast<const uint4*>(lo)[j];
+                }
+              }
+              if (p.devmax && last) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                  const int64_t col = n0 + c + q;
+                  const float e = fabsf(v[q] - (col == row ? 1.f : 0.f));
+                  if (col <= row) dev = max_keep_nan(dev, e);
+                }
+              }
+            }
+            continue;
+          }
           if (p.c_trans) {
             // C[j][i]: for each column j the warp's 32 rows are 32 consecutive floats
             const int64_t row = row0 + lane;
@@ -516,7 +598,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
               for (int j = 0; j < 4; ++j) sq[j] += __shfl_xor_sync(0xffffffffu, sq[j], o);
             if (lane < 4) {
-              const int64_t rb = (int64_t)b * p.tiles_m * 4 + tile_mi(p, rem) * 4 + ew;
+              const int64_t rb = (int64_t)b * p.tiles_m * 4 + tile_mi<TRI>(p, rem) * 4 + ew;
               *reinterpret_cast<float4*>(p.colsq + rb * p.N + n0 + c + sub_c) =
                   make_float4(sq[0], sq[1], sq[2], sq[3]);
             }
@@ -531,7 +613,7 @@ __global__ void __launch_bounds__(NT, 1)
       }
       if (!ok) break;
       if (p.c_trans && p.colsq && row0 + lane < p.M)
-        p.colsq[((int64_t)b * p.tiles_n + tile_ni(p, rem)) * p.M + row0 + lane] = rsq;
+        p.colsq[((int64_t)b * p.tiles_n + tile_ni<TRI>(p, rem)) * p.M + row0 + lane] = rsq;
       if (p.devmax) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) dev = max_keep_nan(dev, __shfl_xor_sync(0xffffffffu, dev, o));
@@ -575,9 +657,26 @@ static cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Gem
   // chunks' running sum
   p.tmem_cols = pow2_cols((SPLIT > 1 && p.kchunk > 0 ? 3 : 2) * p.block_n);
   if (p.tmem_cols > 512) return cudaErrorInvalidValue;
+  // a symmetric result on a square grid of square tiles: enumerate the lower triangle
+  const bool tri = p.lower_only && p.tiles_m == p.tiles_n && p.block_n == BM;
+  // The direct epilogue pays where K is short (a tile's MMAs take less time than its
+  // epilogue, as in the triangular apply) and in the Gram (measured: 7 % faster); over
+  // a long K into a large result (B Q in split mode) the staged path's row-contiguous
+  // stores were faster.  16 columns of a row start on a 16-byte boundary in C (fp32), Cb
+  // and each part of Cs (bf16) when the pointers are 16-byte aligned and every offset is
+  // a multiple of 8.
+  auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  const bool direct = (p.num_kb <= 8 || tri) && !p.c_trans && !p.colsq && p.ldc % 8 == 0 &&
+                      p.c_bs % 8 == 0 && (!p.Cs || p.cs_stride % 8 == 0) && al16(p.C) &&
+                      al16(p.Cb) && al16(p.Cs) && p.block_n % 16 == 0;
+  if (tri) p.lower_only = 0;
+  p.tiles_mat = tri ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
   const size_t smem = 1024 + stages * stage_bytes + (2 * stages + 5) * 8 + 16 +
                       4 * 32 * EPI_LD * sizeof(float);
-  auto kern = k_tc_gemm<A_MN, B_MN, SPLIT>;
+  auto kern = tri ? (direct ? k_tc_gemm<A_MN, B_MN, SPLIT, GM_DIRECT | GM_TRI>
+                            : k_tc_gemm<A_MN, B_MN, SPLIT, GM_TRI>)
+                  : (direct ? k_tc_gemm<A_MN, B_MN, SPLIT, GM_DIRECT>
+                            : k_tc_gemm<A_MN, B_MN, SPLIT, 0>);
   // the device's limit rather than this launch's need: a launch captured into a graph
   // is checked against the attribute when the graph runs, after later launches of the
   // same kernel with other shapes may have set it
@@ -585,7 +684,7 @@ static cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Gem
                                        smem_optin());
   if (e != cudaSuccess) return e;
   if ((int)smem > smem_optin()) return cudaErrorInvalidValue;
-  const int ntiles = p.batch * p.tiles_m * p.tiles_n;
+  const int ntiles = p.batch * p.tiles_mat;
   const int grid = ntiles < sm_count() ? ntiles : sm_count();
   kern<<<grid, NT, smem, s>>>(ma, mb, p);
   return cudaGetLastError();
@@ -785,6 +884,10 @@ cudaError_t tc_apply(const bf16* Xs, const bf16* Ls, float* Y, bf16* Ys, bf16* Y
   p.Cb = Yb;
   p.flags = flags; p.need_mask = need; p.skip_mask = skip;
   p.kr = TC_KR_B_LOWER_NK;  // L^-1 is lower triangular: column tile j needs k <= j only
+  // column tiles have different K ranges: M-fast order spreads both kinds over every
+  // CTA of the static schedule (N-fast with two column tiles and an even grid gave one
+  // CTA in two only the long ones)
+  p.m_fast = 1;
   p.max_spins = max_spins;
   cudaError_t e = launch_gemm<false, false, 3>(ma, mb, p, s);
   if (e == cudaSuccess) { *done = true; *nlaunch = 1; }
@@ -825,6 +928,7 @@ cudaError_t tc_block_gemm(const TcBlockGemm& g, int count, int64_t r, int32_t* f
   p.epi = g.accumulate ? 2 : 1;
   p.alpha = g.alpha;
   p.kr = g.kr;
+  p.m_fast = g.kr != 0;  // uneven K ranges by tile: mix them over the CTAs
   if (g.accumulate) p.kchunk = KCHUNK_SUMSQ;  // W22 -= L21 L21^T: squares on the diagonal
   p.max_spins = max_spins;
   cudaError_t e;
