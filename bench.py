@@ -347,7 +347,8 @@ def run_ours(args):
 
     wl = W.WORKLOADS[args.workload]
     opt = DionB200([(b.count, b.m, b.n, b.r) for b in wl.buckets], mu=wl.mu,
-                   precision=wl.precision, kernel_path=args.kernel_path)
+                   precision=wl.precision, kernel_path=args.kernel_path,
+                   stack_orth=args.stack_orth)
     nb = len(wl.buckets)
     X = [W.weights(wl, i, dev) for i in range(nb)]
     M = [W.momentum(wl, i, dev) for i in range(nb)]
@@ -403,7 +404,7 @@ def run_ours(args):
                    "params_per_gpu": wl.params,
                    "buckets": [[b.count, b.m, b.n, b.r] for b in wl.buckets],
                    "state": "fp32 X, M, G, Q", "gemm_inputs": wl.precision,
-                   "kernel_path": args.kernel_path,
+                   "kernel_path": args.kernel_path, "stack_orth": bool(args.stack_orth),
                    "parallelism": f"matrix-partitioned x{world} (each rank its own matrices)",
                    "l2": l2_note(wl)},
         "roofline": {"bound": "hbm", "kernel": "fused update (M and X)",
@@ -691,6 +692,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE, choices=sorted(W.WORKLOADS))
     ap.add_argument("--kernel-path", default="tensor", choices=["tensor", "simt"])
+    ap.add_argument("--stack-orth", action="store_true",
+                    help="one orthonormalisation stack per (m, r) across buckets")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
