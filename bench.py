@@ -606,7 +606,7 @@ def measure_vector_step(dev, stream, peaks, warmup=3, iters=10,
             gbs = VEC_BYTES[rule] * n / (ms * 1e-3) / 1e9
             r = {"us": ms * 1e3, "launches_per_step": launches // reps,
                  "bytes_per_element": VEC_BYTES[rule], "achieved_GBs": gbs,
-                 "frac_of_measured_copy": gbs / peaks["hbm_gbs"]}
+                 "frac_of_copy_peak": gbs / peaks["hbm_gbs"], "peak_source": peaks["source"]}
             if not big:
                 # the same calls with the host ahead of the device: a bounded spin kernel
                 # (about 20 ms) holds the stream while every call is enqueued, so the
