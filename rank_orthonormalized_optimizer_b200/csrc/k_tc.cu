@@ -19,6 +19,13 @@
 //   acc = P [R | Q]^T per 128 x 128 tile (one N = 256 MMA), then
 //   M <- (M + G) - (1 - mu) acc_R,  X <- X - lr s acc_Q, with M, G, X streamed
 //   through shared memory by TMA in 128 x 32 slabs and M, X stored by TMA.
+// formb_bq (steps 1 and 2 fused): B = M + G converted in shared memory and fed to
+//   the MMA of B Q, with its own warp roles (described where it is defined).
+// The same gemm kernel, with operands split into three bf16 parts, runs the
+// orthonormalisation's contractions: the Gram P0^T P0, the triangular apply P0 L^-T
+// and the block products of the recursive factorisation.  Its epilogue and tile order
+// come in variants fixed at compile time (a direct epilogue for short-K tiles, the
+// lower triangle only for symmetric results), so that each launch carries only its own.
 #include <cuda.h>
 
 #include <cstdio>
