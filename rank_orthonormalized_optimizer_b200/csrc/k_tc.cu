@@ -667,7 +667,7 @@ static cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Gem
   // a symmetric result on a square grid of square tiles: enumerate the lower triangle
   const bool tri = p.lower_only && p.tiles_m == p.tiles_n && p.block_n == BM;
   // The direct epilogue pays where K is short (a tile's MMAs take less time than its
-  // epilogue, as in the triangular apply) and in the Gram (measured: 7 % faster); over
+  // epilogue, as in the triangular apply) and in the Grams (measured: 2-7 % faster); over
   // a long K into a large result (B Q in split mode) the staged path's row-contiguous
   // stores were faster.  16 columns of a row start on a 16-byte boundary in C (fp32), Cb
   // and each part of Cs (bf16) when the pointers are 16-byte aligned and every offset is
