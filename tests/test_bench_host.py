@@ -113,3 +113,25 @@ def test_split_ceiling_of_the_rank_sweep():
     assert f == 8 * (36 * m * n * r + 18 * m * r * r + r ** 3 / 3)
     assert b == 8 * (40 * m * n + 4 * (3 * m * r + 6 * n * r))
     assert t == f / 1672e12 and f / 1672e12 > b / 6458.1e9
+
+
+def test_update_traffic_comes_from_captures_of_this_kernel():
+    """The per-shape DRAM figures behind `roofline.traffic` were captured on the update
+    kernel as committed (its source hash), each figure is read + write over elements of
+    its capture, and the 7B-like step's traffic per launch is their element-weighted
+    mean over the three launches."""
+    per, h = bench.update_traffic()
+    assert per is not None and h == bench.update_kernel_hash()
+    caps = json.load(open(bench.TRAFFIC_FILE))["captures"]
+    for shape, c in caps.items():
+        assert abs(per[shape] - (c["dram_read"] + c["dram_write"]) / c["elements"]) < 1e-9
+    wl = W.WORKLOADS[W.HEADLINE]
+    want = sum(per[f"{b.m}x{b.n}"] * b.params for b in wl.buckets) / len(wl.buckets)
+    assert bench.update_traffic_per_launch(wl, len(wl.buckets)) == pytest.approx(want)
+    assert 20.0 * wl.params / 3 <= want <= 21.0 * wl.params / 3
+
+
+def test_update_traffic_is_null_once_the_kernel_changes(monkeypatch):
+    wl = W.WORKLOADS[W.HEADLINE]
+    monkeypatch.setattr(bench, "update_kernel_hash", lambda: "0" * 16)
+    assert bench.update_traffic_per_launch(wl, 3) is None
